@@ -1,0 +1,193 @@
+"""Pins of the oracle's attention path (CPU only).
+
+Independent references: the transformers Llama RoPE helper, torch's
+scaled-dot-product attention in fp64 on fully materialised keys/values,
+dense attention with W_k = A_k B_k / W_v = A_v B_v, the softmax partition
+identity, and closed-form special cases.
+"""
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+from transformers.models.llama.modeling_llama import apply_rotary_pos_emb
+
+import oracle as O
+from harness import gen
+
+
+def hf_rope(x, pos, base):
+    """RoPE via transformers' Llama helper (rotate_half convention), fp64."""
+    x = torch.as_tensor(np.asarray(x, np.float64))          # [n, d]
+    d = x.shape[-1]
+    inv = 1.0 / (base ** (torch.arange(0, d, 2, dtype=torch.float64) / d))
+    fr = torch.as_tensor(np.asarray(pos, np.float64))[:, None] * inv[None]
+    emb = torch.cat([fr, fr], -1)
+    cos, sin = emb.cos()[None], emb.sin()[None]           # [1, n, d]
+    q, _ = apply_rotary_pos_emb(x[None, None], x[None, None], cos, sin)
+    return q[0, 0].numpy()
+
+
+@pytest.mark.parametrize("d,base", [(64, 1e4), (128, 1e4), (128, 5e5)])
+def test_rope_matches_transformers(d, base):
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((50, d))
+    pos = rng.integers(0, 40000, 50)
+    # the two ways of forming base^(-2i/d) differ by a few fp64 ulp; times a
+    # position up to 4e4 that moves the angle by ~1e-11 rad
+    np.testing.assert_allclose(O.rope(x, pos, base), hf_rope(x, pos, base), atol=1e-10, rtol=0)
+
+
+def test_rope_shift_invariance():
+    rng = np.random.default_rng(1)
+    q, k = rng.standard_normal((1, 128)), rng.standard_normal((30, 128))
+    pk = np.arange(30)
+    s0 = O.rope(k, pk, 1e4) @ O.rope(q, [29], 1e4)[0]
+    s1 = O.rope(k, pk + 12345, 1e4) @ O.rope(q, [29 + 12345], 1e4)[0]
+    np.testing.assert_allclose(s0, s1, atol=1e-10)
+
+
+def _rand_case(H=4, h_kv=2, d=64, r_k=16, R=64, n=37, seed=0, m=1):
+    rng = np.random.default_rng(seed)
+    cfg = O.Config(H=H, h_kv=h_kv, d_h=d, hidden=8, r_k=r_k, R=R)
+    zk = rng.standard_normal((n, h_kv, r_k))
+    zv = rng.standard_normal((n, R))
+    Bk = rng.standard_normal((h_kv, r_k, d)) / np.sqrt(r_k)
+    Bv = rng.standard_normal((R, h_kv * d)) / np.sqrt(R)
+    q = rng.standard_normal((m, H, d))
+    return cfg, zk, zv, Bk, Bv, q
+
+
+def _sdpa_materialised(cfg, zk, zv, Bk, Bv, q, q_pos):
+    """Brute force: decompress the full K (RoPE'd) and V per head, then SDPA."""
+    n = zk.shape[0]
+    d = cfg.d_h
+    K = np.stack([hf_rope(zk[:, kv] @ Bk[kv], np.arange(n), cfg.rope_base) for kv in range(cfg.h_kv)])
+    V = np.stack([zv @ Bv[:, kv * d:(kv + 1) * d] for kv in range(cfg.h_kv)])
+    Q = np.stack([hf_rope(q[:, h], q_pos, cfg.rope_base) for h in range(cfg.H)])      # [H, m, d]
+    mask = torch.as_tensor(np.arange(n)[None, :] <= np.asarray(q_pos)[:, None])
+    o = F.scaled_dot_product_attention(torch.as_tensor(Q)[None], torch.as_tensor(K)[None],
+                                       torch.as_tensor(V)[None], attn_mask=mask,
+                                       enable_gqa=cfg.H != cfg.h_kv)
+    return o[0].numpy().transpose(1, 0, 2)                                           # [m, H, d]
+
+
+@pytest.mark.parametrize("H,h_kv", [(4, 4), (8, 2)])
+def test_reassociated_equals_materialised(H, h_kv):
+    # [Review] eq. 12: p_h (Z_V U_h^T) = (p_h Z_V) U_h^T, plus GQA head mapping
+    cfg, zk, zv, Bk, Bv, q = _rand_case(H=H, h_kv=h_kv, m=5, n=70)
+    q_pos = np.array([69, 3, 40, 0, 69])
+    got = O.attend_latents(cfg, zk, zv, q, q_pos, Bk, Bv)
+    ref = _sdpa_materialised(cfg, zk, zv, Bk, Bv, q, q_pos)
+    np.testing.assert_allclose(got, ref, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("rotate", [False, True])
+def test_full_rank_latents_reproduce_dense_attention(rotate):
+    # r_k = d_h, R = h_kv d_h, orthonormal B: latent attention == dense attention
+    # with W_k = A_k B_k, W_v = A_v B_v; the block rotation (eq. 13) changes nothing.
+    rng = np.random.default_rng(7)
+    H, h_kv, d, hidden, n = 4, 2, 32, 48, 25
+    cfg = O.Config(H=H, h_kv=h_kv, d_h=d, hidden=hidden, r_k=d, R=h_kv * d)
+    X = rng.standard_normal((n, hidden))
+    A_k = rng.standard_normal((hidden, h_kv * d)) / np.sqrt(hidden)
+    A_v = rng.standard_normal((hidden, h_kv * d)) / np.sqrt(hidden)
+    Bk = np.stack([np.linalg.qr(rng.standard_normal((d, d)))[0].T for _ in range(h_kv)])
+    Bv = np.linalg.qr(rng.standard_normal((h_kv * d, h_kv * d)))[0].T
+    q = rng.standard_normal((1, H, d))
+    zk = (X @ A_k).reshape(n, h_kv, d)
+    zv = X @ A_v
+    if rotate:
+        g = cfg.key.g
+        zk = O.unrotate_fp64(zk.reshape(n, -1) @ np.kron(np.eye(h_kv * d // g), O.hadamard_fp64(g)), g).reshape(n, h_kv, d)
+        zv = O.unrotate_fp64(zv @ np.kron(np.eye(h_kv * d // cfg.val.g), O.hadamard_fp64(cfg.val.g)), cfg.val.g)
+    got = O.attend_latents(cfg, zk, zv, q, [n - 1], Bk, Bv)
+    Wk = [A_k[:, kv * d:(kv + 1) * d] @ Bk[kv] for kv in range(h_kv)]
+    Wv = A_v @ Bv
+    K = np.stack([hf_rope(X @ Wk[kv], np.arange(n), cfg.rope_base) for kv in range(h_kv)])
+    V = np.stack([X @ Wv[:, kv * d:(kv + 1) * d] for kv in range(h_kv)])
+    Q = np.stack([hf_rope(q[:, h], [n - 1], cfg.rope_base) for h in range(H)])
+    o = F.scaled_dot_product_attention(torch.as_tensor(Q)[None], torch.as_tensor(K)[None],
+                                       torch.as_tensor(V)[None], enable_gqa=True)[0].numpy()
+    np.testing.assert_allclose(got, o.transpose(1, 0, 2), atol=1e-12, rtol=0)
+
+
+def test_partition_identity_merge():
+    # [CaliDrop] eq. 1: Att over a partition = alpha-weighted sum of subset attentions
+    rng = np.random.default_rng(8)
+    s = rng.standard_normal(1000) * 4
+    v = rng.standard_normal((1000, 33))
+    p = np.exp(s - s.max())
+    ref = p @ v / p.sum()
+    for cuts in ([], [1], [500], [3, 3, 999], sorted(rng.choice(999, 7, replace=False) + 1)):
+        b = [0] + list(cuts) + [1000]
+        parts = [O.partial_softmax(s[lo:hi], v[lo:hi]) for lo, hi in zip(b[:-1], b[1:])]
+        np.testing.assert_allclose(O.lse_merge(parts), ref, atol=1e-13, rtol=0)
+
+
+def test_single_token_returns_its_value():
+    cfg, zk, zv, Bk, Bv, q = _rand_case(n=1)
+    got = O.attend_latents(cfg, zk, zv, q, [0], Bk, Bv)
+    for h in range(cfg.H):
+        kv = h // cfg.group
+        np.testing.assert_allclose(got[0, h], zv[0] @ Bv[:, kv * 64:(kv + 1) * 64], atol=1e-13)
+
+
+def test_identical_keys_average_values():
+    cfg, zk, zv, Bk, Bv, q = _rand_case(n=20)
+    # identical *pre-RoPE* keys still differ after RoPE; take d_h-invariant keys: zero keys
+    zk[:] = 0.0
+    got = O.attend_latents(cfg, zk, zv, q, [19], Bk, Bv)
+    for h in range(cfg.H):
+        kv = h // cfg.group
+        np.testing.assert_allclose(got[0, h], zv.mean(0) @ Bv[:, kv * 64:(kv + 1) * 64], atol=1e-13)
+
+
+def test_decode_through_paged_cache_equals_direct():
+    # gather through a shuffled block table == dequantising the pages in order
+    w = gen.shrink(gen.workload(0), ctx=77)
+    cfg = O.config_of(w)
+    f = gen.make_factors(w)
+    zk, zv = gen.make_latents(w, 77)
+    bt, n_pages = gen.make_block_table([77], extra_pages=3)
+    cache = O.new_cache(cfg, n_pages)
+    O.write_latents(cache, gen.slots_for(bt, 0, np.arange(77)), zk, zv)
+    q = gen.make_queries(1, w.H, w.d_h)
+    got = O.decode(cache, q, f.B_k, f.B_v, bt, [77])
+    ck = [O.quantize_latent(zk[:, h], cfg.key) for h in range(cfg.h_kv)]
+    zkh = np.stack([O.dequantize_codes(*c, cfg.key) for c in ck], 1)
+    zvh = O.dequantize_codes(*O.quantize_latent(zv, cfg.val), cfg.val)
+    ref = _sdpa_materialised(cfg, O.unrotate_fp64(zkh, cfg.key.g), O.unrotate_fp64(zvh, cfg.val.g),
+                             f.B_k.astype(np.float64), f.B_v.astype(np.float64), q.astype(np.float64), [76])
+    np.testing.assert_allclose(got, ref, atol=1e-12, rtol=0)
+
+
+def test_prefill_is_causal_decode_per_query():
+    # each prefill query equals a decode whose sequence ends at that query
+    w = gen.shrink(gen.workload(0), ctx=50)
+    cfg = O.config_of(w)
+    f = gen.make_factors(w)
+    zk, zv = gen.make_latents(w, 50)
+    bt, n_pages = gen.make_block_table([50])
+    cache = O.new_cache(cfg, n_pages)
+    O.write_latents(cache, gen.slots_for(bt, 0, np.arange(50)), zk, zv)
+    q = gen.make_queries(9, w.H, w.d_h)
+    got = O.prefill(cache, q, [0, 9], f.B_k, f.B_v, bt, [50])
+    for i in range(9):
+        d = O.decode(cache, q[i:i + 1], f.B_k, f.B_v, bt, [42 + i])   # query at 41 + i
+        np.testing.assert_allclose(got[i], d[0], atol=1e-13)
+
+
+def test_quantised_attention_close_to_unquantised():
+    # sanity: 4/3-bit latents perturb the output a little, not grossly
+    w = gen.shrink(gen.workload(0), ctx=256)
+    cfg = O.config_of(w)
+    f = gen.make_factors(w)
+    zk, zv = gen.make_latents(w, 256)
+    bt, n_pages = gen.make_block_table([256])
+    cache = O.new_cache(cfg, n_pages)
+    O.write_latents(cache, gen.slots_for(bt, 0, np.arange(256)), zk, zv)
+    q = gen.make_queries(1, w.H, w.d_h)
+    got = O.decode(cache, q, f.B_k, f.B_v, bt, [256])
+    ref = O.attend_latents(cfg, zk, zv, q, [255], f.B_k, f.B_v)
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel < 0.2

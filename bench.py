@@ -1,0 +1,424 @@
+"""Benchmark: decode context-tokens/s and achieved HBM GB/s of STAR-KV latent-cache attention.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl starkv|reference] [--workload NAME]
+
+One step = one pass of the decode hot path over one batch: append one new token
+per sequence (project, rotate, quantise, pack) and then batched single-query
+attention over the packed cache (dequantise, re-expand and RoPE keys, online
+softmax, P Z_v in the latent, split merge, B_v projection).  Default workload:
+LongChat-7B-shaped layer, 32 heads, d_h 128, r_k 32, R 1024, batch 16, context
+4096, 16-token pages.  Inputs are seeded and synthetic (no weights or datasets).
+
+For N > 1 (torchrun), every rank runs its own batch of independent sequences
+(weak scaling, no collective on the data path); the timing is the maximum over
+ranks.  The reference arm times the fp64 CPU oracle on a bounded sample of the
+same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from harness import gen  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (timing only; no data-path collective)
+# ---------------------------------------------------------------------------
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def shard_sequences(batch: int, rank: int, world: int, scaling: str = "weak"):
+    """Sequences owned by `rank`: weak scaling gives every rank its own full batch."""
+    if scaling == "weak":
+        return list(range(batch)), rank
+    per = (batch + world - 1) // world
+    return list(range(rank * per, min(batch, (rank + 1) * per))), 0
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            p = [x.strip() for x in l.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx.append(float(p[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# workload state on the GPU
+# ---------------------------------------------------------------------------
+def bytes_per_token(w) -> int:
+    """Packed cache bytes per token from the library's own layout query."""
+    from rank_mixed_precision_b200 import starkv as S
+    cfg = S.make_config(w.H, w.h_kv, w.d_h, w.hidden, w.r_k, w.R, 16, w.top_fraction, w.rope_base)
+    sz = S.starkv_cache_layout(cfg, 1)
+    return (sz["k_codes_bytes"] + sz["v_codes_bytes"] + sz["k_meta_bytes"] + sz["v_meta_bytes"]) // 16
+
+
+def decode_algorithmic_bytes(w, total_tokens: int, batch: int, max_pages: int) -> int:
+    """What one decode call must move once: packed payload + metadata of every
+    attended token, the bf16 up-projections B_k and B_v, q, out, block table and lengths."""
+    factors = 2 * (w.h_kv * w.r_k * w.d_h + w.R * w.h_kv * w.d_h)
+    io = 2 * 2 * batch * w.H * w.d_h + 4 * batch * max_pages + 4 * batch
+    return total_tokens * bytes_per_token(w) + factors + io
+
+
+class DecodeState:
+    def __init__(self, w, seed, device, replicas):
+        import torch
+        from rank_mixed_precision_b200 import starkv as S
+        self.S = S
+        self.w = w
+        bf = lambda a: torch.from_numpy(gen.bf16_bits(a).view(np.int16).copy()).view(torch.bfloat16).to(device)
+        f = gen.make_factors(w, seed)
+        self.seq_lens = gen.make_seq_lens(w, seed)
+        B = w.batch
+        mp = int(self.seq_lens.max()) + 16
+        cfg = S.make_config(w.H, w.h_kv, w.d_h, w.hidden, w.r_k, w.R, mp, w.top_fraction, w.rope_base)
+        self.kv = S.StarKV(cfg, bf(f.A_k), bf(f.A_v), bf(f.B_k), bf(f.B_v))
+        bt, n_pages = gen.make_block_table(self.seq_lens, seed)
+        self.bt_np = bt
+        self.max_pages = bt.shape[1]
+        self.n_pages = n_pages
+        # fill the context [0, L-1) of every sequence with the library's own append
+        self.caches = [self.kv.new_cache(n_pages) for _ in range(replicas)]
+        chunk = 4096
+        for b in range(B):
+            L = int(self.seq_lens[b])
+            for s0 in range(0, L - 1, chunk):
+                n = min(chunk, L - 1 - s0)
+                X = bf(gen.make_hidden(n, w.hidden, seed, name="X", sub=1000 * b + s0 // chunk))
+                slots = torch.from_numpy(gen.slots_for(bt, b, np.arange(s0, s0 + n))).to(device)
+                self.kv.append(self.caches[0], X, slots)
+        torch.cuda.synchronize()
+        for c in self.caches[1:]:
+            for name in ("k_codes", "v_codes", "k_meta", "v_meta"):
+                getattr(c, name).copy_(getattr(self.caches[0], name))
+        # per-step inputs: one new token per sequence at position L-1, its query
+        self.X_np = gen.make_hidden(B, w.hidden, seed, name="X_step")
+        self.q_np = gen.make_queries(B, w.H, w.d_h, seed, name="q_step")
+        self.slots_np = np.array([gen.slots_for(bt, b, [int(self.seq_lens[b]) - 1])[0] for b in range(B)],
+                                 np.int64)
+        self.X = bf(self.X_np)
+        self.q = bf(self.q_np)
+        self.slots = torch.from_numpy(self.slots_np).to(device)
+        self.bt = torch.from_numpy(bt).to(device)
+        self.sl = torch.from_numpy(self.seq_lens.astype(np.int32)).to(device)
+        self.out = torch.empty_like(self.q)
+        self.ws = self.kv.workspace(S.OP_DECODE, B, self.max_pages)
+        st = self.kv.status()
+        if st:
+            raise RuntimeError(f"device status {st:#x} after cache fill")
+
+    def step(self, i, ev=None):
+        S = self.S
+        c = self.caches[i % len(self.caches)]
+        S.starkv_append(self.kv.ctx, c.struct, self.X, self.slots)
+        if ev is not None:
+            ev[0].record()
+        S.starkv_decode_attn(self.kv.ctx, c.struct, self.q, self.bt, self.sl, self.out, self.ws)
+        if ev is not None:
+            ev[1].record()
+
+
+def run_starkv(args, w, rank, world, local):
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    replicas = max(1, int(np.ceil(3 * L2_BYTES / max(1, w.batch * w.ctx * bytes_per_token(w)))))
+    replicas = max(replicas, 2)
+    st = DecodeState(w, args.seed, device, replicas)
+    S = st.S
+    launches_per_step = 3  # append, decode split, decode merge
+    for i in range(args.warmup):
+        st.step(i)
+    torch.cuda.synchronize()
+    # ---- device-resident timed region
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record()
+        for i in range(args.steps):
+            st.step(i, pairs[i])
+        t1.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = t0.elapsed_time(t1)
+    dec_ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+    status = st.kv.status()
+    if status:
+        raise RuntimeError(f"device status {status:#x} during the timed region")
+    ms_max = max_over_ranks(ms, world, device)
+    tokens_per_step = int(st.seq_lens.sum())
+    value = tokens_per_step * args.steps * world / (ms_max / 1e3)
+    # ---- end to end through the public API with host buffers
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    Xh = pin(gen.bf16_bits(st.X_np).view(np.int16)).view(torch.bfloat16)
+    qh = pin(gen.bf16_bits(st.q_np).view(np.int16)).view(torch.bfloat16)
+    slh, bth, lh = pin(st.slots_np), pin(st.bt_np), pin(st.seq_lens.astype(np.int32))
+    outh = torch.empty(st.q.shape, dtype=torch.bfloat16).pin_memory()
+    Xd, qd, sld, btd, ld = (torch.empty_like(t, device=device) for t in (Xh, qh, slh, bth, lh))
+    h2d = sum(t.numel() * t.element_size() for t in (Xh, qh, slh, bth, lh))
+    d2h = outh.numel() * outh.element_size()
+
+    def e2e_step(i):
+        for d, h in ((Xd, Xh), (qd, qh), (sld, slh), (btd, bth), (ld, lh)):
+            d.copy_(h, non_blocking=True)
+        c = st.caches[i % len(st.caches)]
+        S.starkv_append(st.kv.ctx, c.struct, Xd, sld)
+        S.starkv_decode_attn(st.kv.ctx, c.struct, qd, btd, ld, st.out, st.ws)
+        outh.copy_(st.out, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    e2e_value = tokens_per_step * args.steps * world / (e2e_ms / 1e3)
+
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peaks()
+    alg = decode_algorithmic_bytes(w, tokens_per_step, w.batch, st.max_pages)
+    achieved = alg / (dec_ms / 1e3) / 1e9
+    line = {
+        "metric": "decode context-tokens/s",
+        "value": value,
+        "unit": "context-tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp32",
+        "data": "synthetic (seeded; shapes of the named model, no weights)",
+        "config": {"workload": w.name, "batch": w.batch, "ctx": int(st.seq_lens.max()),
+                   "heads": w.H, "kv_heads": w.h_kv, "head_dim": w.d_h, "rank_k": w.r_k, "rank_v": w.R,
+                   "bits": "4/3 (top 25% of channels 4-bit)", "page_tokens": 16,
+                   "step": "append 1 token per sequence + decode attention",
+                   "parallelism": f"dp{world} (independent sequences per GPU)",
+                   "l2": f"{len(st.caches)} rotating cache replicas "
+                         f"({len(st.caches) * st.caches[0].nbytes() / 2**20:.0f} MiB > 126 MiB L2)"},
+        "roofline": {"bound": "hbm", "kernel": "starkv_decode_attn (split + merge)",
+                     "achieved": achieved, "peak": peak, "peak_kind": f"hbm copy GB/s ({peak_kind})",
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_bytes_per_launch": alg, "launch_ms": dec_ms,
+                     "achieved_context_tokens_per_s_decode_only": tokens_per_step / (dec_ms / 1e3)},
+        "e2e": {"value": e2e_value, "unit": "context-tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.seed, args.cpu_seconds)
+    return line
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------
+def _oracle_setup(w, seed, b):
+    import oracle as O
+    cfg = O.config_of(w)
+    L = int(gen.make_seq_lens(w, seed)[b])
+    bt, n_pages = gen.make_block_table([L], seed)
+    oc = O.new_cache(cfg, n_pages)
+    zk, zv = gen.make_latents(w, L, seed, sub=b)
+    O.write_latents(oc, gen.slots_for(bt, 0, np.arange(L)), zk, zv)
+    f = gen.make_factors(w, seed)
+    q = gen.make_queries(1, w.H, w.d_h, seed, name="q_step", sub=b)
+    return O, oc, bt, L, f, q
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline(w, seed, seconds):
+    O, oc, bt, L, f, q = _oracle_setup(w, seed, 0)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        O.decode(oc, q, f.B_k, f.B_v, bt, [L])
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": done * L / el, "unit": "context-tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{done} oracle decode call(s) of one {L}-token sequence, all {w.H} heads, "
+                      f"fp64 numpy, {el:.1f} s", "host_cpu_count": os.cpu_count()}
+
+
+def run_reference(args, w, rank, world):
+    """The fp64 CPU oracle on the same workload; each step is a bounded sample:
+    one sequence of the batch and a subset of its heads, sized so the whole run
+    stays within a few minutes."""
+    if rank != 0:
+        return None
+    O, oc, bt, L, f, q = _oracle_setup(w, args.seed, 0)
+    t0 = time.perf_counter()
+    O.decode(oc, q, f.B_k, f.B_v, bt, [L])
+    t_full = time.perf_counter() - t0
+    budget = 150.0
+    heads = max(1, min(w.H, int(w.H * budget / max(1e-9, args.steps * t_full))))
+    hs = list(range(heads))
+    for _ in range(min(args.warmup, 1)):
+        O.decode(oc, q, f.B_k, f.B_v, bt, [L], heads=hs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.decode(oc, q, f.B_k, f.B_v, bt, [L], heads=hs)
+    el = time.perf_counter() - t0
+    v = args.steps * L * (heads / w.H) / el
+    sample = f"each step: one {L}-token sequence, {heads} of {w.H} heads (counted as {heads}/{w.H} of its tokens)"
+    return {
+        "metric": "decode context-tokens/s", "value": v, "unit": "context-tokens/s", "impl": "reference",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "batch": w.batch, "ctx": w.ctx, "sample": sample},
+        "cpu_baseline": {"value": v, "unit": "context-tokens/s", "cores": _blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": "context-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="starkv", choices=["starkv", "reference"])
+    ap.add_argument("--workload", default="longchat7b_decode_b16_t4096")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "starkv":
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_env()
+    w = gen.workload(args.workload)
+    if args.impl == "reference":
+        line = run_reference(args, w, rank, world)
+    else:
+        line = run_starkv(args, w, rank, world, local)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,254 @@
+/*
+ * starkv.h -- C ABI of the STAR-KV latent-cache attention library (B200, sm_100a).
+ *
+ * The library computes attention directly on a low-rank, mixed-precision
+ * latent KV cache, following the decode dataflow of "STAR-KV: Learning the
+ * Rank Is Only Half of KV Cache Compression" (technical review of arXiv
+ * 2606.08382), Algorithm 2 "Consume a compressed cache during decoding":
+ *
+ *   keys   : one pre-RoPE latent per KV head, z_k,h (rank r_k), re-expanded
+ *            by B_k,h (r_k x d_h) inside the attention kernel, then RoPE'd
+ *            (section 5.3, "Keys are harder");
+ *   values : one joint latent z_v (rank R) shared by all heads; probabilities
+ *            of all heads multiply it first and B_v (R x h_kv d_h) is applied
+ *            afterwards (section 5.3, eq. 12 and the stacked P Z_V product);
+ *   storage: latents are Hadamard-rotated in groups (section 6.1, eq. 13) and
+ *            quantised 4-bit for the leading (outlier) channels and 3-bit for
+ *            the rest (eq. 14), with an fp16 scale and zero per group.
+ *
+ * Conventions for every entry point
+ *   - Pointers named "device" are CUDA device memory owned by the caller;
+ *     "host" pointers are CPU memory.  The library keeps no pointer to caller
+ *     memory after a call returns, except that work queued on `stream` reads
+ *     and writes it asynchronously: keep buffers alive until the stream has
+ *     passed the work.
+ *   - All compute is queued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and returns before it finishes.  Nothing throws; every function
+ *     returns a starkv_status, and starkv_last_error() gives the calling
+ *     thread's last message.
+ *   - Arguments are checked on the host before anything is launched.  Faults
+ *     that only the data can show (an out-of-range page id in a block table, a
+ *     sequence longer than its pages, a latent whose fp16 scale overflows) set
+ *     bits in a device status word owned by the context; the affected work is
+ *     skipped (its output is written as zeros) and the word is read with
+ *     starkv_read_device_status().
+ *
+ * Data types: "bf16" = IEEE bfloat16 bit patterns (uint16), "fp16" = IEEE
+ * binary16, "fp32" = IEEE binary32.  Arrays are dense and row-major.
+ */
+#ifndef STARKV_H
+#define STARKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define STARKV_API __attribute__((visibility("default")))
+#else
+#define STARKV_API
+#endif
+
+#define STARKV_PAGE_TOKENS 16 /* tokens per cache page (a paged KV block) */
+
+typedef int32_t starkv_status;
+enum {
+  STARKV_OK = 0,
+  STARKV_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad enum   */
+  STARKV_ERR_UNSUPPORTED_SHAPE = 2,  /* a configuration this build cannot run   */
+  STARKV_ERR_WORKSPACE_TOO_SMALL = 3,/* workspace_bytes below the required size */
+  STARKV_ERR_CUDA = 4,               /* a CUDA runtime call failed               */
+  STARKV_ERR_DEVICE_STATUS = 5       /* the device status word is non-zero       */
+};
+
+/* Device status word bits (see starkv_read_device_status). */
+enum {
+  STARKV_DEV_BAD_PAGE = 1u << 0,     /* block-table entry < 0 or >= n_pages      */
+  STARKV_DEV_BAD_SEQ_LEN = 1u << 1,  /* seq_len < 0, > max_pages*16, or beyond
+                                        the context's max_position             */
+  STARKV_DEV_QUANT_OVERFLOW = 1u << 2,/* a group's fp16 scale/zero not finite, or
+                                        a non-finite latent                     */
+  STARKV_DEV_BAD_SLOT = 1u << 3,     /* append slot >= n_pages*16                */
+  STARKV_DEV_BAD_QUERY_SPAN = 1u << 4/* prefill: cu_q not non-decreasing, or a
+                                        sequence's query count > its seq_len    */
+};
+
+/* Opaque stream handle: pass a cudaStream_t. */
+typedef struct CUstream_st* starkv_stream_t;
+
+/* Model shape and quantisation settings.
+ * top_fraction: share of each latent's leading channels (singular-value order)
+ *   stored at 4 bits; the rest are stored at 3 bits ([Review] eq. 14; the
+ *   checkpoint card uses top_fraction = 0.25, top_bits = 4, bottom_bits = 3).
+ *   n_top = floor(top_fraction * r + 0.5).  The rotation and quantisation
+ *   group is g = gcd(16, n_top, r - n_top) channels, so no group straddles the
+ *   two precision blocks; g must be 4, 8 or 16.
+ * Supported: head_dim in {64, 128}; num_q_heads % num_kv_heads == 0;
+ *   rank_k <= head_dim, rank_k % 16 == 0; rank_v <= num_kv_heads*head_dim,
+ *   rank_v % 16 == 0; hidden % 64 == 0; rope_base > 1; max_position >= 1. */
+typedef struct starkv_config {
+  int32_t num_q_heads;  /* H                                            */
+  int32_t num_kv_heads; /* h_kv                                         */
+  int32_t head_dim;     /* d_h                                          */
+  int32_t hidden;       /* width of the hidden states X                 */
+  int32_t rank_k;       /* r_k: key latent rank per KV head             */
+  int32_t rank_v;       /* R: joint value latent rank                   */
+  int32_t max_position; /* positions [0, max_position) are supported    */
+  int32_t flags;        /* reserved, must be 0                          */
+  double top_fraction;  /* 0.25                                         */
+  double rope_base;     /* RoPE theta base (1e4 Llama-2, 5e5 Llama-3)   */
+} starkv_config;
+
+/* The four caller-allocated page pools of a paged latent cache.
+ *   k_codes: [n_pages][num_kv_heads][key_region_bytes]    packed key codes
+ *   v_codes: [n_pages][value_region_bytes]                packed value codes
+ *   k_meta : [n_pages][num_kv_heads][key_groups][16] x 4 B  (fp16 scale, fp16 zero)
+ *   v_meta : [n_pages][value_groups][16] x 4 B
+ * Each pool base must be 16-byte aligned.  A page holds 16 consecutive token
+ * positions of one sequence; a sequence's pages are listed in its block-table
+ * row.  Byte layout of one page of one latent region: group tiles in channel
+ * order; a 4-bit tile holds element (t, c) of its 16 x g block at nibble
+ * index t*g + c (low nibble first); a 3-bit tile is a 2-bit plane of the low
+ * bits (element i at bits 2*(i%4) of byte i/4) followed by a 1-bit plane of
+ * the high bit (bit i%8 of byte i/8).  Meta word: scale in the low 16 bits,
+ * zero-point in the high 16 bits. */
+typedef struct starkv_cache {
+  void* k_codes;
+  void* v_codes;
+  void* k_meta;
+  void* v_meta;
+  int64_t n_pages;
+} starkv_cache;
+
+typedef struct starkv_cache_sizes {
+  int64_t k_codes_bytes; /* pool sizes for the requested n_pages */
+  int64_t v_codes_bytes;
+  int64_t k_meta_bytes;
+  int64_t v_meta_bytes;
+  int32_t key_region_bytes;   /* per page per KV head (payload padded to 16 B) */
+  int32_t value_region_bytes; /* per page                                      */
+  int32_t key_group_size;     /* g of a key latent                             */
+  int32_t value_group_size;   /* g of the value latent                         */
+  int32_t key_top;            /* n_top of a key latent                         */
+  int32_t value_top;          /* n_top of the value latent                     */
+  int32_t key_groups;         /* r_k / g                                       */
+  int32_t value_groups;       /* R / g                                         */
+} starkv_cache_sizes;
+
+typedef struct starkv_ctx starkv_ctx;
+
+enum { STARKV_OP_DECODE = 0, STARKV_OP_PREFILL = 1 };
+enum { STARKV_LATENT_KEY = 0, STARKV_LATENT_VALUE = 1 };
+
+/* Library version string (static storage). */
+STARKV_API const char* starkv_version(void);
+
+/* Message of the calling thread's last failed call (static per thread). */
+STARKV_API const char* starkv_last_error(void);
+
+/* Host-only: check a configuration and return the cache pool sizes for
+ * n_pages pages (the packed layout above; [Review] eq. 15 plus metadata and
+ * padding).  out: host.  Errors: INVALID_ARG, UNSUPPORTED_SHAPE. */
+STARKV_API starkv_status starkv_cache_layout(const starkv_config* cfg, int64_t n_pages,
+                                  starkv_cache_sizes* out);
+
+/* Create a context on the current CUDA device.
+ * A_k: device bf16 [hidden][num_kv_heads*rank_k], head h's columns at h*rank_k
+ *      (its latent channels in singular-value order);
+ * A_v: device bf16 [hidden][rank_v];
+ * B_k: device bf16 [num_kv_heads][rank_k][head_dim];
+ * B_v: device bf16 [rank_v][num_kv_heads*head_dim].
+ * The factors are copied into context-owned memory; the rotation is folded
+ * into the up-projections (B' = H B, exact by [Review] eq. 13) and a RoPE
+ * cos/sin table for [0, max_position) is built in fp64 and stored as fp32.
+ * Synchronises `stream` before returning, so the inputs may be freed after.
+ * out: host, receives the context.  Errors: INVALID_ARG, UNSUPPORTED_SHAPE, CUDA. */
+STARKV_API starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const void* A_v,
+                            const void* B_k, const void* B_v, starkv_stream_t stream,
+                            starkv_ctx** out);
+
+/* Free a context (device-synchronising).  NULL is accepted. */
+STARKV_API starkv_status starkv_destroy(starkv_ctx* ctx);
+
+/* Sizes the context was created with (host copy). */
+STARKV_API starkv_status starkv_get_config(const starkv_ctx* ctx, starkv_config* out);
+
+/* Append n tokens: decode dataflow steps 1-3 ([Review] Algorithm 2: project
+ * the hidden states into latent keys and values, apply the block rotations,
+ * quantise and append).  X: device bf16 [n][hidden].  slot_mapping: device
+ * int64 [n], slot = page*16 + offset; a negative slot skips that token; slots
+ * must be distinct within one call.  Only the written tokens' bits change.
+ * latents_out: optional device fp32 [n][num_kv_heads*rank_k + rank_v], receives
+ * the pre-quantisation latents (debug export; NULL to skip).
+ * Errors: INVALID_ARG; device bits BAD_SLOT, QUANT_OVERFLOW. */
+STARKV_API starkv_status starkv_append(starkv_ctx* ctx, const starkv_cache* cache, const void* X,
+                            const int64_t* slot_mapping, int64_t n, float* latents_out,
+                            starkv_stream_t stream);
+
+/* Workspace bytes needed by decode (op = STARKV_OP_DECODE; total_q ignored) or
+ * prefill (op = STARKV_OP_PREFILL) for `batch` sequences whose block tables
+ * have max_pages columns.  out: host. */
+STARKV_API starkv_status starkv_workspace_bytes(const starkv_ctx* ctx, int32_t op, int32_t batch,
+                                     int32_t max_pages, int64_t total_q, size_t* out);
+
+/* Batched single-query decode attention over the packed cache ([Review]
+ * Algorithm 2 steps 4-8; keys re-expanded and RoPE'd in the kernel, values
+ * aggregated in the R-dim latent and projected by B_v afterwards, split-K
+ * partials merged by the softmax partition identity).
+ * q: device bf16 [batch][num_q_heads][head_dim], pre-RoPE; sequence b's query
+ *    sits at position seq_lens[b]-1 and attends to positions [0, seq_lens[b]).
+ * block_table: device int32 [batch][max_pages]; seq_lens: device int32 [batch].
+ * out: device bf16 [batch][num_q_heads][head_dim], each head's attention output
+ *      before the output projection W_o.  seq_len 0 gives a zero row.
+ * workspace: device, >= starkv_workspace_bytes(DECODE), 256-byte aligned.
+ * Errors: INVALID_ARG, WORKSPACE_TOO_SMALL; device bits BAD_PAGE, BAD_SEQ_LEN. */
+STARKV_API starkv_status starkv_decode_attn(starkv_ctx* ctx, const starkv_cache* cache, const void* q,
+                                 const int32_t* block_table, const int32_t* seq_lens,
+                                 int32_t batch, int32_t max_pages, void* out, void* workspace,
+                                 size_t workspace_bytes, starkv_stream_t stream);
+
+/* Causal chunk attention over the packed cache (the chunked form of the same
+ * dataflow).  q: device bf16 [total_q][num_q_heads][head_dim], pre-RoPE, rows of
+ * sequence b at cu_q[b] .. cu_q[b+1]-1 (cu_q: device int32 [batch+1], cu_q[0]=0,
+ * cu_q[batch] = total_q).  Query i of sequence b sits at position
+ * seq_lens[b] - n_b + i (n_b = its query count, <= seq_lens[b]) and attends to
+ * positions <= its own; the chunk's own tokens must already be appended.
+ * max_q_len: upper bound of n_b.  out: device bf16 [total_q][num_q_heads][head_dim].
+ * workspace: >= starkv_workspace_bytes(PREFILL, batch, max_pages, total_q).
+ * Errors: INVALID_ARG, WORKSPACE_TOO_SMALL; device bits BAD_PAGE, BAD_SEQ_LEN,
+ * BAD_QUERY_SPAN. */
+STARKV_API starkv_status starkv_prefill_attn(starkv_ctx* ctx, const starkv_cache* cache, const void* q,
+                                  const int32_t* cu_q, const int32_t* block_table,
+                                  const int32_t* seq_lens, int32_t batch, int32_t max_pages,
+                                  int64_t total_q, int32_t max_q_len, void* out,
+                                  void* workspace, size_t workspace_bytes,
+                                  starkv_stream_t stream);
+
+/* Rotate, quantise and pack n pre-quantisation latents of one latent kind
+ * (which = STARKV_LATENT_KEY: a KV head's r_k channels; STARKV_LATENT_VALUE:
+ * the R channels) into ceil(n/16) pages of one region ([Review] section 6.1,
+ * eq. 13-14).  z: device fp32 [n][r].  codes: device [ceil(n/16)][region_bytes];
+ * meta: device [ceil(n/16)][groups][16] x 4 B; both fully overwritten (rows
+ * past n: zero codes, zero scale and zero-point).  Same arithmetic as the
+ * append kernel's quantiser.  Errors: INVALID_ARG; device bit QUANT_OVERFLOW. */
+STARKV_API starkv_status starkv_quantize_pack(starkv_ctx* ctx, int32_t which, const float* z, int64_t n,
+                                   void* codes, void* meta, starkv_stream_t stream);
+
+/* Unpack and dequantise the first n tokens of packed pages of one region:
+ * z_hat = code*scale + zero in fp32, rotated domain.  z_out: device fp32 [n][r]. */
+STARKV_API starkv_status starkv_dequantize(starkv_ctx* ctx, int32_t which, const void* codes,
+                                const void* meta, int64_t n, float* z_out,
+                                starkv_stream_t stream);
+
+/* Synchronise `stream`, return the device status word in *status (host) and
+ * clear it.  Returns DEVICE_STATUS when the word was non-zero. */
+STARKV_API starkv_status starkv_read_device_status(starkv_ctx* ctx, starkv_stream_t stream,
+                                        uint32_t* status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* STARKV_H */

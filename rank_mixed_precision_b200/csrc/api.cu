@@ -1,0 +1,335 @@
+// Host side of the C ABI: argument checks, context lifetime, dispatch.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "internal.cuh"
+
+using namespace starkv;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+starkv_status fail(starkv_status code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+starkv_status ok() {
+  g_err[0] = 0;
+  return STARKV_OK;
+}
+
+starkv_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(STARKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int gcd_int(int a, int b) {
+  while (b) {
+    int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
+
+// Channel split of an r-channel latent: n_top = floor(top_fraction * r + 0.5),
+// g = gcd(16, n_top, r - n_top).
+bool make_geom(int r, double frac, LatentGeom* L) {
+  const int n_top = (int)floor(frac * r + 0.5);
+  const int n_bot = r - n_top;
+  if (n_top < 0 || n_bot < 0) return false;
+  const int g = gcd_int(16, gcd_int(n_top, n_bot));
+  if (g != 4 && g != 8 && g != 16) return false;
+  L->r = r;
+  L->n_top = n_top;
+  L->g = g;
+  L->groups = r / g;
+  L->top_groups = n_top / g;
+  L->payload_bytes = 2 * (4 * n_top + 3 * n_bot);
+  L->region_bytes = (L->payload_bytes + 15) / 16 * 16;
+  return true;
+}
+
+starkv_status check_config(const starkv_config* c, LatentGeom* key, LatentGeom* val) {
+  if (!c) return fail(STARKV_ERR_INVALID_ARG, "config is NULL");
+  if (c->num_q_heads <= 0 || c->num_kv_heads <= 0 || c->head_dim <= 0 || c->hidden <= 0 ||
+      c->rank_k <= 0 || c->rank_v <= 0 || c->max_position <= 0)
+    return fail(STARKV_ERR_INVALID_ARG, "config sizes must be positive");
+  if (c->flags != 0) return fail(STARKV_ERR_INVALID_ARG, "config.flags must be 0");
+  if (!(c->top_fraction >= 0.0 && c->top_fraction <= 1.0))
+    return fail(STARKV_ERR_INVALID_ARG, "top_fraction must lie in [0, 1]");
+  if (!(c->rope_base > 1.0)) return fail(STARKV_ERR_INVALID_ARG, "rope_base must exceed 1");
+  if (c->head_dim != 64 && c->head_dim != 128)
+    return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "head_dim %d: only 64 and 128 are supported", c->head_dim);
+  if (c->num_q_heads % c->num_kv_heads != 0)
+    return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "num_q_heads %% num_kv_heads != 0");
+  if (c->rank_k > c->head_dim || c->rank_k % 16 != 0 || c->rank_k > 64)
+    return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "rank_k %d: need a multiple of 16, <= head_dim and <= 64", c->rank_k);
+  if (c->rank_v > c->num_kv_heads * c->head_dim || c->rank_v % 16 != 0 || c->rank_v > 1024)
+    return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "rank_v %d: need a multiple of 16, <= h_kv*head_dim and <= 1024", c->rank_v);
+  if (c->hidden % 64 != 0) return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "hidden %% 64 != 0");
+  if (c->max_position > (1 << 24)) return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "max_position too large");
+  LatentGeom k, v;
+  if (!make_geom(c->rank_k, c->top_fraction, &k))
+    return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "key latent: group size gcd(16, n_top, n_bot) must be 4, 8 or 16");
+  if (!make_geom(c->rank_v, c->top_fraction, &v))
+    return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "value latent: group size gcd(16, n_top, n_bot) must be 4, 8 or 16");
+  if (key) *key = k;
+  if (val) *val = v;
+  return STARKV_OK;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+starkv_status check_cache(const Ctx* c, const starkv_cache* cache) {
+  if (!cache) return fail(STARKV_ERR_INVALID_ARG, "cache is NULL");
+  if (cache->n_pages < 0) return fail(STARKV_ERR_INVALID_ARG, "cache.n_pages < 0");
+  if (cache->n_pages > 0 && (!cache->k_codes || !cache->v_codes || !cache->k_meta || !cache->v_meta))
+    return fail(STARKV_ERR_INVALID_ARG, "cache pool pointer is NULL");
+  if (!aligned16(cache->k_codes) || !aligned16(cache->v_codes) || !aligned16(cache->k_meta) ||
+      !aligned16(cache->v_meta))
+    return fail(STARKV_ERR_INVALID_ARG, "cache pools must be 16-byte aligned");
+  (void)c;
+  return STARKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* starkv_version(void) { return "starkv-b200 0.1 (sm_100a)"; }
+
+const char* starkv_last_error(void) { return g_err; }
+
+starkv_status starkv_cache_layout(const starkv_config* cfg, int64_t n_pages, starkv_cache_sizes* out) {
+  LatentGeom k, v;
+  starkv_status st = check_config(cfg, &k, &v);
+  if (st) return st;
+  if (!out) return fail(STARKV_ERR_INVALID_ARG, "out is NULL");
+  if (n_pages < 0) return fail(STARKV_ERR_INVALID_ARG, "n_pages < 0");
+  out->key_region_bytes = k.region_bytes;
+  out->value_region_bytes = v.region_bytes;
+  out->key_group_size = k.g;
+  out->value_group_size = v.g;
+  out->key_top = k.n_top;
+  out->value_top = v.n_top;
+  out->key_groups = k.groups;
+  out->value_groups = v.groups;
+  out->k_codes_bytes = n_pages * cfg->num_kv_heads * (int64_t)k.region_bytes;
+  out->v_codes_bytes = n_pages * (int64_t)v.region_bytes;
+  out->k_meta_bytes = n_pages * cfg->num_kv_heads * (int64_t)k.groups * kPage * 4;
+  out->v_meta_bytes = n_pages * (int64_t)v.groups * kPage * 4;
+  return ok();
+}
+
+starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const void* A_v, const void* B_k,
+                            const void* B_v, starkv_stream_t stream, starkv_ctx** out) {
+  LatentGeom k, v;
+  starkv_status st = check_config(cfg, &k, &v);
+  if (st) return st;
+  if (!out) return fail(STARKV_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!A_k || !A_v || !B_k || !B_v) return fail(STARKV_ERR_INVALID_ARG, "factor pointer is NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  Ctx* c = new (std::nothrow) Ctx();
+  if (!c) return fail(STARKV_ERR_CUDA, "out of host memory");
+  c->cfg = *cfg;
+  c->key = k;
+  c->val = v;
+  c->group = cfg->num_q_heads / cfg->num_kv_heads;
+  c->lat_cols = cfg->num_kv_heads * cfg->rank_k + cfg->rank_v;
+  cudaGetDevice(&c->device);
+  const int d = cfg->head_dim, half = d / 2;
+  const size_t a_bytes = (size_t)cfg->hidden * c->lat_cols * 2;
+  const size_t bk_bytes = (size_t)cfg->num_kv_heads * cfg->rank_k * d * 4;
+  const size_t bv_bytes = (size_t)cfg->rank_v * cfg->num_kv_heads * d * 4;
+  const size_t rope_bytes = (size_t)cfg->max_position * half * sizeof(float2);
+  cudaError_t e;
+  auto cleanup = [&]() {
+    cudaFree(c->A);
+    cudaFree(c->Bk);
+    cudaFree(c->Bv);
+    cudaFree(c->rope);
+    cudaFree(c->status);
+    delete c;
+  };
+  if ((e = cudaMalloc(&c->A, a_bytes)) != cudaSuccess || (e = cudaMalloc(&c->Bk, bk_bytes)) != cudaSuccess ||
+      (e = cudaMalloc(&c->Bv, bv_bytes)) != cudaSuccess || (e = cudaMalloc(&c->rope, rope_bytes)) != cudaSuccess ||
+      (e = cudaMalloc(&c->status, sizeof(unsigned int))) != cudaSuccess) {
+    cleanup();
+    return cuda_fail(e, "cudaMalloc (context factors)");
+  }
+  // A = [A_k | A_v], row-major [hidden][lat_cols]
+  const size_t kcols = (size_t)cfg->num_kv_heads * cfg->rank_k;
+  e = cudaMemcpy2DAsync(c->A, c->lat_cols * 2, A_k, kcols * 2, kcols * 2, cfg->hidden, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpy2DAsync((char*)c->A + kcols * 2, c->lat_cols * 2, A_v, (size_t)cfg->rank_v * 2,
+                          (size_t)cfg->rank_v * 2, cfg->hidden, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = launch_prepare_factors(*c, (const __nv_bfloat16*)B_k, (const __nv_bfloat16*)B_v, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->status, 0, sizeof(unsigned int), s);
+  // RoPE table: angle p * base^(-2i/d) in fp64, cos/sin in fp64, stored as fp32
+  std::vector<float2> rope((size_t)cfg->max_position * half);
+  std::vector<double> theta(half);
+  for (int i = 0; i < half; ++i) theta[i] = pow(cfg->rope_base, -2.0 * i / d);
+  for (int p = 0; p < cfg->max_position; ++p)
+    for (int i = 0; i < half; ++i) {
+      const double ang = (double)p * theta[i];
+      rope[(size_t)p * half + i] = make_float2((float)cos(ang), (float)sin(ang));
+    }
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->rope, rope.data(), rope_bytes, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    cleanup();
+    return cuda_fail(e, "starkv_create");
+  }
+  *out = reinterpret_cast<starkv_ctx*>(c);
+  return ok();
+}
+
+starkv_status starkv_destroy(starkv_ctx* ctx) {
+  if (!ctx) return ok();
+  Ctx* c = reinterpret_cast<Ctx*>(ctx);
+  cudaDeviceSynchronize();
+  cudaFree(c->A);
+  cudaFree(c->Bk);
+  cudaFree(c->Bv);
+  cudaFree(c->rope);
+  cudaFree(c->status);
+  delete c;
+  return ok();
+}
+
+starkv_status starkv_get_config(const starkv_ctx* ctx, starkv_config* out) {
+  if (!ctx || !out) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
+  *out = reinterpret_cast<const Ctx*>(ctx)->cfg;
+  return ok();
+}
+
+starkv_status starkv_append(starkv_ctx* ctx, const starkv_cache* cache, const void* X, const int64_t* slot_mapping,
+                            int64_t n, float* latents_out, starkv_stream_t stream) {
+  if (!ctx) return fail(STARKV_ERR_INVALID_ARG, "ctx is NULL");
+  Ctx* c = reinterpret_cast<Ctx*>(ctx);
+  starkv_status st = check_cache(c, cache);
+  if (st) return st;
+  if (n < 0) return fail(STARKV_ERR_INVALID_ARG, "n < 0");
+  if (n > 0 && (!X || !slot_mapping)) return fail(STARKV_ERR_INVALID_ARG, "X or slot_mapping is NULL");
+  if (n > 0 && cache->n_pages == 0) return fail(STARKV_ERR_INVALID_ARG, "cache has no pages");
+  cudaError_t e = launch_append(*c, *cache, (const __nv_bfloat16*)X, slot_mapping, n, latents_out, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  return ok();
+}
+
+starkv_status starkv_workspace_bytes(const starkv_ctx* ctx, int32_t op, int32_t batch, int32_t max_pages,
+                                     int64_t total_q, size_t* out) {
+  if (!ctx || !out) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
+  if (batch < 0 || max_pages < 0 || total_q < 0) return fail(STARKV_ERR_INVALID_ARG, "negative size");
+  const Ctx* c = reinterpret_cast<const Ctx*>(ctx);
+  if (op == STARKV_OP_DECODE) {
+    *out = plan_decode(*c, batch, max_pages).ws_bytes;
+  } else if (op == STARKV_OP_PREFILL) {
+    *out = plan_prefill(*c, batch, max_pages, total_q).ws_bytes;
+  } else {
+    return fail(STARKV_ERR_INVALID_ARG, "unknown op %d", op);
+  }
+  return ok();
+}
+
+starkv_status starkv_decode_attn(starkv_ctx* ctx, const starkv_cache* cache, const void* q, const int32_t* block_table,
+                                 const int32_t* seq_lens, int32_t batch, int32_t max_pages, void* out,
+                                 void* workspace, size_t workspace_bytes, starkv_stream_t stream) {
+  if (!ctx) return fail(STARKV_ERR_INVALID_ARG, "ctx is NULL");
+  Ctx* c = reinterpret_cast<Ctx*>(ctx);
+  starkv_status st = check_cache(c, cache);
+  if (st) return st;
+  if (batch < 0 || max_pages < 0) return fail(STARKV_ERR_INVALID_ARG, "negative size");
+  if (batch == 0) return ok();
+  if (max_pages == 0) return fail(STARKV_ERR_INVALID_ARG, "max_pages must be >= 1");
+  if (!q || !block_table || !seq_lens || !out) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
+  const DecodePlan plan = plan_decode(*c, batch, max_pages);
+  if (!workspace || workspace_bytes < plan.ws_bytes)
+    return fail(STARKV_ERR_WORKSPACE_TOO_SMALL, "decode needs %zu workspace bytes, got %zu", plan.ws_bytes,
+                workspace ? workspace_bytes : (size_t)0);
+  if (((uintptr_t)workspace & 255) != 0) return fail(STARKV_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  cudaError_t e = launch_decode(*c, *cache, (const __nv_bfloat16*)q, block_table, seq_lens, batch, max_pages,
+                                (__nv_bfloat16*)out, workspace, plan, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return ok();
+}
+
+starkv_status starkv_prefill_attn(starkv_ctx* ctx, const starkv_cache* cache, const void* q, const int32_t* cu_q,
+                                  const int32_t* block_table, const int32_t* seq_lens, int32_t batch,
+                                  int32_t max_pages, int64_t total_q, int32_t max_q_len, void* out,
+                                  void* workspace, size_t workspace_bytes, starkv_stream_t stream) {
+  if (!ctx) return fail(STARKV_ERR_INVALID_ARG, "ctx is NULL");
+  Ctx* c = reinterpret_cast<Ctx*>(ctx);
+  starkv_status st = check_cache(c, cache);
+  if (st) return st;
+  if (batch < 0 || max_pages < 0 || total_q < 0 || max_q_len < 0)
+    return fail(STARKV_ERR_INVALID_ARG, "negative size");
+  if (batch == 0 || total_q == 0) return ok();
+  if (max_pages == 0) return fail(STARKV_ERR_INVALID_ARG, "max_pages must be >= 1");
+  if (max_q_len == 0 || max_q_len > max_pages * kPage)
+    return fail(STARKV_ERR_INVALID_ARG, "max_q_len must lie in [1, max_pages*16]");
+  if (!q || !cu_q || !block_table || !seq_lens || !out) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
+  const PrefillPlan plan = plan_prefill(*c, batch, max_pages, total_q);
+  if (!workspace || workspace_bytes < plan.ws_bytes)
+    return fail(STARKV_ERR_WORKSPACE_TOO_SMALL, "prefill needs %zu workspace bytes, got %zu", plan.ws_bytes,
+                workspace ? workspace_bytes : (size_t)0);
+  if (((uintptr_t)workspace & 255) != 0) return fail(STARKV_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  cudaError_t e = launch_prefill(*c, *cache, (const __nv_bfloat16*)q, cu_q, block_table, seq_lens, batch, max_pages,
+                                 total_q, max_q_len, (__nv_bfloat16*)out, workspace, plan, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  return ok();
+}
+
+starkv_status starkv_quantize_pack(starkv_ctx* ctx, int32_t which, const float* z, int64_t n, void* codes,
+                                   void* meta, starkv_stream_t stream) {
+  if (!ctx) return fail(STARKV_ERR_INVALID_ARG, "ctx is NULL");
+  Ctx* c = reinterpret_cast<Ctx*>(ctx);
+  if (which != STARKV_LATENT_KEY && which != STARKV_LATENT_VALUE) return fail(STARKV_ERR_INVALID_ARG, "bad latent kind");
+  if (n < 0) return fail(STARKV_ERR_INVALID_ARG, "n < 0");
+  if (n > 0 && (!z || !codes || !meta)) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
+  if (!aligned16(codes) || !aligned16(meta)) return fail(STARKV_ERR_INVALID_ARG, "codes/meta must be 16-byte aligned");
+  const LatentGeom& L = which == STARKV_LATENT_KEY ? c->key : c->val;
+  cudaError_t e = launch_quantize_pack(*c, L, z, n, (uint8_t*)codes, (uint32_t*)meta, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize_pack launch");
+  return ok();
+}
+
+starkv_status starkv_dequantize(starkv_ctx* ctx, int32_t which, const void* codes, const void* meta, int64_t n,
+                                float* z_out, starkv_stream_t stream) {
+  if (!ctx) return fail(STARKV_ERR_INVALID_ARG, "ctx is NULL");
+  Ctx* c = reinterpret_cast<Ctx*>(ctx);
+  if (which != STARKV_LATENT_KEY && which != STARKV_LATENT_VALUE) return fail(STARKV_ERR_INVALID_ARG, "bad latent kind");
+  if (n < 0) return fail(STARKV_ERR_INVALID_ARG, "n < 0");
+  if (n > 0 && (!z_out || !codes || !meta)) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
+  const LatentGeom& L = which == STARKV_LATENT_KEY ? c->key : c->val;
+  cudaError_t e = launch_dequantize(*c, L, (const uint8_t*)codes, (const uint32_t*)meta, n, z_out, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
+  return ok();
+}
+
+starkv_status starkv_read_device_status(starkv_ctx* ctx, starkv_stream_t stream, uint32_t* status) {
+  if (!ctx || !status) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
+  Ctx* c = reinterpret_cast<Ctx*>(ctx);
+  cudaStream_t s = (cudaStream_t)stream;
+  unsigned int h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, c->status, sizeof(h), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->status, 0, sizeof(unsigned int), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "read_device_status");
+  *status = h;
+  if (h) return fail(STARKV_ERR_DEVICE_STATUS, "device status 0x%x", h);
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,224 @@
+// Internal definitions shared by the library's CUDA sources.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/starkv.h"
+
+namespace starkv {
+
+constexpr int kPage = STARKV_PAGE_TOKENS;
+
+// Geometry of one latent (a KV head's key latent, or the joint value latent).
+struct LatentGeom {
+  int r;             // channels
+  int n_top;         // leading 4-bit channels
+  int g;             // rotation / quantisation group size (4, 8 or 16)
+  int groups;        // r / g
+  int top_groups;    // n_top / g
+  int payload_bytes; // 2 * (4 n_top + 3 (r - n_top)) per page
+  int region_bytes;  // payload rounded up to 16
+};
+
+// Byte offset of group tile `gi` inside a page region.
+__host__ __device__ inline int tile_offset(const LatentGeom& L, int gi) {
+  return gi < L.top_groups ? gi * 8 * L.g : L.top_groups * 8 * L.g + (gi - L.top_groups) * 6 * L.g;
+}
+
+struct Ctx {
+  starkv_config cfg;
+  LatentGeom key, val;
+  int group;              // H / h_kv
+  int lat_cols;           // h_kv * r_k + R
+  int device;
+  // context-owned device memory
+  __nv_bfloat16* A;       // [hidden][lat_cols] bf16: A_k | A_v side by side
+  float* Bk;              // [h_kv][r_k][d_h]  fp32, B'_k = H B_k (rotation folded)
+  float* Bv;              // [R][h_kv*d_h]     fp32, B'_v = H B_v
+  float2* rope;           // [max_position][d_h/2] (cos, sin), built in fp64
+  unsigned int* status;   // device status word
+};
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+__device__ inline void set_status(unsigned int* st, unsigned int bit) { atomicOr(st, bit); }
+
+// fl32(1/sqrt(g)) written as decimal literals the compiler rounds correctly.
+__device__ inline float inv_sqrt_group(int g) {
+  switch (g) {
+    case 4: return 0.5f;
+    case 8: return 0.353553390593273762200422181052424519642f;
+    case 16: return 0.25f;
+    default: return 0.707106781186547524400844362104849039284f;  // g == 2
+  }
+}
+
+// In-place z <- z H_g (normalised Sylvester Hadamard) with fp32 butterflies of
+// half-width 1, 2, 4, ... followed by one multiply by fl32(1/sqrt g).
+template <int G>
+__device__ inline void fwht_fl32(float (&x)[G]) {
+#pragma unroll
+  for (int h = 1; h < G; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      if ((i & h) == 0) {
+        float a = x[i], b = x[i + h];
+        x[i] = __fadd_rn(a, b);
+        x[i + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+  const float c = inv_sqrt_group(G);
+#pragma unroll
+  for (int i = 0; i < G; ++i) x[i] = __fmul_rn(x[i], c);
+}
+
+// Asymmetric min/max quantiser of one group: fp16 scale and zero (= min),
+// round-half-even, clamp.  Returns false when the scale or zero is not finite
+// (or an input is not finite); codes are then all zero.
+template <int G>
+__device__ inline bool quantize_group(const float (&x)[G], int bits, uint8_t (&code)[G],
+                                      __half& s16, __half& zp16) {
+  float mn = x[0], mx = x[0];
+  bool finite = isfinite(x[0]);
+#pragma unroll
+  for (int i = 1; i < G; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+    finite = finite && isfinite(x[i]);
+  }
+  const float qmax = (float)((1 << bits) - 1);
+  s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), qmax));
+  zp16 = __float2half_rn(mn);
+  const float sf = __half2float(s16), zf = __half2float(zp16);
+  if (!finite || !isfinite(sf) || !isfinite(zf)) {
+#pragma unroll
+    for (int i = 0; i < G; ++i) code[i] = 0;
+    s16 = __float2half_rn(0.f);
+    zp16 = __float2half_rn(0.f);
+    return false;
+  }
+#pragma unroll
+  for (int i = 0; i < G; ++i) {
+    float q = 0.f;
+    if (sf != 0.f) q = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(x[i], zf), sf)), 0.f), qmax);
+    code[i] = (uint8_t)q;
+  }
+  return true;
+}
+
+// Write one token's codes of one group into its page tile.  The token's bits
+// are cleared and set with 32-bit atomics, so tokens sharing a word (and a
+// page being written by other threads) stay intact.  region: 4-byte aligned
+// base of the page region; t: token offset in the page.
+template <int G>
+__device__ inline void store_group_codes(uint8_t* region, const LatentGeom& L, int gi, int t,
+                                         const uint8_t (&code)[G]) {
+  uint32_t* tile = reinterpret_cast<uint32_t*>(region + tile_offset(L, gi));
+  if (gi < L.top_groups) {
+    // 4-bit: nibble index i = t*G + c, nibble (i % 8) of word i / 8
+#pragma unroll
+    for (int c0 = 0; c0 < G; c0 += (G < 8 ? G : 8)) {
+      const int i0 = t * G + c0;
+      const int w = i0 >> 3, sh = (i0 & 7) * 4;
+      const int cnt = G < 8 ? G : 8;
+      uint32_t bits = 0, mask = 0;
+#pragma unroll
+      for (int c = 0; c < cnt; ++c) {
+        bits |= (uint32_t)(code[c0 + c] & 0xF) << (4 * c);
+        mask |= 0xFu << (4 * c);
+      }
+      atomicAnd(&tile[w], ~(mask << sh));
+      atomicOr(&tile[w], bits << sh);
+    }
+  } else {
+    // 2-bit plane (4G bytes) then 1-bit plane (2G bytes)
+    uint32_t* plane2 = tile;
+    uint32_t* plane1 = tile + G;  // 4G bytes = G words
+#pragma unroll
+    for (int c0 = 0; c0 < G; c0 += (G < 16 ? G : 16)) {
+      const int cnt = G < 16 ? G : 16;
+      const int i0 = t * G + c0;
+      const int w = i0 >> 4, sh = (i0 & 15) * 2;
+      uint32_t bits = 0, mask = 0;
+#pragma unroll
+      for (int c = 0; c < cnt; ++c) {
+        bits |= (uint32_t)(code[c0 + c] & 3) << (2 * c);
+        mask |= 3u << (2 * c);
+      }
+      atomicAnd(&plane2[w], ~(mask << sh));
+      atomicOr(&plane2[w], bits << sh);
+    }
+    {
+      const int i0 = t * G;
+      const int w = i0 >> 5, sh = i0 & 31;
+      uint32_t bits = 0, mask = 0;
+#pragma unroll
+      for (int c = 0; c < G; ++c) {
+        bits |= (uint32_t)((code[c] >> 2) & 1) << c;
+        mask |= 1u << c;
+      }
+      atomicAnd(&plane1[w], ~(mask << sh));
+      atomicOr(&plane1[w], bits << sh);
+    }
+  }
+}
+
+// Code of element (t, c) of group gi of a page region (generic, unoptimised).
+__device__ inline int load_code(const uint8_t* region, const LatentGeom& L, int gi, int t, int c) {
+  const uint8_t* tile = region + tile_offset(L, gi);
+  const int i = t * L.g + c;
+  if (gi < L.top_groups) {
+    const uint8_t b = tile[i >> 1];
+    return (i & 1) ? (b >> 4) : (b & 0xF);
+  }
+  const uint8_t b2 = tile[i >> 2];
+  const uint8_t b1 = tile[4 * L.g + (i >> 3)];
+  return ((b2 >> (2 * (i & 3))) & 3) | (((b1 >> (i & 7)) & 1) << 2);
+}
+
+__device__ inline float2 unpack_meta(uint32_t m) {
+  __half_raw s, z;
+  s.x = (unsigned short)(m & 0xFFFF);
+  z.x = (unsigned short)(m >> 16);
+  return make_float2(__half2float(__half(s)), __half2float(__half(z)));
+}
+
+// ---------------------------------------------------------------------------
+// Launchers (defined in the .cu files)
+// ---------------------------------------------------------------------------
+cudaError_t launch_prepare_factors(const Ctx& c, const __nv_bfloat16* Bk, const __nv_bfloat16* Bv,
+                                   cudaStream_t s);
+cudaError_t launch_quantize_pack(const Ctx& c, const LatentGeom& L, const float* z, int64_t n,
+                                 uint8_t* codes, uint32_t* meta, cudaStream_t s);
+cudaError_t launch_dequantize(const Ctx& c, const LatentGeom& L, const uint8_t* codes,
+                              const uint32_t* meta, int64_t n, float* z, cudaStream_t s);
+cudaError_t launch_append(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* X,
+                          const int64_t* slots, int64_t n, float* latents_out, cudaStream_t s);
+
+struct DecodePlan {
+  int splits;
+  int pages_per_split;
+  size_t ws_bytes;
+};
+DecodePlan plan_decode(const Ctx& c, int batch, int max_pages);
+cudaError_t launch_decode(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
+                          const int32_t* block_table, const int32_t* seq_lens, int batch,
+                          int max_pages, __nv_bfloat16* out, void* ws, const DecodePlan& plan,
+                          cudaStream_t s);
+
+struct PrefillPlan {
+  int chunk;          // key positions expanded per pass
+  size_t ws_bytes;
+};
+PrefillPlan plan_prefill(const Ctx& c, int batch, int max_pages, int64_t total_q);
+cudaError_t launch_prefill(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
+                           const int32_t* cu_q, const int32_t* block_table, const int32_t* seq_lens,
+                           int batch, int max_pages, int64_t total_q, int max_q_len,
+                           __nv_bfloat16* out, void* ws, const PrefillPlan& plan, cudaStream_t s);
+
+}  // namespace starkv

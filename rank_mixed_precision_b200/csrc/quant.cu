@@ -1,0 +1,262 @@
+// Factor preparation, the append kernel (projection with rotation, quantisation
+// and packing fused into its epilogue), and the quantise/dequantise entries.
+//
+// Source: "STAR-KV: Learning the Rank Is Only Half of KV Cache Compression",
+// Algorithm 2 steps 1-3 (project the new hidden state into latent keys and
+// values; apply the prepared block rotations; quantise and append), section 6.1
+// eq. 13 (block-diagonal orthogonal rotation, absorbed by the up-projection)
+// and eq. 14 (4-bit leading channels, 3-bit the rest).
+#include "internal.cuh"
+
+namespace starkv {
+
+// ---------------------------------------------------------------------------
+// B' = H B: fold the per-group rotation into an up-projection (eq. 13: the
+// up-projection absorbs H^T; H is symmetric).  One thread per output element,
+// fp64 accumulation of the g signed terms, rounded once to fp32.
+// B: [rows][cols] bf16 with rows grouped by g, out: [rows][cols] fp32.
+// ---------------------------------------------------------------------------
+__global__ void fold_rotation_kernel(const __nv_bfloat16* __restrict__ B, float* __restrict__ out,
+                                     int64_t rows, int cols, int g) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * cols) return;
+  const int64_t row = idx / cols;
+  const int col = (int)(idx % cols);
+  const int i = (int)(row % g);
+  const int64_t base = row - i;
+  double acc = 0.0;
+  for (int j = 0; j < g; ++j) {
+    const double v = (double)__bfloat162float(B[(base + j) * cols + col]);
+    acc += (__popc(i & j) & 1) ? -v : v;
+  }
+  out[idx] = (float)(acc / sqrt((double)g));
+}
+
+cudaError_t launch_prepare_factors(const Ctx& c, const __nv_bfloat16* Bk, const __nv_bfloat16* Bv,
+                                   cudaStream_t s) {
+  const starkv_config& f = c.cfg;
+  {
+    const int64_t rows = (int64_t)f.num_kv_heads * f.rank_k;  // groups never cross heads (g | r_k)
+    const int64_t total = rows * f.head_dim;
+    fold_rotation_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(Bk, c.Bk, rows, f.head_dim, c.key.g);
+  }
+  {
+    const int64_t rows = f.rank_v;
+    const int cols = f.num_kv_heads * f.head_dim;
+    const int64_t total = rows * cols;
+    fold_rotation_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(Bv, c.Bv, rows, cols, c.val.g);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Rotate + quantise + store one group of one token (shared by append and the
+// quantise entry).  x: the group's g pre-rotation latents.
+// ---------------------------------------------------------------------------
+template <int G>
+__device__ inline void rotate_quantize_store(const float* x_in, const LatentGeom& L, int gi,
+                                             uint8_t* region, uint32_t* meta_page, int t,
+                                             unsigned int* status) {
+  float x[G];
+#pragma unroll
+  for (int i = 0; i < G; ++i) x[i] = x_in[i];
+  fwht_fl32<G>(x);
+  uint8_t code[G];
+  __half s16, zp16;
+  const int bits = gi < L.top_groups ? 4 : 3;
+  if (!quantize_group<G>(x, bits, code, s16, zp16)) set_status(status, STARKV_DEV_QUANT_OVERFLOW);
+  store_group_codes<G>(region, L, gi, t, code);
+  const uint32_t m = (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(zp16) << 16);
+  meta_page[gi * kPage + t] = m;
+}
+
+__device__ inline void rotate_quantize_store_any(const float* x, const LatentGeom& L, int gi,
+                                                 uint8_t* region, uint32_t* meta_page, int t,
+                                                 unsigned int* status) {
+  switch (L.g) {
+    case 4: rotate_quantize_store<4>(x, L, gi, region, meta_page, t, status); break;
+    case 8: rotate_quantize_store<8>(x, L, gi, region, meta_page, t, status); break;
+    default: rotate_quantize_store<16>(x, L, gi, region, meta_page, t, status); break;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Quantise/pack entry: one thread per (token, group).  The pages are zeroed
+// by the launcher first.
+// ---------------------------------------------------------------------------
+__global__ void quantize_pack_kernel(LatentGeom L, const float* __restrict__ z, int64_t n,
+                                     uint8_t* __restrict__ codes, uint32_t* __restrict__ meta,
+                                     unsigned int* status) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n * L.groups) return;
+  const int64_t tok = idx / L.groups;
+  const int gi = (int)(idx % L.groups);
+  const int64_t page = tok / kPage;
+  const int t = (int)(tok % kPage);
+  rotate_quantize_store_any(z + tok * L.r + gi * L.g, L, gi, codes + page * L.region_bytes,
+                            meta + page * L.groups * kPage, t, status);
+}
+
+cudaError_t launch_quantize_pack(const Ctx& c, const LatentGeom& L, const float* z, int64_t n,
+                                 uint8_t* codes, uint32_t* meta, cudaStream_t s) {
+  const int64_t pages = (n + kPage - 1) / kPage;
+  cudaError_t e = cudaMemsetAsync(codes, 0, (size_t)pages * L.region_bytes, s);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(meta, 0, (size_t)pages * L.groups * kPage * 4, s);
+  if (e != cudaSuccess) return e;
+  const int64_t total = n * L.groups;
+  if (total == 0) return cudaSuccess;
+  quantize_pack_kernel<<<(unsigned)((total + 127) / 128), 128, 0, s>>>(L, z, n, codes, meta, c.status);
+  return cudaGetLastError();
+}
+
+// z_hat = fl32(code * s + zp): code * s is exact, so one fused multiply-add rounds once.
+__global__ void dequantize_kernel(LatentGeom L, const uint8_t* __restrict__ codes,
+                                  const uint32_t* __restrict__ meta, int64_t n, float* __restrict__ z) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n * L.r) return;
+  const int64_t tok = idx / L.r;
+  const int ch = (int)(idx % L.r);
+  const int64_t page = tok / kPage;
+  const int t = (int)(tok % kPage);
+  const int gi = ch / L.g;
+  const int code = load_code(codes + page * L.region_bytes, L, gi, t, ch % L.g);
+  const float2 sz = unpack_meta(meta[(page * L.groups + gi) * kPage + t]);
+  z[idx] = __fmaf_rn((float)code, sz.x, sz.y);
+}
+
+cudaError_t launch_dequantize(const Ctx&, const LatentGeom& L, const uint8_t* codes,
+                              const uint32_t* meta, int64_t n, float* z, cudaStream_t s) {
+  const int64_t total = n * L.r;
+  if (total == 0) return cudaSuccess;
+  dequantize_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(L, codes, meta, n, z);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Append: Z = X [A_k | A_v] (bf16 inputs, fp32 accumulation), then per
+// (token, group): rotate, quantise, pack into the token's page slot.
+// Tile: 32 tokens x 64 latent columns, 256 threads, 2 x 4 outputs per thread.
+// Every 64-column tile starts on a group boundary of whichever latent it
+// covers, because h_kv r_k and R are multiples of 16 and g divides 16.
+// ---------------------------------------------------------------------------
+struct AppendArgs {
+  LatentGeom key, val;
+  int h_kv, hidden, lat_cols;
+  int64_t n, n_pages;
+  const __nv_bfloat16* X;
+  const __nv_bfloat16* A;
+  const int64_t* slots;
+  float* lat_out;
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  uint32_t* k_meta;
+  uint32_t* v_meta;
+  unsigned int* status;
+};
+
+constexpr int kAppBM = 32, kAppBN = 64, kAppBK = 32;
+
+__global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
+  __shared__ float Xs[kAppBK][kAppBM + 1];
+  __shared__ float As[kAppBK][kAppBN];
+  __shared__ float Zs[kAppBM][kAppBN + 1];
+  const int tid = threadIdx.x;
+  const int64_t row0 = (int64_t)blockIdx.x * kAppBM;
+  const int col0 = blockIdx.y * kAppBN;
+  const int ty = tid / 16, tx = tid % 16;
+  float acc[2][4] = {};
+  for (int k0 = 0; k0 < a.hidden; k0 += kAppBK) {
+    for (int e = tid; e < kAppBM * kAppBK; e += 256) {
+      const int m = e / kAppBK, k = e % kAppBK;
+      const int64_t row = row0 + m;
+      Xs[k][m] = row < a.n ? __bfloat162float(a.X[row * a.hidden + k0 + k]) : 0.f;
+    }
+    for (int e = tid; e < kAppBK * kAppBN; e += 256) {
+      const int k = e / kAppBN, cc = e % kAppBN;
+      const int col = col0 + cc;
+      As[k][cc] = col < a.lat_cols ? __bfloat162float(a.A[(int64_t)(k0 + k) * a.lat_cols + col]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < kAppBK; ++k) {
+      const float x0 = Xs[k][ty * 2], x1 = Xs[k][ty * 2 + 1];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float w = As[k][tx * 4 + j];
+        acc[0][j] = fmaf(x0, w, acc[0][j]);
+        acc[1][j] = fmaf(x1, w, acc[1][j]);
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) Zs[ty * 2 + i][tx * 4 + j] = acc[i][j];
+  __syncthreads();
+  if (a.lat_out) {
+    for (int e = tid; e < kAppBM * kAppBN; e += 256) {
+      const int m = e / kAppBN, cc = e % kAppBN;
+      const int64_t row = row0 + m;
+      if (row < a.n && col0 + cc < a.lat_cols) a.lat_out[row * a.lat_cols + col0 + cc] = Zs[m][cc];
+    }
+  }
+  // epilogue: one item per (token, 4-column unit); the unit that starts a group does the group
+  const int key_cols = a.h_kv * a.key.r;
+  for (int e = tid; e < kAppBM * (kAppBN / 4); e += 256) {
+    const int m = e / (kAppBN / 4);
+    const int cc = (e % (kAppBN / 4)) * 4;
+    const int col = col0 + cc;
+    const int64_t row = row0 + m;
+    if (row >= a.n || col >= a.lat_cols) continue;
+    const bool is_key = col < key_cols;
+    const LatentGeom& L = is_key ? a.key : a.val;
+    const int cin = is_key ? col % a.key.r : col - key_cols;
+    if (cin % L.g != 0) continue;
+    const int64_t slot = a.slots[row];
+    if (slot < 0) continue;
+    if (slot >= a.n_pages * kPage) {
+      set_status(a.status, STARKV_DEV_BAD_SLOT);
+      continue;
+    }
+    const int64_t page = slot / kPage;
+    const int t = (int)(slot % kPage);
+    const int gi = cin / L.g;
+    if (is_key) {
+      const int kv = col / a.key.r;
+      rotate_quantize_store_any(&Zs[m][cc], L, gi, a.k_codes + (page * a.h_kv + kv) * L.region_bytes,
+                                a.k_meta + (page * a.h_kv + kv) * L.groups * kPage, t, a.status);
+    } else {
+      rotate_quantize_store_any(&Zs[m][cc], L, gi, a.v_codes + page * L.region_bytes,
+                                a.v_meta + page * L.groups * kPage, t, a.status);
+    }
+  }
+}
+
+cudaError_t launch_append(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* X,
+                          const int64_t* slots, int64_t n, float* latents_out, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  AppendArgs a;
+  a.key = c.key;
+  a.val = c.val;
+  a.h_kv = c.cfg.num_kv_heads;
+  a.hidden = c.cfg.hidden;
+  a.lat_cols = c.lat_cols;
+  a.n = n;
+  a.n_pages = cache.n_pages;
+  a.X = X;
+  a.A = c.A;
+  a.slots = slots;
+  a.lat_out = latents_out;
+  a.k_codes = (uint8_t*)cache.k_codes;
+  a.v_codes = (uint8_t*)cache.v_codes;
+  a.k_meta = (uint32_t*)cache.k_meta;
+  a.v_meta = (uint32_t*)cache.v_meta;
+  a.status = c.status;
+  dim3 grid((unsigned)((n + kAppBM - 1) / kAppBM), (unsigned)((c.lat_cols + kAppBN - 1) / kAppBN));
+  append_kernel<<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace starkv

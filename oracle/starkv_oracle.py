@@ -440,7 +440,9 @@ def attend_latents(cfg: Config, z_k, z_v, q, q_pos, B_k, B_v, heads=None):
 
 def decode(cache: Cache, q, B_k, B_v, block_table, seq_lens, seqs=None, heads=None):
     """starkv_decode_attn: each sequence's single query, at position seq_len - 1,
-    attends to positions [0, seq_len) of the quantised cache.
+    attends to positions [0, seq_len) of the quantised cache.  A sequence with
+    no tokens (seq_len 0) has nothing to attend to; the boundary defines its
+    output row as zeros.
 
     Returns o [B, H, d_h] fp64 (NaN where not requested by ``seqs``/``heads``).
     """
@@ -451,6 +453,9 @@ def decode(cache: Cache, q, B_k, B_v, block_table, seq_lens, seqs=None, heads=No
     heads = list(range(cfg.H)) if heads is None else list(heads)
     for b in (range(Bn) if seqs is None else seqs):
         n = int(seq_lens[b])
+        if n == 0:
+            out[b, heads] = 0.0
+            continue
         zk, zv = gather_sequence(cache, block_table[b], n)
         zk = unrotate_fp64(zk, cfg.key.g)
         zv = unrotate_fp64(zv, cfg.val.g)

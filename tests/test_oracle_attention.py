@@ -191,3 +191,12 @@ def test_quantised_attention_close_to_unquantised():
     ref = O.attend_latents(cfg, zk, zv, q, [255], f.B_k, f.B_v)
     rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     assert rel < 0.2
+
+
+def test_empty_sequence_decodes_to_zero_row():
+    w = gen.workload(0)
+    cfg = O.config_of(w)
+    f = gen.make_factors(w)
+    cache = O.new_cache(cfg, 1)
+    q = gen.make_queries(1, w.H, w.d_h)
+    assert np.all(O.decode(cache, q, f.B_k, f.B_v, np.zeros((1, 1), np.int32), [0]) == 0)

@@ -210,6 +210,27 @@ STARKV_API starkv_status starkv_decode_attn(starkv_ctx* ctx, const starkv_cache*
                                  int32_t batch, int32_t max_pages, void* out, void* workspace,
                                  size_t workspace_bytes, starkv_stream_t stream);
 
+/* Decode without any device allocation: the same computation and arguments as
+ * starkv_decode_attn, minus the workspace.  (The paper has no counterpart; this
+ * is a deployment variant.)  It is meant for callers that cannot call
+ * cudaMalloc, for example a plugin running inside a serving engine that owns
+ * the whole device memory pool, or a latency-critical loop that must never
+ * enter the allocator.  The split partials live in a built-in 16 MiB scratch
+ * array that every GPU loading this library holds until the process exits;
+ * the call itself allocates nothing.  The first call on a device looks up that
+ * array's device address (once per device, with the device current); make this
+ * first call before any stream capture.  All calls on a device share the
+ * scratch, so calls that overlap on the GPU (other streams, other contexts on
+ * the same device) race; serialise them.  A shape whose partials exceed the
+ * scratch (batch * num_q_heads * splits * (rank_v + 2) * 4 bytes > 16 MiB) is
+ * rejected with STARKV_ERR_UNSUPPORTED_SHAPE before anything is launched.
+ * Errors: as starkv_decode_attn, plus UNSUPPORTED_SHAPE for oversize shapes. */
+STARKV_API starkv_status starkv_decode_attn_noalloc(starkv_ctx* ctx, const starkv_cache* cache,
+                                                    const void* q, const int32_t* block_table,
+                                                    const int32_t* seq_lens, int32_t batch,
+                                                    int32_t max_pages, void* out,
+                                                    starkv_stream_t stream);
+
 /* Causal chunk attention over the packed cache (the chunked form of the same
  * dataflow).  q: device bf16 [total_q][num_q_heads][head_dim], pre-RoPE, rows of
  * sequence b at cu_q[b] .. cu_q[b+1]-1 (cu_q: device int32 [batch+1], cu_q[0]=0,

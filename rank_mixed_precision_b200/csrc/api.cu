@@ -265,6 +265,32 @@ starkv_status starkv_decode_attn(starkv_ctx* ctx, const starkv_cache* cache, con
   return ok();
 }
 
+starkv_status starkv_decode_attn_noalloc(starkv_ctx* ctx, const starkv_cache* cache, const void* q,
+                                         const int32_t* block_table, const int32_t* seq_lens, int32_t batch,
+                                         int32_t max_pages, void* out, starkv_stream_t stream) {
+  if (!ctx) return fail(STARKV_ERR_INVALID_ARG, "ctx is NULL");
+  Ctx* c = reinterpret_cast<Ctx*>(ctx);
+  starkv_status st = check_cache(c, cache);
+  if (st) return st;
+  if (batch < 0 || max_pages < 0) return fail(STARKV_ERR_INVALID_ARG, "negative size");
+  if (batch == 0) return ok();
+  if (max_pages == 0) return fail(STARKV_ERR_INVALID_ARG, "max_pages must be >= 1");
+  if (!q || !block_table || !seq_lens || !out) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
+  const DecodePlan plan = plan_decode(*c, batch, max_pages);
+  if (plan.ws_bytes > kNoAllocScratchBytes)
+    return fail(STARKV_ERR_UNSUPPORTED_SHAPE,
+                "decode of %d sequences x %d pages needs %zu scratch bytes; the built-in scratch holds %zu "
+                "(use starkv_decode_attn with a caller workspace)",
+                batch, max_pages, plan.ws_bytes, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "built-in scratch lookup (cudaGetSymbolAddress)");
+  e = launch_decode(*c, *cache, (const __nv_bfloat16*)q, block_table, seq_lens, batch, max_pages,
+                    (__nv_bfloat16*)out, scratch, plan, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return ok();
+}
+
 starkv_status starkv_prefill_attn(starkv_ctx* ctx, const starkv_cache* cache, const void* q, const int32_t* cu_q,
                                   const int32_t* block_table, const int32_t* seq_lens, int32_t batch,
                                   int32_t max_pages, int64_t total_q, int32_t max_q_len, void* out,

@@ -16,6 +16,8 @@
 // and the dot product.
 #include <float.h>
 
+#include <mutex>
+
 #include "internal.cuh"
 
 namespace starkv {
@@ -338,6 +340,46 @@ cudaError_t launch_decode(const Ctx& c, const starkv_cache& cache, const __nv_bf
   }
   decode_merge_kernel<<<dim3(a.H, batch), kDecThreads, msmem, s>>>(a);
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Built-in scratch for starkv_decode_attn_noalloc.
+//
+// Some callers cannot allocate device memory (for example a plugin inside a
+// serving engine that owns the whole memory pool, or a latency-critical loop
+// that must never enter the allocator).  For them, the decode's split partials
+// live in this file-scope array instead of a caller workspace.  Every GPU that
+// loads the library holds these bytes until the process exits.  All calls on a
+// device share the array and it keeps the last call's contents; nothing in it
+// needs to start at zero, because the split kernel writes every partial that
+// the merge kernel reads in the same call.  Calls that overlap on the GPU
+// (other streams, other contexts on the same device) race on it.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+}  // namespace
+
+// Device address of the built-in scratch on the current device.  The first call
+// on a device looks it up (cudaGetSymbolAddress, with that device current) and
+// caches it; host code must never pass the array's own name to a kernel.
+cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace starkv

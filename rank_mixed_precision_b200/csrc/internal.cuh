@@ -211,6 +211,10 @@ cudaError_t launch_decode(const Ctx& c, const starkv_cache& cache, const __nv_bf
                           int max_pages, __nv_bfloat16* out, void* ws, const DecodePlan& plan,
                           cudaStream_t s);
 
+// Built-in scratch of starkv_decode_attn_noalloc (see decode.cu).
+constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;  // 16 MiB
+cudaError_t noalloc_scratch(void** out);
+
 struct PrefillPlan {
   int chunk;          // key positions expanded per pass
   size_t ws_bytes;

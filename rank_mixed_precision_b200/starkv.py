@@ -25,6 +25,7 @@ LATENT_KEY, LATENT_VALUE = 0, 1
 EXPORTS = [
     "starkv_version", "starkv_last_error", "starkv_cache_layout", "starkv_create", "starkv_destroy",
     "starkv_get_config", "starkv_append", "starkv_workspace_bytes", "starkv_decode_attn",
+    "starkv_decode_attn_noalloc",
     "starkv_prefill_attn", "starkv_quantize_pack", "starkv_dequantize", "starkv_read_device_status",
 ]
 
@@ -70,6 +71,7 @@ _SIGS = {
     "starkv_append": ([_vp, ctypes.POINTER(starkv_cache), _vp, _vp, _i64, _vp, _vp], _i32),
     "starkv_workspace_bytes": ([_vp, _i32, _i32, _i32, _i64, ctypes.POINTER(_sz)], _i32),
     "starkv_decode_attn": ([_vp, ctypes.POINTER(starkv_cache), _vp, _vp, _vp, _i32, _i32, _vp, _vp, _sz, _vp], _i32),
+    "starkv_decode_attn_noalloc": ([_vp, ctypes.POINTER(starkv_cache), _vp, _vp, _vp, _i32, _i32, _vp, _vp], _i32),
     "starkv_prefill_attn": ([_vp, ctypes.POINTER(starkv_cache), _vp, _vp, _vp, _vp, _i32, _i32, _i64, _i32, _vp,
                              _vp, _sz, _vp], _i32),
     "starkv_quantize_pack": ([_vp, _i32, _vp, _i64, _vp, _vp, _vp], _i32),
@@ -198,6 +200,20 @@ def starkv_decode_attn(ctx, cache: starkv_cache, q, block_table, seq_lens, out, 
     _check(lib().starkv_decode_attn(ctx, ctypes.byref(cache), _p(q), _p(block_table), _p(seq_lens), B,
                                     block_table.shape[1], _p(out), _p(workspace), workspace.numel(),
                                     _stream(stream)))
+
+
+def starkv_decode_attn_noalloc(ctx, cache: starkv_cache, q, block_table, seq_lens, out, stream=None):
+    """Decode with the library's built-in scratch instead of a caller workspace
+    (for callers that cannot allocate device memory; see include/starkv.h)."""
+    _need(q, torch.bfloat16, "q", 3)
+    _need(block_table, torch.int32, "block_table", 2)
+    _need(seq_lens, torch.int32, "seq_lens", 1)
+    _need(out, torch.bfloat16, "out", 3)
+    B = q.shape[0]
+    if block_table.shape[0] != B or seq_lens.shape[0] != B or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q / block_table / seq_lens / out disagree on the batch")
+    _check(lib().starkv_decode_attn_noalloc(ctx, ctypes.byref(cache), _p(q), _p(block_table), _p(seq_lens), B,
+                                            block_table.shape[1], _p(out), _stream(stream)))
 
 
 def starkv_prefill_attn(ctx, cache: starkv_cache, q, cu_q, block_table, seq_lens, max_q_len, out, workspace,

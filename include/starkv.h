@@ -72,8 +72,11 @@ enum {
   STARKV_DEV_QUANT_OVERFLOW = 1u << 2,/* a group's fp16 scale/zero not finite, or
                                         a non-finite latent                     */
   STARKV_DEV_BAD_SLOT = 1u << 3,     /* append slot >= n_pages*16                */
-  STARKV_DEV_BAD_QUERY_SPAN = 1u << 4/* prefill: cu_q not non-decreasing, or a
+  STARKV_DEV_BAD_QUERY_SPAN = 1u << 4,/* prefill: cu_q not non-decreasing, or a
                                         sequence's query count > its seq_len    */
+  STARKV_DEV_WAIT_TIMEOUT = 1u << 5  /* a pipelined kernel gave up waiting on one
+                                        of its own stages (bounded wait); its
+                                        outputs for that call are not valid    */
 };
 
 /* Opaque stream handle: pass a cudaStream_t. */

@@ -4,6 +4,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <stdlib.h>
+
 #include <new>
 #include <vector>
 
@@ -90,6 +92,29 @@ starkv_status check_config(const starkv_config* c, LatentGeom* key, LatentGeom* 
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// TMA map of the fp16 cos/sin table [max_position][d]: 64-column x 128-row boxes,
+// 128-byte swizzle (the tensor-core operand layout), zero fill past the last row.
+bool make_trig_map(Ctx* c) {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess || !fn ||
+      q != cudaDriverEntryPointSuccess)
+    return false;
+  const int d = c->cfg.head_dim;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)c->cfg.max_position};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = ((EncodeTiledFn)fn)(&c->trig_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->trig, dims, strides, box, es,
+                                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 starkv_status check_cache(const Ctx* c, const starkv_cache* cache) {
   if (!cache) return fail(STARKV_ERR_INVALID_ARG, "cache is NULL");
   if (cache->n_pages < 0) return fail(STARKV_ERR_INVALID_ARG, "cache.n_pages < 0");
@@ -153,17 +178,21 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
   const size_t bk_bytes = (size_t)cfg->num_kv_heads * cfg->rank_k * d * 4;
   const size_t bv_bytes = (size_t)cfg->rank_v * cfg->num_kv_heads * d * 4;
   const size_t rope_bytes = (size_t)cfg->max_position * half * sizeof(float2);
+  const size_t trig_bytes = (size_t)cfg->max_position * d * sizeof(__half);
   cudaError_t e;
   auto cleanup = [&]() {
     cudaFree(c->A);
     cudaFree(c->Bk);
     cudaFree(c->Bv);
     cudaFree(c->rope);
+    cudaFree(c->trig);
+    cudaFree(c->Bv16);
     cudaFree(c->status);
     delete c;
   };
   if ((e = cudaMalloc(&c->A, a_bytes)) != cudaSuccess || (e = cudaMalloc(&c->Bk, bk_bytes)) != cudaSuccess ||
       (e = cudaMalloc(&c->Bv, bv_bytes)) != cudaSuccess || (e = cudaMalloc(&c->rope, rope_bytes)) != cudaSuccess ||
+      (e = cudaMalloc(&c->trig, trig_bytes)) != cudaSuccess || (e = cudaMalloc(&c->Bv16, bv_bytes / 2)) != cudaSuccess ||
       (e = cudaMalloc(&c->status, sizeof(unsigned int))) != cudaSuccess) {
     cleanup();
     return cuda_fail(e, "cudaMalloc (context factors)");
@@ -175,22 +204,32 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
     e = cudaMemcpy2DAsync((char*)c->A + kcols * 2, c->lat_cols * 2, A_v, (size_t)cfg->rank_v * 2,
                           (size_t)cfg->rank_v * 2, cfg->hidden, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = launch_prepare_factors(*c, (const __nv_bfloat16*)B_k, (const __nv_bfloat16*)B_v, s);
+  if (e == cudaSuccess) e = launch_prepare_tc_factors(*c, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->status, 0, sizeof(unsigned int), s);
   // RoPE table: angle p * base^(-2i/d) in fp64, cos/sin in fp64, stored as fp32
+  // and the same angles as an fp16 [cos.. | sin..] row per position (tensor-core operand)
   std::vector<float2> rope((size_t)cfg->max_position * half);
+  std::vector<__half> trig((size_t)cfg->max_position * d);
   std::vector<double> theta(half);
   for (int i = 0; i < half; ++i) theta[i] = pow(cfg->rope_base, -2.0 * i / d);
   for (int p = 0; p < cfg->max_position; ++p)
     for (int i = 0; i < half; ++i) {
       const double ang = (double)p * theta[i];
-      rope[(size_t)p * half + i] = make_float2((float)cos(ang), (float)sin(ang));
+      const double cv = cos(ang), sv = sin(ang);
+      rope[(size_t)p * half + i] = make_float2((float)cv, (float)sv);
+      trig[(size_t)p * d + i] = __float2half_rn((float)cv);
+      trig[(size_t)p * d + half + i] = __float2half_rn((float)sv);
     }
   if (e == cudaSuccess) e = cudaMemcpyAsync(c->rope, rope.data(), rope_bytes, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->trig, trig.data(), trig_bytes, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     cleanup();
     return cuda_fail(e, "starkv_create");
   }
+  const char* path = getenv("STARKV_DECODE_PATH");
+  const bool want_simt = path && strcmp(path, "simt") == 0;
+  c->tc = !want_simt && tc_decode_supported(c->cfg) && c->val.g >= 8 && make_trig_map(c);
   *out = reinterpret_cast<starkv_ctx*>(c);
   return ok();
 }
@@ -203,6 +242,8 @@ starkv_status starkv_destroy(starkv_ctx* ctx) {
   cudaFree(c->Bk);
   cudaFree(c->Bv);
   cudaFree(c->rope);
+  cudaFree(c->trig);
+  cudaFree(c->Bv16);
   cudaFree(c->status);
   delete c;
   return ok();

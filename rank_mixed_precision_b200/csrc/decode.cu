@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_merge_kernel(DecodeArgs a)
   }
 }
 
-DecodePlan plan_decode(const Ctx& c, int batch, int max_pages) {
+DecodePlan plan_decode_simt(const Ctx& c, int batch, int max_pages) {
   DecodePlan p;
   const int H = c.cfg.num_q_heads;
   // enough CTAs for a few waves on 148 SMs, at least 256 tokens per split
@@ -272,10 +272,10 @@ DecodePlan plan_decode(const Ctx& c, int batch, int max_pages) {
   return p;
 }
 
-cudaError_t launch_decode(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
-                          const int32_t* block_table, const int32_t* seq_lens, int batch,
-                          int max_pages, __nv_bfloat16* out, void* ws, const DecodePlan& plan,
-                          cudaStream_t s) {
+cudaError_t launch_decode_simt(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
+                               const int32_t* block_table, const int32_t* seq_lens, int batch,
+                               int max_pages, __nv_bfloat16* out, void* ws, const DecodePlan& plan,
+                               cudaStream_t s) {
   if (batch == 0) return cudaSuccess;
   DecodeArgs a;
   a.key = c.key;
@@ -340,6 +340,22 @@ cudaError_t launch_decode(const Ctx& c, const starkv_cache& cache, const __nv_bf
   }
   decode_merge_kernel<<<dim3(a.H, batch), kDecThreads, msmem, s>>>(a);
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Path selection: the tensor-core kernels (decode_tc.cu) for every shape they
+// cover, the CUDA-core kernels above otherwise.
+// ---------------------------------------------------------------------------
+DecodePlan plan_decode(const Ctx& c, int batch, int max_pages) {
+  return c.tc ? plan_decode_tc(c, batch, max_pages) : plan_decode_simt(c, batch, max_pages);
+}
+
+cudaError_t launch_decode(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
+                          const int32_t* block_table, const int32_t* seq_lens, int batch,
+                          int max_pages, __nv_bfloat16* out, void* ws, const DecodePlan& plan,
+                          cudaStream_t s) {
+  if (c.tc) return launch_decode_tc(c, cache, q, block_table, seq_lens, batch, max_pages, out, ws, plan, s);
+  return launch_decode_simt(c, cache, q, block_table, seq_lens, batch, max_pages, out, ws, plan, s);
 }
 
 // ---------------------------------------------------------------------------

@@ -1,6 +1,7 @@
 // Internal definitions shared by the library's CUDA sources.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -39,8 +40,15 @@ struct Ctx {
   float* Bk;              // [h_kv][r_k][d_h]  fp32, B'_k = H B_k (rotation folded)
   float* Bv;              // [R][h_kv*d_h]     fp32, B'_v = H B_v
   float2* rope;           // [max_position][d_h/2] (cos, sin), built in fp64
+  __half* trig;           // [max_position][d_h] fp16: cos(p th_0..), sin(p th_0..) (tensor-core operand)
+  __half* Bv16;           // [R][h_kv*d_h] fp16, B'_v
   unsigned int* status;   // device status word
+  CUtensorMap trig_map;   // TMA map of `trig`: box 64 x 128, 128-byte swizzle
+  bool tc;                // tensor-core decode available for this shape
 };
+
+// Extra device status bit: a pipeline wait in a tensor-core kernel gave up.
+constexpr unsigned int kDevWaitTimeout = STARKV_DEV_WAIT_TIMEOUT;
 
 // ---------------------------------------------------------------------------
 // Device helpers
@@ -206,6 +214,17 @@ struct DecodePlan {
   size_t ws_bytes;
 };
 DecodePlan plan_decode(const Ctx& c, int batch, int max_pages);
+DecodePlan plan_decode_simt(const Ctx& c, int batch, int max_pages);
+cudaError_t launch_decode_simt(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
+                               const int32_t* block_table, const int32_t* seq_lens, int batch, int max_pages,
+                               __nv_bfloat16* out, void* ws, const DecodePlan& plan, cudaStream_t s);
+// tensor-core decode (decode_tc.cu)
+bool tc_decode_supported(const starkv_config& cfg);
+DecodePlan plan_decode_tc(const Ctx& c, int batch, int max_pages);
+cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
+                             const int32_t* block_table, const int32_t* seq_lens, int batch, int max_pages,
+                             __nv_bfloat16* out, void* ws, const DecodePlan& plan, cudaStream_t s);
+cudaError_t launch_prepare_tc_factors(const Ctx& c, cudaStream_t s);
 cudaError_t launch_decode(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
                           const int32_t* block_table, const int32_t* seq_lens, int batch,
                           int max_pages, __nv_bfloat16* out, void* ws, const DecodePlan& plan,

@@ -46,7 +46,7 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 
 // Wait for phase `parity` to complete, giving up after `limit` polls.
 // Returns false on time-out (the caller records the failure and bails out).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = (1u << 26)) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = (1u << 22)) {
   for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_test(bar, parity)) return true;
   }

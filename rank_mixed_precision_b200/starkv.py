@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libstarkv.s
 
 PAGE_TOKENS = 16
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_WORKSPACE_TOO_SMALL, ERR_CUDA, ERR_DEVICE_STATUS = range(6)
-DEV_BAD_PAGE, DEV_BAD_SEQ_LEN, DEV_QUANT_OVERFLOW, DEV_BAD_SLOT, DEV_BAD_QUERY_SPAN = 1, 2, 4, 8, 16
+DEV_BAD_PAGE, DEV_BAD_SEQ_LEN, DEV_QUANT_OVERFLOW, DEV_BAD_SLOT, DEV_BAD_QUERY_SPAN, DEV_WAIT_TIMEOUT = 1, 2, 4, 8, 16, 32
 OP_DECODE, OP_PREFILL = 0, 1
 LATENT_KEY, LATENT_VALUE = 0, 1
 

@@ -63,6 +63,15 @@ def test_llama3_gqa_shapes_small():
     check_attention(got, ref, "llama3 gqa small")
 
 
+def test_cuda_core_path_longchat_shapes(monkeypatch):
+    # the CUDA-core kernels remain the path for shapes the tensor-core kernels do not cover
+    monkeypatch.setenv("STARKV_DECODE_PATH", "simt")
+    w = gen.workload(1)
+    got, ref, st = run_decode(w, [1, 33, 300])
+    assert st == 0
+    check_attention(got, ref, "longchat small, cuda-core path")
+
+
 def test_page_table_with_spare_capacity():
     # block tables longer than the sequences (the decode step's usual state)
     w = gen.workload(1)

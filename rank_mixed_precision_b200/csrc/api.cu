@@ -99,20 +99,9 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 // TMA map of the fp16 cos/sin table [max_position][d]: 64-column x 128-row boxes,
 // 128-byte swizzle (the tensor-core operand layout), zero fill past the last row.
 bool make_trig_map(Ctx* c) {
-  void* fn = nullptr;
-  cudaDriverEntryPointQueryResult q;
-  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess || !fn ||
-      q != cudaDriverEntryPointSuccess)
-    return false;
   const int d = c->cfg.head_dim;
-  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)c->cfg.max_position};
-  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t es[2] = {1, 1};
-  CUresult r = ((EncodeTiledFn)fn)(&c->trig_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->trig, dims, strides, box, es,
-                                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return starkv::encode_map_2d(&c->trig_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, c->trig, (uint64_t)d,
+                               (uint64_t)c->cfg.max_position, (uint64_t)d * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 starkv_status check_cache(const Ctx* c, const starkv_cache* cache) {
@@ -128,6 +117,27 @@ starkv_status check_cache(const Ctx* c, const starkv_cache* cache) {
 }
 
 }  // namespace
+
+namespace starkv {
+bool encode_map_2d(CUtensorMap* map, CUtensorMapDataType type, void* base, uint64_t inner, uint64_t rows,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess || !f ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    fn = (EncodeTiledFn)f;
+  }
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, type, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace starkv
 
 extern "C" {
 
@@ -187,12 +197,14 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
     cudaFree(c->rope);
     cudaFree(c->trig);
     cudaFree(c->Bv16);
+    cudaFree(c->zacc);
     cudaFree(c->status);
     delete c;
   };
   if ((e = cudaMalloc(&c->A, a_bytes)) != cudaSuccess || (e = cudaMalloc(&c->Bk, bk_bytes)) != cudaSuccess ||
       (e = cudaMalloc(&c->Bv, bv_bytes)) != cudaSuccess || (e = cudaMalloc(&c->rope, rope_bytes)) != cudaSuccess ||
       (e = cudaMalloc(&c->trig, trig_bytes)) != cudaSuccess || (e = cudaMalloc(&c->Bv16, bv_bytes / 2)) != cudaSuccess ||
+      (e = cudaMalloc(&c->zacc, (size_t)kSmallAppend * c->lat_cols * 4)) != cudaSuccess ||
       (e = cudaMalloc(&c->status, sizeof(unsigned int))) != cudaSuccess) {
     cleanup();
     return cuda_fail(e, "cudaMalloc (context factors)");
@@ -206,6 +218,7 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
   if (e == cudaSuccess) e = launch_prepare_factors(*c, (const __nv_bfloat16*)B_k, (const __nv_bfloat16*)B_v, s);
   if (e == cudaSuccess) e = launch_prepare_tc_factors(*c, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->status, 0, sizeof(unsigned int), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->zacc, 0, (size_t)kSmallAppend * c->lat_cols * 4, s);
   // RoPE table: angle p * base^(-2i/d) in fp64, cos/sin in fp64, stored as fp32
   // and the same angles as an fp16 [cos.. | sin..] row per position (tensor-core operand)
   std::vector<float2> rope((size_t)cfg->max_position * half);
@@ -229,7 +242,7 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
   }
   const char* path = getenv("STARKV_DECODE_PATH");
   const bool want_simt = path && strcmp(path, "simt") == 0;
-  c->tc = !want_simt && tc_decode_supported(c->cfg) && c->val.g >= 8 && make_trig_map(c);
+  c->tc = !want_simt && tc_decode_supported(c->cfg) && c->val.g == 16 && make_trig_map(c);
   *out = reinterpret_cast<starkv_ctx*>(c);
   return ok();
 }
@@ -244,6 +257,7 @@ starkv_status starkv_destroy(starkv_ctx* ctx) {
   cudaFree(c->rope);
   cudaFree(c->trig);
   cudaFree(c->Bv16);
+  cudaFree(c->zacc);
   cudaFree(c->status);
   delete c;
   return ok();
@@ -392,6 +406,7 @@ starkv_status starkv_read_device_status(starkv_ctx* ctx, starkv_stream_t stream,
   unsigned int h = 0;
   cudaError_t e = cudaMemcpyAsync(&h, c->status, sizeof(h), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->status, 0, sizeof(unsigned int), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->zacc, 0, (size_t)kSmallAppend * c->lat_cols * 4, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "read_device_status");
   *status = h;

@@ -33,18 +33,21 @@ using namespace sm100;
 namespace {
 constexpr int kT = 128;                 // tokens per key tile (MMA M)
 constexpr int kPagesPerTile = kT / kPage;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;
 constexpr int kAThreads = (2 + kEpiWarps) * 32;
 constexpr int kVT = 64;                 // tokens per value stage
 constexpr int kVPages = kVT / kPage;
-constexpr int kVStages = 3;
+constexpr int kVStages = 2;
 constexpr int kZBufs = 4;
-constexpr int kVWarps = 8;
+constexpr int kVWarps = 16;
 constexpr int kBThreads = (2 + kVWarps) * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
+// 1024-byte aligned base inside the dynamic shared-memory array.  The offset is
+// added to the __shared__ array itself so the compiler keeps the shared state
+// space (plain shared loads/stores instead of generic ones).
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+  return p + ((1024u - (sm100::smem_u32(p) & 1023u)) & 1023u);
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -72,17 +75,95 @@ struct ScoreArgs {
   const float2* rope;  // [max_position][d/2]
   float* S;            // [B][H][tpad]      scores, log2 domain
   float* Smax;         // [B][H][tpad/32]   maxima of 32-token blocks
-  float* acc;          // [B][H][R] zeroed here for kernel B
-  float* lsum;         // [B][H]    zeroed here
-  int64_t acc_elems;   // B * H * R
-  int64_t lsum_elems;  // B * H
+  float* oacc;         // [B][H][d] zeroed here for the projection
+  unsigned int* ocnt;  // [H][ceil(B/16)] zeroed here
+  int64_t oacc_elems;  // B * H * d
+  int ocnt_elems;
+  const uint8_t* wimg; // [B][HG][ncols * d * 2] W in its shared-memory image
   unsigned int* status;
-  uint32_t off_trig, off_codes, off_meta, off_flags, off_q, off_bar;
-  uint32_t trig_stage, codes_page, meta_page, codes_stage, meta_stage;
+  uint32_t off_trig, off_codes, off_meta, off_flags, off_bt, off_bar;
+  uint32_t trig_stage, codes_page, meta_page, codes_stage, meta_stage, w_bytes;
+  uint32_t codes_pitch, meta_pitch;  // shared-memory page strides (padded against bank conflicts)
 };
+
+// ---------------------------------------------------------------------------
+// W prep: one CTA per (sequence, head), thread i owns the frequency pair
+// (i, i + d/2) for every latent channel c:
+//   W[c][i]       = (q~_i B'[c,i] + q~_{i+d/2} B'[c,i+d/2]) * log2(e)/sqrt(d)
+//   W[c][i + d/2] = (q~_{i+d/2} B'[c,i] - q~_i B'[c,i+d/2]) * log2(e)/sqrt(d)
+// with q~ the query rotated to its position.  Written as fp16 directly in the
+// score kernel's shared-memory image (K-major, 128-byte swizzle).
+// ---------------------------------------------------------------------------
+template <int RK>
+__global__ void __launch_bounds__(64) decode_wprep_kernel(const __nv_bfloat16* __restrict__ q,
+                                                          const int32_t* __restrict__ seq_lens,
+                                                          const float* __restrict__ Bk, const float2* __restrict__ rope,
+                                                          uint8_t* __restrict__ wimg, int H, int group, int d, int hpc,
+                                                          int ncols, int max_pages, int max_position) {
+  const int h = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
+  const int half = d / 2;
+  if (i >= half) return;
+  int L = seq_lens[b];
+  if (L <= 0 || L > max_pages * kPage || L > max_position) L = 1;  // unused (no tiles), keep reads in range
+  const int kv = h / group, hg = h / hpc, hl = h % hpc;
+  const float2 cs = rope[(int64_t)(L - 1) * half + i];
+  const __nv_bfloat16* qv = q + ((int64_t)b * H + h) * d;
+  const float scale = kLog2e * rsqrtf((float)d);
+  const float x0 = __bfloat162float(qv[i]), x1 = __bfloat162float(qv[i + half]);
+  const float qa = (x0 * cs.x - x1 * cs.y) * scale;
+  const float qb = (x1 * cs.x + x0 * cs.y) * scale;
+  const float* B = Bk + (int64_t)kv * RK * d;
+  float ba[RK], bb[RK];
+#pragma unroll
+  for (int c = 0; c < RK; ++c) {
+    ba[c] = B[c * d + i];
+    bb[c] = B[c * d + i + half];
+  }
+  uint8_t* img = wimg + ((int64_t)b * (H / hpc) + hg) * ((int64_t)ncols * d * 2);
+#pragma unroll
+  for (int c = 0; c < RK; ++c) {
+    const int n = hl * RK + c;
+    *reinterpret_cast<__half*>(img + sw128_kmajor_offset(n, i, ncols)) = __float2half_rn(fmaf(qa, ba[c], qb * bb[c]));
+    *reinterpret_cast<__half*>(img + sw128_kmajor_offset(n, i + half, ncols)) =
+        __float2half_rn(fmaf(qb, ba[c], -qa * bb[c]));
+  }
+}
 
 // TMEM columns of the score accumulators: two buffers of up to 256 columns.
 constexpr uint32_t kScoreTmemCols = 512;
+
+// Issue the TMEM loads of one RK-column row into raw registers (no wait).
+template <int RK>
+__device__ __forceinline__ void tmem_issue_row(uint32_t taddr, uint32_t (&r)[RK]) {
+  if constexpr (RK == 16) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+  } else {
+#pragma unroll
+    for (int h = 0; h < RK / 32; ++h) {
+      uint32_t(&rr)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[h * 32]);
+      tmem_ld32(taddr + h * 32, rr);
+    }
+  }
+}
+
+// Wait for the row's TMEM loads; the registers pass through the wait so no use
+// of them can be scheduled before it.
+template <int RK>
+__device__ __forceinline__ void tmem_wait_row(uint32_t (&r)[RK]) {
+#pragma unroll
+  for (int q = 0; q < RK; q += 16) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[q + 0]), "+r"(r[q + 1]), "+r"(r[q + 2]), "+r"(r[q + 3]), "+r"(r[q + 4]), "+r"(r[q + 5]),
+                   "+r"(r[q + 6]), "+r"(r[q + 7]), "+r"(r[q + 8]), "+r"(r[q + 9]), "+r"(r[q + 10]), "+r"(r[q + 11]),
+                   "+r"(r[q + 12]), "+r"(r[q + 13]), "+r"(r[q + 14]), "+r"(r[q + 15])
+                 :
+                 : "memory");
+  }
+}
 
 template <int RK>
 __device__ __forceinline__ void tmem_load_row(uint32_t taddr, float (&G)[RK]) {
@@ -107,26 +188,139 @@ __device__ __forceinline__ void tmem_load_row(uint32_t taddr, float (&G)[RK]) {
   }
 }
 
-// sum_c z_hat_c G_c over one token's key latent in a staged page region.
-template <int RK>
-__device__ __forceinline__ float key_dot(const uint8_t* region, const uint32_t* meta, const LatentGeom& L, int t16,
-                                         const float (&G)[RK]) {
-  float score = 0.f;
-  const int g = L.g;
-  for (int gi = 0; gi < L.groups; ++gi) {
-    const float2 sz = unpack_meta(meta[gi * kPage + t16]);
-    float a = 0.f, gs = 0.f;
-    for (int c = 0; c < g; ++c) {
-      const float Gc = G[gi * g + c];
-      a = fmaf((float)load_code(region, L, gi, t16, c), Gc, a);
-      gs += Gc;
+// ---------------------------------------------------------------------------
+// Key dot product on packed codes (one token, one head), compile-time layout.
+//
+// Codes become floats by writing their bits into the mantissa of 1.0:
+// x = 1 + code / 2^k exactly (k = 4 for a 4-bit nibble; for 3-bit codes the
+// 2-bit low plane gives 1 + lo/4 and the high bit 1 + hi/2).  With
+// gs = sum_c G_c over the group:
+//   4-bit:  sum_c code_c G_c = 16 (sum_c x_c G_c - gs)
+//   3-bit:  sum_c code_c G_c = 4 sum_c xlo_c G_c + 8 sum_c xhi_c G_c - 12 gs
+// and the group's contribution is s * sum code G + zp * gs.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float mant(uint32_t bits) { return __uint_as_float(0x3F800000u | bits); }
+
+// field of `width` bits at bit `pos` of w, moved to mantissa bits [23 - width, 23)
+template <int POS, int WIDTH>
+__device__ __forceinline__ float field_as_unit(uint32_t w) {
+  constexpr int dst = 23 - WIDTH;
+  constexpr uint32_t mask = ((1u << WIDTH) - 1u) << dst;
+  if constexpr (POS <= dst) return mant((w << (dst - POS)) & mask);
+  else return mant((w >> (POS - dst)) & mask);
+}
+
+// Packed fp32 pairs (sm_100a f32x2 arithmetic: two lanes of fp32 per instruction).
+typedef unsigned long long f32x2_t;
+__device__ __forceinline__ f32x2_t pk2(float x, float y) {
+  f32x2_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+  return r;
+}
+__device__ __forceinline__ float2 upk2(f32x2_t r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+__device__ __forceinline__ f32x2_t ffma2(f32x2_t a, f32x2_t b, f32x2_t c) {
+  f32x2_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2_t fadd2(f32x2_t a, f32x2_t b) {
+  f32x2_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float hsum2(f32x2_t r) {
+  const float2 v = upk2(r);
+  return v.x + v.y;
+}
+
+template <int G>
+struct KeyGroup {
+  // 4-bit tile: token t16's G nibbles; 3-bit tile: its 2-bit and 1-bit planes
+  __device__ __forceinline__ static float dot4(const uint8_t* tile, int t16, const float* Gv, float& gs) {
+    f32x2_t a2 = 0ull, g2 = 0ull;
+    if constexpr (G == 4) {
+      const uint32_t w = *reinterpret_cast<const uint16_t*>(tile + 2 * t16);
+#pragma unroll
+      for (int c = 0; c < 4; c += 2) {
+        const f32x2_t gp = pk2(Gv[c], Gv[c + 1]);
+        a2 = ffma2(pk2(field_as_unit<0, 4>(w >> (4 * c)), field_as_unit<0, 4>(w >> (4 * c + 4))), gp, a2);
+        g2 = fadd2(g2, gp);
+      }
+    } else {
+      const uint32_t* wp = reinterpret_cast<const uint32_t*>(tile + (G / 2) * t16);
+#pragma unroll
+      for (int q = 0; q < G / 8; ++q) {
+        const uint32_t w = wp[q];
+        const float* g8 = Gv + 8 * q;
+        f32x2_t gp = pk2(g8[0], g8[1]);
+        a2 = ffma2(pk2(field_as_unit<0, 4>(w), field_as_unit<4, 4>(w)), gp, a2);
+        g2 = fadd2(g2, gp);
+        gp = pk2(g8[2], g8[3]);
+        a2 = ffma2(pk2(field_as_unit<8, 4>(w), field_as_unit<12, 4>(w)), gp, a2);
+        g2 = fadd2(g2, gp);
+        gp = pk2(g8[4], g8[5]);
+        a2 = ffma2(pk2(field_as_unit<16, 4>(w), field_as_unit<20, 4>(w)), gp, a2);
+        g2 = fadd2(g2, gp);
+        gp = pk2(g8[6], g8[7]);
+        a2 = ffma2(pk2(field_as_unit<24, 4>(w), field_as_unit<28, 4>(w)), gp, a2);
+        g2 = fadd2(g2, gp);
+      }
     }
-    score = fmaf(sz.x, a, fmaf(sz.y, gs, score));
+    gs = hsum2(g2);
+    return 16.f * (hsum2(a2) - gs);
+  }
+  __device__ __forceinline__ static float dot3(const uint8_t* tile, int t16, const float* Gv, float& gs) {
+    uint32_t lo, hi;
+    if constexpr (G == 4) {
+      lo = tile[t16];
+      hi = (uint32_t)(tile[16 + (t16 >> 1)] >> ((t16 & 1) * 4));
+    } else if constexpr (G == 8) {
+      lo = *reinterpret_cast<const uint16_t*>(tile + 2 * t16);
+      hi = tile[32 + t16];
+    } else {
+      lo = *reinterpret_cast<const uint32_t*>(tile + 4 * t16);
+      hi = *reinterpret_cast<const uint16_t*>(tile + 64 + 2 * t16);
+    }
+    f32x2_t al = 0ull, ah = 0ull, g2 = 0ull;
+#pragma unroll
+    for (int c = 0; c < G; c += 2) {
+      const f32x2_t gp = pk2(Gv[c], Gv[c + 1]);
+      al = ffma2(pk2(field_as_unit<0, 2>(lo >> (2 * c)), field_as_unit<0, 2>(lo >> (2 * c + 2))), gp, al);
+      ah = ffma2(pk2(field_as_unit<0, 1>(hi >> c), field_as_unit<0, 1>(hi >> (c + 1))), gp, ah);
+      g2 = fadd2(g2, gp);
+    }
+    gs = hsum2(g2);
+    return 4.f * hsum2(al) + 8.f * hsum2(ah) - 12.f * gs;
+  }
+};
+
+// sum_c z_hat_c G_c over one token's key latent in a staged page region.
+template <int RK, int G>
+__device__ __forceinline__ float key_dot(const uint8_t* region, const uint32_t* meta, int top_groups, int t16,
+                                         const uint32_t (&raw)[RK]) {
+  const float* Gv = reinterpret_cast<const float*>(raw);
+  float score = 0.f;
+#pragma unroll
+  for (int gi = 0; gi < RK / G; ++gi) {
+    const uint32_t m = meta[gi * kPage + t16];
+    const float s = __half2float(__ushort_as_half((unsigned short)(m & 0xFFFF)));
+    const float zp = __half2float(__ushort_as_half((unsigned short)(m >> 16)));
+    float gs, cg;
+    if (gi < top_groups) {
+      cg = KeyGroup<G>::dot4(region + gi * 8 * G, t16, Gv + gi * G, gs);
+    } else {
+      cg = KeyGroup<G>::dot3(region + top_groups * 8 * G + (gi - top_groups) * 6 * G, t16, Gv + gi * G, gs);
+    }
+    score = fmaf(s, cg, fmaf(zp, gs, score));
   }
   return score;
 }
 
-template <int RK>
+template <int RK, int G>
 __global__ void __launch_bounds__(kAThreads, 1)
     decode_scores_kernel(const __grid_constant__ CUtensorMap trig_map, const ScoreArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -140,15 +334,15 @@ __global__ void __launch_bounds__(kAThreads, 1)
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 8);
   int* failed = reinterpret_cast<int*>(bar + 9);
   int* flags = reinterpret_cast<int*>(sm + a.off_flags);    // [2][8] page ids (-1 = invalid)
-  float* qbuf = reinterpret_cast<float*>(sm + a.off_q);     // [hpc][d]
+  int* bt_s = reinterpret_cast<int*>(sm + a.off_bt);        // this job's block-table entries
+  uint64_t* wbar = bar + 10;                                 // W image loaded
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int d = a.d, half = d / 2;
+  const int d = a.d;
 
-  // zero kernel B's accumulators (grid-stride over all CTAs)
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + tid; i < a.acc_elems; i += (int64_t)gridDim.x * blockDim.x)
-    a.acc[i] = 0.f;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + tid; i < a.lsum_elems; i += (int64_t)gridDim.x * blockDim.x)
-    a.lsum[i] = 0.f;
+  // zero the projection's sums and arrival counters (grid-stride over all CTAs)
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + tid; i < a.oacc_elems; i += (int64_t)gridDim.x * blockDim.x)
+    a.oacc[i] = 0.f;
+  for (int i = blockIdx.x * blockDim.x + tid; i < a.ocnt_elems; i += gridDim.x * blockDim.x) a.ocnt[i] = 0u;
 
   if (warp == 1) tmem_alloc(tslot, kScoreTmemCols);
   if (tid == 0) {
@@ -158,6 +352,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
       mbar_init(&tfull[s], 1);
       mbar_init(&tempty[s], kEpiWarps);
     }
+    mbar_init(wbar, 1);
     *failed = 0;
     fence_mbar_init();
   }
@@ -166,6 +361,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const uint32_t idesc = make_idesc_f16(128, a.ncols, false, false);
+  uint32_t jobs = 0;
 
   uint32_t it = 0;  // tiles through the pipeline so far (same count in every role)
   int item = blockIdx.x * a.items_per_cta;
@@ -185,33 +381,27 @@ __global__ void __launch_bounds__(kAThreads, 1)
     if (*failed) break;
     const int h0 = hg * a.hpc;
     const int kv0 = h0 / a.group;
-    // ---- W for this (sequence, head group): rotated query folded into B'
-    {
-      const int pos = L - 1;
-      const float scale = kLog2e * rsqrtf((float)d);
-      for (int e = tid; e < a.hpc * half; e += blockDim.x) {
-        const int hl = e / half, i = e % half;
-        const __nv_bfloat16* qv = a.q + ((int64_t)b * a.H + h0 + hl) * d;
-        const float2 cs = a.rope[(int64_t)pos * half + i];
-        const float x0 = __bfloat162float(qv[i]), x1 = __bfloat162float(qv[i + half]);
-        qbuf[hl * d + i] = (x0 * cs.x - x1 * cs.y) * scale;
-        qbuf[hl * d + i + half] = (x1 * cs.x + x0 * cs.y) * scale;
-      }
-      __syncthreads();
-      for (int e = tid; e < a.ncols * d; e += blockDim.x) {
-        const int n = e / d, k = e % d;
-        const int hl = n / RK, c = n % RK;
-        const int kv = (h0 + hl) / a.group;
-        const int i = k < half ? k : k - half;
-        const float* B = a.Bk + ((int64_t)kv * RK + c) * d;
-        const float ba = B[i], bb = B[i + half];
-        const float qa = qbuf[hl * d + i], qb = qbuf[hl * d + i + half];
-        const float w = k < half ? fmaf(qa, ba, qb * bb) : fmaf(qb, ba, -qa * bb);
-        *reinterpret_cast<__half*>(Wsm + sw128_kmajor_offset(n, k, a.ncols)) = __float2half_rn(w);
-      }
-      fence_async_smem();
-      __syncthreads();
+    // ---- W for this (sequence, head group): one bulk copy of its prepared image;
+    //      this job's page ids into shared memory (coalesced)
+    if (tid == 0) {
+      mbar_arrive_expect_tx(wbar, a.w_bytes);
+      bulk_g2s(Wsm, a.wimg + ((int64_t)b * a.HG + hg) * a.w_bytes, a.w_bytes, wbar);
     }
+    {
+      const int p0 = t0 * kPagesPerTile;
+      const int np_job = min((t1 - t0) * kPagesPerTile, (L + kPage - 1) / kPage - p0);
+      for (int e = tid; e < np_job; e += blockDim.x) bt_s[e] = a.block_table[(int64_t)b * a.max_pages + p0 + e];
+    }
+    __syncthreads();
+    if (!mbar_wait(wbar, jobs & 1)) {
+      if (tid == 0) {
+        set_status(a.status, kDevWaitTimeout);
+        *failed = 1;
+      }
+    }
+    ++jobs;
+    __syncthreads();
+    if (*failed) break;
     const int ntile = t1 - t0;
     if (warp == 0) {
       if (lane == 0) {
@@ -231,7 +421,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
           for (int p = 0; p < kPagesPerTile; ++p) {
             int pid = -1;
             if (p < np) {
-              pid = a.block_table[(int64_t)b * a.max_pages + j0 / kPage + p];
+              pid = bt_s[(j0 / kPage + p) - t0 * kPagesPerTile];
               if (pid < 0 || pid >= a.n_pages) {
                 set_status(a.status, STARKV_DEV_BAD_PAGE);
                 pid = -1;
@@ -247,9 +437,9 @@ __global__ void __launch_bounds__(kAThreads, 1)
           for (int p = 0; p < np; ++p) {
             const int pid = fl[p];
             if (pid < 0) continue;
-            bulk_g2s(sm + a.off_codes + s * a.codes_stage + p * a.codes_page,
+            bulk_g2s(sm + a.off_codes + s * a.codes_stage + p * a.codes_pitch,
                      a.k_codes + ((int64_t)pid * a.h_kv + kv0) * a.key.region_bytes, a.codes_page, &full[s]);
-            bulk_g2s(sm + a.off_meta + s * a.meta_stage + p * a.meta_page,
+            bulk_g2s(sm + a.off_meta + s * a.meta_stage + p * a.meta_pitch,
                      a.k_meta + ((int64_t)pid * a.h_kv + kv0) * a.key.groups * kPage, a.meta_page, &full[s]);
           }
         }
@@ -280,10 +470,10 @@ __global__ void __launch_bounds__(kAThreads, 1)
       }
     } else {
       // ---------------- epilogue: one thread per token ----------------
-      const int q4 = warp & 3, hhalf = (warp - 2) >> 2;
+      const int q4 = warp & 3, hq = (warp - 2) >> 2;   // TMEM lane quarter, head quarter
       const int t = q4 * 32 + lane;
       const int t16 = t % kPage, p = t / kPage;
-      const int hper = a.hpc / 2;
+      const int hper = a.hpc / 4;
       for (int k = 0; k < ntile; ++k) {
         const uint32_t c = it + k, s = c & 1, ph = (c >> 1) & 1;
         if (!mbar_wait(&tfull[s], ph) || !mbar_wait(&full[s], ph)) {
@@ -298,20 +488,43 @@ __global__ void __launch_bounds__(kAThreads, 1)
         const int j = tile * kT + t;
         const int pid = flags[s * kPagesPerTile + p];
         const bool valid = j < L && pid >= 0;
-        const uint8_t* cstage = sm + a.off_codes + s * a.codes_stage + p * a.codes_page;
-        const uint32_t* mstage = reinterpret_cast<const uint32_t*>(sm + a.off_meta + s * a.meta_stage + p * a.meta_page);
-        for (int hh = 0; hh < hper; ++hh) {
-          const int hl = hhalf * hper + hh;
+        const uint8_t* cstage = sm + a.off_codes + s * a.codes_stage + p * a.codes_pitch;
+        const uint32_t* mstage = reinterpret_cast<const uint32_t*>(sm + a.off_meta + s * a.meta_stage + p * a.meta_pitch);
+        const uint32_t trow = tmem + s * 256 + ((uint32_t)(q4 * 32) << 16);
+        auto head = [&](int hl, const uint32_t(&raw)[RK]) {
           const int h = h0 + hl;
           const int kvl = h / a.group - kv0;
-          float G[RK];
-          tmem_load_row<RK>(tmem + s * 256 + hl * RK + ((uint32_t)(q4 * 32) << 16), G);
           float score = -INFINITY;
           if (valid)
-            score = key_dot<RK>(cstage + kvl * a.key.region_bytes, mstage + kvl * a.key.groups * kPage, a.key, t16, G);
+            score = key_dot<RK, G>(cstage + kvl * a.key.region_bytes, mstage + kvl * a.key.groups * kPage,
+                                   a.key.top_groups, t16, raw);
           if (j < L) a.S[((int64_t)b * a.H + h) * a.tpad + j] = score;
           const float m = warp_max(score);
           if (lane == 0) a.Smax[((int64_t)b * a.H + h) * (a.tpad / 32) + tile * 4 + q4] = m;
+        };
+        const int hl0 = hq * hper;
+        if constexpr (RK >= 64) {
+          // one 64-column row per head (a 256-column accumulator holds 4 heads: one per warp)
+          for (int hh = 0; hh < hper; ++hh) {
+            uint32_t rA[RK];
+            tmem_issue_row<RK>(trow + (hl0 + hh) * RK, rA);
+            tmem_wait_row<RK>(rA);
+            head(hl0 + hh, rA);
+          }
+        } else {
+          // ping-pong: the next head's accumulator row lands while this one computes
+          uint32_t rA[RK], rB[RK];
+          tmem_issue_row<RK>(trow + hl0 * RK, rA);
+          for (int hh = 0; hh < hper; hh += 2) {
+            tmem_wait_row<RK>(rA);
+            if (hh + 1 < hper) tmem_issue_row<RK>(trow + (hl0 + hh + 1) * RK, rB);
+            head(hl0 + hh, rA);
+            if (hh + 1 < hper) {
+              tmem_wait_row<RK>(rB);
+              if (hh + 2 < hper) tmem_issue_row<RK>(trow + (hl0 + hh + 2) * RK, rA);
+              head(hl0 + hh + 1, rB);
+            }
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -344,19 +557,79 @@ struct ValueArgs {
   const int32_t* seq_lens;
   const uint8_t* v_codes;
   const uint32_t* v_meta;
-  const float* S;
   const float* Smax;
-  float* acc;    // [B][H][R]
-  float* lsum;   // [B][H]
+  float* part;   // [B][splits][H][R] per-split sums (common maximum)
+  float* lpart;  // [B][splits][H]
   unsigned int* status;
-  uint32_t off_codes, off_meta, off_z, off_p, off_flags, off_m, off_l, off_bar;
-  uint32_t codes_page, meta_page, codes_stage, meta_stage, tmem_cols;
+  uint32_t off_codes, off_meta, off_z, off_p, off_flags, off_m, off_l, off_bar, off_s, off_bt;
+  uint32_t codes_page, meta_page, codes_stage, meta_stage, tmem_cols, s_stage;
+  uint32_t codes_pitch, meta_pitch;  // shared-memory page strides (padded against bank conflicts)
 };
+
+// ---------------------------------------------------------------------------
+// 16-channel value group of one token -> fp16 z_hat = code * s + zp, as two
+// 16-byte chunks.  Codes become fp16 (1024 + code) by OR-ing them under the
+// exponent of 1024 (0x6400); subtracting 1024 is exact, and one half2 fma
+// applies the scale and zero.  The pairs come out as (c, c+4) per nibble word
+// and (c, c+8) per 3-bit plane, so the 16 positions hold channels
+//   4-bit: 0 4 1 5 2 6 3 7 | 8 12 9 13 10 14 11 15
+//   3-bit: 0 8 1 9 2 10 3 11 | 4 12 5 13 6 14 7 15
+// (value_channel_of_position undoes this).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t h2bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 bits2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+__device__ __forceinline__ void scale_zero(uint32_t mw, __half2& s2, __half2& z2) {
+  s2 = bits2h(__byte_perm(mw, mw, 0x1010));
+  z2 = bits2h(__byte_perm(mw, mw, 0x3232));
+}
+
+__device__ __forceinline__ uint32_t deq_pair(uint32_t magic_bits, __half2 s2, __half2 z2) {
+  const __half2 k1024 = __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400));
+  return h2bits(__hfma2(__hsub2(bits2h(magic_bits), k1024), s2, z2));
+}
+
+__device__ __forceinline__ void dequant16_4bit(const uint8_t* p, uint32_t mw, uint4& c0, uint4& c1) {
+  __half2 s2, z2;
+  scale_zero(mw, s2, z2);
+  const uint2 w = *reinterpret_cast<const uint2*>(p);
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    o[i] = deq_pair(((w.x >> (4 * i)) & 0x000F000Fu) | 0x64006400u, s2, z2);
+    o[4 + i] = deq_pair(((w.y >> (4 * i)) & 0x000F000Fu) | 0x64006400u, s2, z2);
+  }
+  c0 = make_uint4(o[0], o[1], o[2], o[3]);
+  c1 = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+__device__ __forceinline__ void dequant16_3bit(const uint8_t* tile, int t16, uint32_t mw, uint4& c0, uint4& c1) {
+  __half2 s2, z2;
+  scale_zero(mw, s2, z2);
+  const uint32_t lo = *reinterpret_cast<const uint32_t*>(tile + 4 * t16);
+  const uint32_t hi16 = *reinterpret_cast<const uint16_t*>(tile + 64 + 2 * t16);
+  const uint32_t hs = __byte_perm(hi16, 0u, 0x4140);  // bits 0-7 stay, bits 8-15 -> 16-23
+  uint32_t o[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t l = ((lo >> (2 * c)) & 0x00030003u) | 0x64006400u;
+    const uint32_t h = (c >= 2 ? (hs >> (c - 2)) : (hs << (2 - c))) & 0x00040004u;
+    o[c] = deq_pair(l | h, s2, z2);
+  }
+  c0 = make_uint4(o[0], o[1], o[2], o[3]);
+  c1 = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+__device__ __forceinline__ int value_channel_of_position(int p, bool top) {
+  const int k = p >> 3, e = p & 7;
+  return top ? 8 * k + (e >> 1) + 4 * (e & 1) : 4 * k + (e >> 1) + 8 * (e & 1);
+}
 
 constexpr uint32_t kZBytes = kVT * 128 * 2;   // one M tile of Z: 64 tokens x 128 channels fp16
 constexpr uint32_t kPBytes = 64 * kVT * 2;    // P buffer: up to 64 heads x 64 tokens fp16
 
-__global__ void __launch_bounds__(kBThreads, 1) decode_values_kernel(const ValueArgs a) {
+__global__ void __launch_bounds__(kBThreads, 1)
+    decode_values_kernel(const __grid_constant__ CUtensorMap s_map, const ValueArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + a.off_bar);
@@ -372,6 +645,7 @@ __global__ void __launch_bounds__(kBThreads, 1) decode_values_kernel(const Value
   int* flags = reinterpret_cast<int*>(sm + a.off_flags);   // [kVStages][kVPages]
   float* Mh = reinterpret_cast<float*>(sm + a.off_m);      // [N]
   float* Lh = reinterpret_cast<float*>(sm + a.off_l);      // [N]
+  int* bt_s = reinterpret_cast<int*>(sm + a.off_bt);       // this split's block-table entries
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, b = blockIdx.y;
   const LatentGeom& V = a.val;
@@ -406,17 +680,26 @@ __global__ void __launch_bounds__(kBThreads, 1) decode_values_kernel(const Value
     *failed = 0;
     fence_mbar_init();
   }
-  // sequence-wide maxima per head (common reference of every split), l = 0,
-  // P buffers zeroed once (rows >= H stay zero)
-  for (int h = tid; h < a.N; h += blockDim.x) {
-    float m = -INFINITY;
-    if (h < a.H) {
-      const int nblk = (L + 31) / 32;
-      const float* sm_row = a.Smax + ((int64_t)b * a.H + h) * (a.tpad / 32);
-      for (int i = 0; i < nblk; ++i) m = fmaxf(m, sm_row[i]);
+  // sequence-wide maxima per head (common reference of every split; one warp
+  // per head, lanes over the 32-token block maxima), l = 0, this split's page
+  // ids, P buffers zeroed once (rows >= H stay zero)
+  {
+    const int nblk = (L + 31) / 32;
+    for (int h = warp; h < a.N; h += kBThreads / 32) {
+      float m = -INFINITY;
+      if (h < a.H) {
+        const float* sm_row = a.Smax + ((int64_t)b * a.H + h) * (a.tpad / 32);
+        for (int i = lane; i < nblk; i += 32) m = fmaxf(m, sm_row[i]);
+      }
+      m = warp_max(m);
+      if (lane == 0) {
+        Mh[h] = m;
+        Lh[h] = 0.f;
+      }
     }
-    Mh[h] = m;
-    Lh[h] = 0.f;
+    const int p0 = st_lo * kVPages;
+    const int np_split = min(nst * kVPages, (L + kPage - 1) / kPage - p0);
+    for (int e = tid; e < np_split; e += blockDim.x) bt_s[e] = a.block_table[(int64_t)b * a.max_pages + p0 + e];
   }
   for (int i = tid; i < (int)(2 * kPBytes / 16); i += blockDim.x)
     reinterpret_cast<uint4*>(sm + a.off_p)[i] = make_uint4(0, 0, 0, 0);
@@ -445,7 +728,7 @@ __global__ void __launch_bounds__(kBThreads, 1) decode_values_kernel(const Value
         for (int p = 0; p < kVPages; ++p) {
           int pid = -1;
           if (p < np) {
-            pid = a.block_table[(int64_t)b * a.max_pages + j0 / kPage + p];
+            pid = bt_s[k * kVPages + p];
             if (pid < 0 || pid >= a.n_pages) {
               set_status(a.status, STARKV_DEV_BAD_PAGE);
               pid = -1;
@@ -455,13 +738,16 @@ __global__ void __launch_bounds__(kBThreads, 1) decode_values_kernel(const Value
           }
           fl[p] = pid;
         }
+        // score rows of the stage: one 2-D TMA box of H rows x 64 tokens (fp32)
+        bytes += a.s_stage;
         mbar_arrive_expect_tx(&cfull[cs], bytes);
+        tma_load_2d(sm + a.off_s + cs * a.s_stage, &s_map, j0, b * a.H, &cfull[cs]);
         for (int p = 0; p < np; ++p) {
           const int pid = fl[p];
           if (pid < 0) continue;
-          bulk_g2s(sm + a.off_codes + cs * a.codes_stage + p * a.codes_page,
+          bulk_g2s(sm + a.off_codes + cs * a.codes_stage + p * a.codes_pitch,
                    a.v_codes + (int64_t)pid * V.region_bytes, a.codes_page, &cfull[cs]);
-          bulk_g2s(sm + a.off_meta + cs * a.meta_stage + p * a.meta_page,
+          bulk_g2s(sm + a.off_meta + cs * a.meta_stage + p * a.meta_pitch,
                    a.v_meta + (int64_t)pid * V.groups * kPage, a.meta_page, &cfull[cs]);
         }
       }
@@ -532,7 +818,7 @@ __global__ void __launch_bounds__(kBThreads, 1) decode_values_kernel(const Value
             const int j = j0 + t;
             float p = 0.f;
             if (j < L && fl[t / kPage] >= 0) {
-              const float sc = a.S[((int64_t)b * a.H + h) * a.tpad + j];
+              const float sc = reinterpret_cast<const float*>(sm + a.off_s + cs * a.s_stage)[h * kVT + t];
               if (sc != -INFINITY) p = exp2f(sc - Mh[h]);
             }
             pv[v] = p;
@@ -548,12 +834,12 @@ __global__ void __launch_bounds__(kBThreads, 1) decode_values_kernel(const Value
       __syncwarp();
       if (lane == 0) mbar_arrive(&pfull[ps]);
       // Z tiles: 64 tokens x 128 channels, MN-major (channels contiguous), fp16
-      const int t = wt >> 2, qq = wt & 3;
+      const int q8 = (warp - 2) & 7, t = ((warp - 2) >> 3) * 32 + lane;  // warp: 16-channel group; lane: token
       const int j = j0 + t;
       const int pg = t / kPage, t16 = t % kPage;
       const bool tvalid = j < L && fl[pg] >= 0;
-      const uint8_t* region = sm + a.off_codes + cs * a.codes_stage + pg * a.codes_page;
-      const uint32_t* meta = reinterpret_cast<const uint32_t*>(sm + a.off_meta + cs * a.meta_stage + pg * a.meta_page);
+      const uint8_t* region = sm + a.off_codes + cs * a.codes_stage + pg * a.codes_pitch;
+      const uint32_t* meta = reinterpret_cast<const uint32_t*>(sm + a.off_meta + cs * a.meta_stage + pg * a.meta_pitch);
       for (int mt = 0; mt < a.MT; ++mt, ++zc) {
         const uint32_t zs = zc % kZBufs, zph = (zc / kZBufs) & 1;
         if (!mbar_wait(&zempty[zs], zph ^ 1)) {
@@ -561,23 +847,19 @@ __global__ void __launch_bounds__(kBThreads, 1) decode_values_kernel(const Value
           break;
         }
         uint8_t* zbuf = sm + a.off_z + zs * kZBytes;
-        for (int c8 = 0; c8 < 4; ++c8) {
-          const int m = qq * 32 + c8 * 8;          // channel within the tile
-          const int ch0 = mt * 128 + m;
-          uint32_t w4[4] = {0, 0, 0, 0};
-          if (tvalid && ch0 < V.r) {
-            const int gi = ch0 / V.g;
-            const float2 sz = unpack_meta(meta[gi * kPage + t16]);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int c = ch0 % V.g + 2 * u;
-              const float z0 = __fmaf_rn((float)load_code(region, V, gi, t16, c), sz.x, sz.y);
-              const float z1 = __fmaf_rn((float)load_code(region, V, gi, t16, c + 1), sz.x, sz.y);
-              const __half2 h2 = __floats2half2_rn(z0, z1);
-              w4[u] = *reinterpret_cast<const uint32_t*>(&h2);
-            }
+        {
+          const int m0 = q8 * 16;                    // first M position of this 16-channel group
+          const int gi = (mt * 128 + m0) >> 4;
+          uint4 c0 = make_uint4(0, 0, 0, 0), c1 = make_uint4(0, 0, 0, 0);
+          if (tvalid && gi < V.groups) {
+            const uint32_t mw = meta[gi * kPage + t16];
+            if (gi < V.top_groups)
+              dequant16_4bit(region + gi * 128 + 8 * t16, mw, c0, c1);
+            else
+              dequant16_3bit(region + V.top_groups * 128 + (gi - V.top_groups) * 96, t16, mw, c0, c1);
           }
-          *reinterpret_cast<uint4*>(zbuf + sw128_mnmajor_offset(t, m, 2)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          *reinterpret_cast<uint4*>(zbuf + sw128_mnmajor_offset(t, m0, 2)) = c0;
+          *reinterpret_cast<uint4*>(zbuf + sw128_mnmajor_offset(t, m0 + 8, 2)) = c1;
         }
         fence_async_smem();
         __syncwarp();
@@ -590,12 +872,15 @@ __global__ void __launch_bounds__(kBThreads, 1) decode_values_kernel(const Value
       set_status(a.status, kDevWaitTimeout);
       *failed = 1;
     }
-    // drain D (TMEM) into the per-(sequence, head) accumulator
+    // drain D (TMEM) into this split's partial sums (plain coalesced stores)
     if (mbar_wait(dfull, 0)) {
       tc_fence_after();
       const int q4 = warp & 3, hsel = (warp - 2) >> 2;
-      for (int mt = hsel; mt < a.MT; mt += 2) {
-        const int ch = mt * 128 + q4 * 32 + lane;
+      float* prow = a.part + ((int64_t)b * a.splits + split) * a.H * a.R;
+      for (int mt = hsel; mt < a.MT; mt += kVWarps / 4) {
+        const int mpos = mt * 128 + q4 * 32 + lane;
+        const int gidx = mpos >> 4;
+        const int ch = gidx * 16 + value_channel_of_position(mpos & 15, gidx < V.top_groups);
         for (int c0 = 0; c0 < a.N; c0 += 16) {
           uint32_t r[16];
           asm volatile(
@@ -605,11 +890,12 @@ __global__ void __launch_bounds__(kBThreads, 1) decode_values_kernel(const Value
                 "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
                 "=r"(r[15])
               : "r"(tmem + mt * a.N + c0 + ((uint32_t)(q4 * 32) << 16)));
-          tmem_ld_wait();
+          tmem_wait_row<16>(r);
           if (ch < a.R) {
+#pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int h = c0 + i;
-              if (h < a.H) atomicAdd(&a.acc[((int64_t)b * a.H + h) * a.R + ch], __uint_as_float(r[i]));
+              if (h < a.H) prow[(int64_t)h * a.R + ch] = __uint_as_float(r[i]);
             }
           }
         }
@@ -620,7 +906,7 @@ __global__ void __launch_bounds__(kBThreads, 1) decode_values_kernel(const Value
   }
   tc_fence_before();
   __syncthreads();
-  for (int h = tid; h < a.H; h += blockDim.x) atomicAdd(&a.lsum[(int64_t)b * a.H + h], Lh[h]);
+  for (int h = tid; h < a.H; h += blockDim.x) a.lpart[((int64_t)b * a.splits + split) * a.H + h] = Lh[h];
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, a.tmem_cols);
@@ -632,8 +918,11 @@ __global__ void __launch_bounds__(kBThreads, 1) decode_values_kernel(const Value
 // ===========================================================================
 struct ProjArgs {
   int H, h_kv, group, d, R;
-  const float* acc;
-  const float* lsum;
+  int splits, stages_total;
+  const float* part;     // [B][splits][H][R]
+  const float* lpart;    // [B][splits][H]
+  float* oacc;           // [B][H][d] fp32 sums (zeroed by the score kernel)
+  unsigned int* ocnt;    // [H][ceil(B/16)] arrival counters (zeroed by the score kernel)
   const float* Smax;
   const int32_t* seq_lens;
   int tpad, max_pages, max_position;
@@ -641,27 +930,132 @@ struct ProjArgs {
   __nv_bfloat16* out;
 };
 
-__global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a) {
-  extern __shared__ float psm[];
-  float* olat = psm;            // [R]
-  float* red = psm + a.R;       // [256]
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+constexpr int kProjM = 16;    // sequences per projection CTA (the MMA's M)
+constexpr int kProjK = 64;    // channels per staged B'_v slice
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// grid (H, R / kProjK, ceil(B / 16)), 256 threads; warp w owns output columns
+// [16 w, 16 w + 16) (d = 64: warps 4..7 idle in the MMA).  Each CTA multiplies a
+// 64-channel slice, o_lat[16 seq x 64] (fp16, = acc / l) . B'_v[64 x d], adds it
+// into the fp32 sums and the last CTA of a (head, sequence block) to arrive
+// writes the bf16 output (arrival counter, no waiting).
+constexpr int kProjC = 256;  // channels per projection CTA
+
+__global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, int batch, int slices) {
+  extern __shared__ __align__(16) uint8_t proj_smem[];
+  __half(*As)[kProjC + 8] = reinterpret_cast<__half(*)[kProjC + 8]>(proj_smem);                 // [16][256 + 8]
+  __half(*Bs)[128 + 8] = reinterpret_cast<__half(*)[128 + 8]>(proj_smem + kProjM * (kProjC + 8) * 2);  // [256][136]
+  __shared__ float linv[kProjM];
+  __shared__ int last;
+  const int R = a.R, d = a.d;
+  const int h = blockIdx.x, kc = blockIdx.y, bc = blockIdx.z;
+  const int b0 = bc * kProjM;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int kv = h / a.group;
-  const float l = a.lsum[(int64_t)b * a.H + h];
-  const float inv = l > 0.f ? 1.f / l : 0.f;
-  for (int ch = tid; ch < a.R; ch += 256) olat[ch] = a.acc[((int64_t)b * a.H + h) * a.R + ch] * inv;
+  const int ldg = a.h_kv * d;
+  const int nch = slices * kProjK;           // channels of this CTA (<= 256)
+  const int ch0 = kc * nch;
+  // B'_v rows of this chunk: issue every load first
+  for (int e = tid; e < nch * (d / 8); e += 256) {
+    const int r = e / (d / 8), q = e % (d / 8);
+    *reinterpret_cast<uint4*>(&Bs[r][q * 8]) =
+        *reinterpret_cast<const uint4*>(a.Bv16 + (int64_t)(ch0 + r) * ldg + kv * d + q * 8);
+  }
+  // l per sequence = sum of its splits' l
+  auto n_splits = [&](int b) {
+    int L = a.seq_lens[b];
+    if (L < 0 || L > a.max_pages * kPage || L > a.max_position) L = 0;
+    const int nst = (L + kVT - 1) / kVT;
+    return nst > 0 ? min(a.splits, (int)(((int64_t)nst * a.splits - 1) / a.stages_total) + 1) : 0;
+  };
+  if (tid < kProjM) {
+    const int b = b0 + tid;
+    float l = 0.f;
+    if (b < batch) {
+      const int nsp = n_splits(b);
+      for (int sp = 0; sp < nsp; ++sp) l += a.lpart[((int64_t)b * a.splits + sp) * a.H + h];
+    }
+    linv[tid] = l > 0.f ? 1.f / l : 0.f;
+  }
   __syncthreads();
-  const int nh = 256 / a.d;
-  const int col = tid % a.d, sub = tid / a.d;
-  const int ldb = a.h_kv * a.d;
-  float o = 0.f;
-  for (int ch = sub; ch < a.R; ch += nh) o = fmaf(olat[ch], __half2float(a.Bv16[(int64_t)ch * ldb + kv * a.d + col]), o);
-  red[sub * a.d + col] = o;
+  // o_lat = (sum over splits of the partials) / l, four channels per item
+  for (int e = tid; e < kProjM * (nch / 4); e += 256) {
+    const int r = e / (nch / 4), c4 = (e % (nch / 4)) * 4;
+    const int b = b0 + r;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (b < batch) {
+      const int nsp = n_splits(b);
+      const float* base = a.part + ((int64_t)b * a.splits * a.H + h) * R + ch0 + c4;
+      const int64_t stride = (int64_t)a.H * R;
+#pragma unroll 3
+      for (int sp = 0; sp < nsp; ++sp) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(base + sp * stride));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+    }
+    const float li = linv[r];
+    *reinterpret_cast<__half2*>(&As[r][c4]) = __floats2half2_rn(acc.x * li, acc.y * li);
+    *reinterpret_cast<__half2*>(&As[r][c4 + 2]) = __floats2half2_rn(acc.z * li, acc.w * li);
+  }
   __syncthreads();
-  if (sub == 0) {
-    float t = 0.f;
-    for (int k = 0; k < nh; ++k) t += red[k * a.d + col];
-    a.out[((int64_t)b * a.H + h) * a.d + col] = __float2bfloat16_rn(t);
+  float c[2][4] = {};
+  if (warp * 16 < d) {
+#pragma unroll 4
+    for (int kk = 0; kk < nch; kk += 16) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(sm100::smem_u32(&As[lane & 15][kk + (lane >> 4) * 8]), a0, a1, a2, a3);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        uint32_t b0r, b1r;
+        ldsm_x2_t(sm100::smem_u32(&Bs[kk + (lane & 15)][warp * 16 + nt * 8]), b0r, b1r);
+        mma16816(c[nt], a0, a1, a2, a3, b0r, b1r);
+      }
+    }
+  }
+  if (warp * 16 < d) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int col = warp * 16 + nt * 8 + (lane & 3) * 2;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int b = b0 + (lane >> 2) + hf * 8;
+        if (b < batch)
+          atomicAdd(reinterpret_cast<float2*>(a.oacc + ((int64_t)b * a.H + h) * d + col),
+                    make_float2(c[nt][hf * 2], c[nt][hf * 2 + 1]));
+      }
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last = atomicAdd(&a.ocnt[h * gridDim.z + bc], 1u) == gridDim.y - 1;
+  __syncthreads();
+  if (last) {
+    __threadfence();
+    for (int e = tid; e < kProjM * d; e += 256) {
+      const int b = b0 + e / d, col = e % d;
+      if (b < batch) {
+        const int64_t o = ((int64_t)b * a.H + h) * d + col;
+        a.out[o] = __float2bfloat16_rn(__ldcg(a.oacc + o));
+      }
+    }
   }
 }
 
@@ -673,10 +1067,11 @@ bool tc_decode_supported(const starkv_config& cfg) {
   if (rk != 16 && rk != 32 && rk != 64) return false;
   const int hpc = (256 / rk) < cfg.num_q_heads ? 256 / rk : cfg.num_q_heads;
   const int group = cfg.num_q_heads / cfg.num_kv_heads;
-  if (cfg.num_q_heads % hpc != 0 || hpc % 2 != 0) return false;
+  if (cfg.num_q_heads % hpc != 0 || hpc % 4 != 0) return false;
   if (hpc % group != 0 && group % hpc != 0) return false;
   if (group > hpc) return false;  // a CTA's heads must cover whole KV heads
   if (cfg.num_q_heads > 64) return false;
+  if (cfg.rank_v % 64 != 0) return false;  // projection stages 64-channel slices
   return true;
 }
 
@@ -694,7 +1089,7 @@ int sm_count() {
 
 struct TcLayout {
   int hpc, kvpc, ncols, HG, tiles_per_seq, tpad, splits, stages_total, N, MT;
-  size_t off_S, off_Smax, off_acc, off_l, ws;
+  size_t off_S, off_Smax, off_acc, off_l, off_w, off_oacc, off_ocnt, w_bytes, ws;
 };
 
 TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
@@ -707,7 +1102,7 @@ TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
   t.tiles_per_seq = (max_pages * kPage + kT - 1) / kT;
   t.tpad = t.tiles_per_seq * kT;
   t.stages_total = t.tpad / kVT;
-  int splits = (sm_count() + batch - 1) / (batch > 0 ? batch : 1);
+  int splits = sm_count() / (batch > 0 ? batch : 1);  // one CTA per SM: stay within a single wave
   if (splits > t.stages_total) splits = t.stages_total;
   if (splits < 1) splits = 1;
   t.splits = splits;
@@ -720,9 +1115,16 @@ TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
   t.off_Smax = o;
   o += al((size_t)batch * f.num_q_heads * (t.tpad / 32) * 4);
   t.off_acc = o;
-  o += al((size_t)batch * f.num_q_heads * f.rank_v * 4);
+  o += al((size_t)batch * t.splits * f.num_q_heads * f.rank_v * 4);
   t.off_l = o;
-  o += al((size_t)batch * f.num_q_heads * 4);
+  o += al((size_t)batch * t.splits * f.num_q_heads * 4);
+  t.w_bytes = (size_t)t.ncols * f.head_dim * 2;
+  t.off_w = o;
+  o += al((size_t)batch * t.HG * t.w_bytes);
+  t.off_oacc = o;
+  o += al((size_t)batch * f.num_q_heads * f.head_dim * 4);
+  t.off_ocnt = o;
+  o += al((size_t)f.num_q_heads * ((batch + 15) / 16) * 4);
   t.ws = o;
   return t;
 }
@@ -749,12 +1151,22 @@ cudaError_t launch_prepare_tc_factors(const Ctx& c, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <int RK, int G>
+static cudaError_t launch_scores_g(const Ctx& c, const ScoreArgs& a, int grid, size_t smem, cudaStream_t s) {
+  cudaError_t e =
+      cudaFuncSetAttribute(decode_scores_kernel<RK, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  decode_scores_kernel<RK, G><<<grid, kAThreads, smem, s>>>(c.trig_map, a);
+  return cudaGetLastError();
+}
+
 template <int RK>
 static cudaError_t launch_scores(const Ctx& c, const ScoreArgs& a, int grid, size_t smem, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(decode_scores_kernel<RK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  decode_scores_kernel<RK><<<grid, kAThreads, smem, s>>>(c.trig_map, a);
-  return cudaGetLastError();
+  switch (c.key.g) {
+    case 4: return launch_scores_g<RK, 4>(c, a, grid, smem, s);
+    case 8: return launch_scores_g<RK, 8>(c, a, grid, smem, s);
+    default: return launch_scores_g<RK, 16>(c, a, grid, smem, s);
+  }
 }
 
 cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
@@ -768,7 +1180,31 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   float* Smax = (float*)(w + t.off_Smax);
   float* acc = (float*)(w + t.off_acc);
   float* lsum = (float*)(w + t.off_l);
+  uint8_t* wimg = (uint8_t*)(w + t.off_w);
+  float* oacc = (float*)(w + t.off_oacc);
+  unsigned int* ocnt = (unsigned int*)(w + t.off_ocnt);
   const int d = f.head_dim;
+
+  // ---------------- W images: rotated query folded into B'_k, per (sequence, head)
+  {
+    dim3 g(f.num_q_heads, batch);
+    switch (f.rank_k) {
+      case 16:
+        decode_wprep_kernel<16><<<g, 64, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, f.num_q_heads, c.group, d, t.hpc,
+                                                t.ncols, max_pages, f.max_position);
+        break;
+      case 32:
+        decode_wprep_kernel<32><<<g, 64, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, f.num_q_heads, c.group, d, t.hpc,
+                                                t.ncols, max_pages, f.max_position);
+        break;
+      default:
+        decode_wprep_kernel<64><<<g, 64, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, f.num_q_heads, c.group, d, t.hpc,
+                                                t.ncols, max_pages, f.max_position);
+        break;
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
 
   // ---------------- A: scores
   ScoreArgs A;
@@ -800,16 +1236,20 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   A.rope = c.rope;
   A.S = S;
   A.Smax = Smax;
-  A.acc = acc;
-  A.lsum = lsum;
-  A.acc_elems = (int64_t)batch * f.num_q_heads * f.rank_v;
-  A.lsum_elems = (int64_t)batch * f.num_q_heads;
+  A.oacc = oacc;
+  A.ocnt = ocnt;
+  A.oacc_elems = (int64_t)batch * f.num_q_heads * d;
+  A.ocnt_elems = f.num_q_heads * ((batch + 15) / 16);
+  A.wimg = wimg;
+  A.w_bytes = (uint32_t)t.w_bytes;
   A.status = c.status;
   A.trig_stage = kT * d * 2;
   A.codes_page = t.kvpc * c.key.region_bytes;
   A.meta_page = t.kvpc * c.key.groups * kPage * 4;
-  A.codes_stage = kPagesPerTile * A.codes_page;
-  A.meta_stage = kPagesPerTile * A.meta_page;
+  A.codes_pitch = A.codes_page + 64;
+  A.meta_pitch = A.meta_page + 64;
+  A.codes_stage = kPagesPerTile * A.codes_pitch;
+  A.meta_stage = kPagesPerTile * A.meta_pitch;
   {
     uint32_t o = (uint32_t)t.ncols * d * 2;  // W
     o = (o + 1023) / 1024 * 1024;
@@ -821,8 +1261,8 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
     o += 2 * A.meta_stage;
     A.off_flags = o;
     o += 2 * kPagesPerTile * 4;
-    A.off_q = (o + 15) / 16 * 16;
-    o = A.off_q + t.hpc * d * 4;
+    A.off_bt = (o + 15) / 16 * 16;
+    o = A.off_bt + A.items_per_cta * kPagesPerTile * 4;
     A.off_bar = (o + 15) / 16 * 16;
     o = A.off_bar + 16 * 8;
     const size_t smem = o + 1024;  // alignment slack
@@ -853,15 +1293,17 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   B.seq_lens = seq_lens;
   B.v_codes = (const uint8_t*)cache.v_codes;
   B.v_meta = (const uint32_t*)cache.v_meta;
-  B.S = S;
   B.Smax = Smax;
-  B.acc = acc;
-  B.lsum = lsum;
+  B.part = acc;
+  B.lpart = lsum;
   B.status = c.status;
   B.codes_page = c.val.region_bytes;
   B.meta_page = c.val.groups * kPage * 4;
-  B.codes_stage = kVPages * B.codes_page;
-  B.meta_stage = kVPages * B.meta_page;
+  B.codes_pitch = B.codes_page + 64;
+  B.meta_pitch = B.meta_page + 64;
+  B.codes_stage = kVPages * B.codes_pitch;
+  B.meta_stage = kVPages * B.meta_pitch;
+  B.s_stage = f.num_q_heads * kVT * 4;
   uint32_t cols = 32;
   while (cols < (uint32_t)(t.MT * t.N)) cols <<= 1;
   B.tmem_cols = cols;
@@ -875,8 +1317,13 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
     o += kVStages * B.codes_stage;
     B.off_meta = o;
     o += kVStages * B.meta_stage;
+    o = (o + 127) / 128 * 128;  // TMA destination
+    B.off_s = o;
+    o += kVStages * B.s_stage;
     B.off_flags = o;
     o += kVStages * kVPages * 4;
+    B.off_bt = (o + 15) / 16 * 16;
+    o = B.off_bt + ((t.stages_total + t.splits - 1) / t.splits + 1) * kVPages * 4;
     B.off_m = (o + 15) / 16 * 16;
     o = B.off_m + t.N * 4;
     B.off_l = o;
@@ -884,9 +1331,13 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
     B.off_bar = (o + 15) / 16 * 16;
     o = B.off_bar + 32 * 8;
     const size_t smem = o + 1024;
+    CUtensorMap s_map;
+    if (!encode_map_2d(&s_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, S, (uint64_t)t.tpad, (uint64_t)batch * f.num_q_heads,
+                       (uint64_t)t.tpad * 4, kVT, (uint32_t)f.num_q_heads, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(decode_values_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    decode_values_kernel<<<dim3(t.splits, batch), kBThreads, smem, s>>>(B);
+    decode_values_kernel<<<dim3(t.splits, batch), kBThreads, smem, s>>>(s_map, B);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -898,8 +1349,10 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   P.group = c.group;
   P.d = d;
   P.R = f.rank_v;
-  P.acc = acc;
-  P.lsum = lsum;
+  P.splits = t.splits;
+  P.stages_total = t.stages_total;
+  P.part = acc;
+  P.lpart = lsum;
   P.Smax = Smax;
   P.seq_lens = seq_lens;
   P.tpad = t.tpad;
@@ -907,8 +1360,16 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   P.max_position = f.max_position;
   P.Bv16 = c.Bv16;
   P.out = out;
-  const size_t psmem = (size_t)(f.rank_v + 256) * 4;
-  decode_project_kernel<<<dim3(f.num_q_heads, batch), 256, psmem, s>>>(P);
+  P.oacc = oacc;
+  P.ocnt = ocnt;
+  const int slices = f.rank_v % (4 * kProjK) == 0 ? 4 : (f.rank_v % (2 * kProjK) == 0 ? 2 : 1);
+  const size_t psmem = (size_t)kProjM * (kProjC + 8) * 2 + (size_t)kProjC * (128 + 8) * 2;
+  {
+    cudaError_t e = cudaFuncSetAttribute(decode_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+    if (e != cudaSuccess) return e;
+  }
+  decode_project_kernel<<<dim3(f.num_q_heads, f.rank_v / (kProjK * slices), (batch + kProjM - 1) / kProjM), 256, psmem,
+                          s>>>(P, batch, slices);
   return cudaGetLastError();
 }
 

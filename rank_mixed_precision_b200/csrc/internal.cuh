@@ -42,10 +42,18 @@ struct Ctx {
   float2* rope;           // [max_position][d_h/2] (cos, sin), built in fp64
   __half* trig;           // [max_position][d_h] fp16: cos(p th_0..), sin(p th_0..) (tensor-core operand)
   __half* Bv16;           // [R][h_kv*d_h] fp16, B'_v
+  float* zacc;            // [kSmallAppend][h_kv*r_k + R] fp32 split-K sums of small appends (kept zero)
   unsigned int* status;   // device status word
   CUtensorMap trig_map;   // TMA map of `trig`: box 64 x 128, 128-byte swizzle
   bool tc;                // tensor-core decode available for this shape
 };
+
+// 2-D TMA map over a row-major [rows][inner] array (no interleave, zero fill).
+bool encode_map_2d(CUtensorMap* map, CUtensorMapDataType type, void* base, uint64_t inner, uint64_t rows,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle);
+
+// Appends of at most this many tokens use the split-K projection path.
+constexpr int kSmallAppend = 64;
 
 // Extra device status bit: a pipeline wait in a tensor-core kernel gave up.
 constexpr unsigned int kDevWaitTimeout = STARKV_DEV_WAIT_TIMEOUT;

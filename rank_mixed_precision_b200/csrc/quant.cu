@@ -234,6 +234,103 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Small appends (a decode step adds one token per sequence): the projection is
+// a thin GEMM bound by reading A once.  Split K over 128-row slices so the whole
+// GPU streams A: each CTA owns 64 columns x 128 rows of A and adds its n x 64
+// partial sums into the context's fp32 buffer; a second kernel rotates,
+// quantises and packs each (token, group) and returns the buffer to zero.
+// ---------------------------------------------------------------------------
+constexpr int kSkRows = 128, kSkCols = 64;
+
+constexpr int kSkSub = 4;  // 128-row sub-slices per CTA
+
+__global__ void __launch_bounds__(256) append_splitk_kernel(AppendArgs a, float* zacc) {
+  __shared__ __align__(16) __nv_bfloat16 As[kSkRows][kSkCols];   // 16 KB
+  __shared__ __nv_bfloat16 Xs[kSmallAppend][kSkRows];             // 16 KB
+  const int tid = threadIdx.x;
+  const int col0 = blockIdx.x * kSkCols;
+  const int n = (int)a.n;
+  const int cq = (tid % 16) * 4;
+  float acc[kSmallAppend / 16][4] = {};
+  for (int sub = 0; sub < kSkSub; ++sub) {
+    const int k0 = (blockIdx.y * kSkSub + sub) * kSkRows;
+    if (k0 >= a.hidden) break;
+    __syncthreads();
+    for (int e = tid; e < kSkRows * (kSkCols / 8); e += 256) {
+      const int r = e / (kSkCols / 8), q = e % (kSkCols / 8);
+      const int col = col0 + q * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (col < a.lat_cols) v = *reinterpret_cast<const uint4*>(a.A + (int64_t)(k0 + r) * a.lat_cols + col);
+      *reinterpret_cast<uint4*>(&As[r][q * 8]) = v;
+    }
+    for (int e = tid; e < n * kSkRows; e += 256) {
+      const int i = e / kSkRows, k = e % kSkRows;
+      Xs[i][k] = a.X[(int64_t)i * a.hidden + k0 + k];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int ii = 0; ii < kSmallAppend / 16; ++ii) {
+      const int i = tid / 16 + 16 * ii;
+      if (i >= n) break;
+      for (int k = 0; k < kSkRows; ++k) {
+        const float x = __bfloat162float(Xs[i][k]);
+        const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&As[k][cq]);
+        const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&As[k][cq + 2]);
+        acc[ii][0] = fmaf(x, __low2float(w01), acc[ii][0]);
+        acc[ii][1] = fmaf(x, __high2float(w01), acc[ii][1]);
+        acc[ii][2] = fmaf(x, __low2float(w23), acc[ii][2]);
+        acc[ii][3] = fmaf(x, __high2float(w23), acc[ii][3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int ii = 0; ii < kSmallAppend / 16; ++ii) {
+    const int i = tid / 16 + 16 * ii;
+    if (i >= n) break;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (col0 + cq + j < a.lat_cols) atomicAdd(&zacc[(int64_t)i * a.lat_cols + col0 + cq + j], acc[ii][j]);
+  }
+}
+
+// one thread per (token, 4-column unit); the unit that starts a group quantises it
+__global__ void append_quant_kernel(AppendArgs a, float* zacc) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int units = a.lat_cols / 4;
+  if (idx >= a.n * units) return;
+  const int64_t row = idx / units;
+  const int col = (int)(idx % units) * 4;
+  float* z = zacc + row * a.lat_cols + col;
+  const int key_cols = a.h_kv * a.key.r;
+  const bool is_key = col < key_cols;
+  const LatentGeom& L = is_key ? a.key : a.val;
+  const int cin = is_key ? col % a.key.r : col - key_cols;
+  if (cin % L.g == 0) {
+    float x[16];
+    for (int i = 0; i < L.g; ++i) x[i] = z[i];
+    if (a.lat_out)
+      for (int i = 0; i < L.g; ++i) a.lat_out[row * a.lat_cols + col + i] = x[i];
+    const int64_t slot = a.slots[row];
+    if (slot >= a.n_pages * kPage) {
+      set_status(a.status, STARKV_DEV_BAD_SLOT);
+    } else if (slot >= 0) {
+      const int64_t page = slot / kPage;
+      const int t = (int)(slot % kPage);
+      const int gi = cin / L.g;
+      if (is_key) {
+        const int kv = col / a.key.r;
+        rotate_quantize_store_any(x, L, gi, a.k_codes + (page * a.h_kv + kv) * L.region_bytes,
+                                  a.k_meta + (page * a.h_kv + kv) * L.groups * kPage, t, a.status);
+      } else {
+        rotate_quantize_store_any(x, L, gi, a.v_codes + page * L.region_bytes, a.v_meta + page * L.groups * kPage,
+                                  t, a.status);
+      }
+    }
+    for (int i = 0; i < L.g; ++i) z[i] = 0.f;  // leave the buffer zeroed for the next call
+  }
+}
+
 cudaError_t launch_append(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* X,
                           const int64_t* slots, int64_t n, float* latents_out, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
@@ -254,6 +351,14 @@ cudaError_t launch_append(const Ctx& c, const starkv_cache& cache, const __nv_bf
   a.k_meta = (uint32_t*)cache.k_meta;
   a.v_meta = (uint32_t*)cache.v_meta;
   a.status = c.status;
+  if (n <= kSmallAppend && c.cfg.hidden % kSkRows == 0) {
+    dim3 g1((unsigned)((c.lat_cols + kSkCols - 1) / kSkCols),
+            (unsigned)((c.cfg.hidden / kSkRows + kSkSub - 1) / kSkSub));
+    append_splitk_kernel<<<g1, 256, 0, s>>>(a, c.zacc);
+    const int64_t units = n * (c.lat_cols / 4);
+    append_quant_kernel<<<(unsigned)((units + 127) / 128), 128, 0, s>>>(a, c.zacc);
+    return cudaGetLastError();
+  }
   dim3 grid((unsigned)((n + kAppBM - 1) / kAppBM), (unsigned)((c.lat_cols + kAppBN - 1) / kAppBN));
   append_kernel<<<grid, 256, 0, s>>>(a);
   return cudaGetLastError();

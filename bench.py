@@ -64,6 +64,23 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def sum_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def job_throughput(units_local: float, ms_local: float, world: int, device=None):
+    """Whole-job rate: the units every rank processed over the slowest rank's time."""
+    ms_max = max_over_ranks(ms_local, world, device)
+    units = sum_over_ranks(units_local, world, device)
+    return units / (ms_max / 1e3), ms_max
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -259,9 +276,8 @@ def run_starkv(args, w, rank, world, local):
     status = st.kv.status()
     if status:
         raise RuntimeError(f"device status {status:#x} during the timed region")
-    ms_max = max_over_ranks(ms, world, device)
     tokens_per_step = int(st.seq_lens.sum())
-    value = tokens_per_step * args.steps * world / (ms_max / 1e3)
+    value, ms_max = job_throughput(tokens_per_step * args.steps, ms, world, device)
     # ---- end to end through the public API with host buffers
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
     Xh = pin(gen.bf16_bits(st.X_np).view(np.int16)).view(torch.bfloat16)
@@ -291,8 +307,7 @@ def run_starkv(args, w, rank, world, local):
     e1.record()
     torch.cuda.synchronize()
     barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
-    e2e_value = tokens_per_step * args.steps * world / (e2e_ms / 1e3)
+    e2e_value, _ = job_throughput(tokens_per_step * args.steps, e0.elapsed_time(e1), world, device)
 
     if rank != 0:
         return None

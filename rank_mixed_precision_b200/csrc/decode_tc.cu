@@ -24,6 +24,8 @@
 // kernel winds down instead of spinning.
 #include <float.h>
 
+#include <mutex>
+
 #include "internal.cuh"
 #include "sm100.cuh"
 
@@ -35,12 +37,6 @@ constexpr int kT = 128;                 // tokens per key tile (MMA M)
 constexpr int kPagesPerTile = kT / kPage;
 constexpr int kEpiWarps = 16;
 constexpr int kAThreads = (2 + kEpiWarps) * 32;
-constexpr int kVT = 64;                 // tokens per value stage
-constexpr int kVPages = kVT / kPage;
-constexpr int kVStages = 2;
-constexpr int kZBufs = 4;
-constexpr int kVWarps = 16;
-constexpr int kBThreads = (2 + kVWarps) * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // 1024-byte aligned base inside the dynamic shared-memory array.  The offset is
@@ -54,6 +50,16 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
+}
+
+// Order-preserving map of a float onto unsigned integers (so an integer
+// atomicMax takes a float maximum); 0 stands below every float.
+__device__ __forceinline__ unsigned int ordered_bits(float f) {
+  const unsigned int u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ordered_float(unsigned int o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
 }
 }  // namespace
 
@@ -74,7 +80,7 @@ struct ScoreArgs {
   const float* Bk;     // [h_kv][r_k][d] fp32 B'_k
   const float2* rope;  // [max_position][d/2]
   float* S;            // [B][H][tpad]      scores, log2 domain
-  float* Smax;         // [B][H][tpad/32]   maxima of 32-token blocks
+  unsigned int* Mx;    // [B][H] running score maximum (ordered bits; zeroed by the W prep)
   float* oacc;         // [B][H][d] zeroed here for the projection
   unsigned int* ocnt;  // [H][ceil(B/16)] zeroed here
   int64_t oacc_elems;  // B * H * d
@@ -98,10 +104,12 @@ template <int RK>
 __global__ void __launch_bounds__(64) decode_wprep_kernel(const __nv_bfloat16* __restrict__ q,
                                                           const int32_t* __restrict__ seq_lens,
                                                           const float* __restrict__ Bk, const float2* __restrict__ rope,
-                                                          uint8_t* __restrict__ wimg, int H, int group, int d, int hpc,
-                                                          int ncols, int max_pages, int max_position) {
+                                                          uint8_t* __restrict__ wimg, unsigned int* __restrict__ Mx,
+                                                          int H, int group, int d, int hpc, int ncols, int max_pages,
+                                                          int max_position) {
   const int h = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
   const int half = d / 2;
+  if (i == 0) Mx[b * H + h] = 0u;
   if (i >= half) return;
   int L = seq_lens[b];
   if (L <= 0 || L > max_pages * kPage || L > max_position) L = 1;  // unused (no tiles), keep reads in range
@@ -500,7 +508,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
                                    a.key.top_groups, t16, raw);
           if (j < L) a.S[((int64_t)b * a.H + h) * a.tpad + j] = score;
           const float m = warp_max(score);
-          if (lane == 0) a.Smax[((int64_t)b * a.H + h) * (a.tpad / 32) + tile * 4 + q4] = m;
+          if (lane == 0 && m != -INFINITY) atomicMax(&a.Mx[b * a.H + h], ordered_bits(m));
         };
         const int hl0 = hq * hper;
         if constexpr (RK >= 64) {
@@ -550,20 +558,22 @@ __global__ void __launch_bounds__(kAThreads, 1)
 // ===========================================================================
 struct ValueArgs {
   LatentGeom val;
-  int H, N, R, MT, d;
+  int H, N, R, MT;        // heads, heads padded to the MMA's N, value rank, 128-channel M tiles
+  int PS, nW, ST, NS;     // pages per stage, dequant warps (= MT * PS), tokens per stage, ring depth
   int max_pages, tpad, splits, stages_total, max_position;
   int64_t n_pages;
   const int32_t* block_table;
   const int32_t* seq_lens;
   const uint8_t* v_codes;
   const uint32_t* v_meta;
-  const float* Smax;
-  float* part;   // [B][splits][H][R] per-split sums (common maximum)
-  float* lpart;  // [B][splits][H]
+  const unsigned int* Mx;  // [B][H] sequence-wide score maxima (ordered bits)
+  float* part;   // [B][nclust][H][R] per-cluster sums (common maximum)
+  float* lpart;  // [B][nclust][H]
   unsigned int* status;
-  uint32_t off_codes, off_meta, off_z, off_p, off_flags, off_m, off_l, off_bar, off_s, off_bt;
-  uint32_t codes_page, meta_page, codes_stage, meta_stage, tmem_cols, s_stage;
-  uint32_t codes_pitch, meta_pitch;  // shared-memory page strides (padded against bank conflicts)
+  int CS, nclust;         // CTAs per cluster, clusters per sequence
+  uint32_t off_z, off_p, off_s, off_codes, off_meta, off_flags, off_bt, off_m, off_l, off_bar;
+  uint32_t p_stage, s_box, s_box_bytes, s_stage;
+  uint32_t codes_page, meta_page, codes_pitch, meta_pitch, codes_stage, meta_stage, tmem_cols;
 };
 
 // ---------------------------------------------------------------------------
@@ -625,30 +635,52 @@ __device__ __forceinline__ int value_channel_of_position(int p, bool top) {
   return top ? 8 * k + (e >> 1) + 4 * (e & 1) : 4 * k + (e >> 1) + 8 * (e & 1);
 }
 
-constexpr uint32_t kZBytes = kVT * 128 * 2;   // one M tile of Z: 64 tokens x 128 channels fp16
-constexpr uint32_t kPBytes = 64 * kVT * 2;    // P buffer: up to 64 heads x 64 tokens fp16
+constexpr int kVMaxWarps = 16;                      // dequant warps at most
+constexpr int kVThreads = (2 + kVMaxWarps) * 32;
+constexpr int kVMaxStages = 8;
+constexpr uint32_t kZTile = kPage * 128 * 2;        // one page x one 128-channel M tile, fp16
 
-__global__ void __launch_bounds__(kBThreads, 1)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// One CTA per (token split, sequence); the CS splits of a cluster add their
+// sums on chip and write one partial.  Warp roles:
+//   warp 0, lane 0   producer: per stage of ST tokens, the score rows (TMA boxes
+//                    of 32 tokens x H heads, 128-byte swizzle) and the value
+//                    codes + metadata of its PS pages (bulk copies), NS stages deep
+//   warp 1           P: lane = head; P[h, t] = exp2(s - M_h) as fp16 into a
+//                    K-major tile, l_h summed in registers
+//   warps 2..nW+1    dequant warp w = (M tile w % MT, page w / MT of the stage):
+//                    dequantises its 16 tokens x 128 channels into its own Z tile
+//                    and issues its own MMA  D_w[ch, h] += sum_t Z[t, ch] P[h, t]
+//                    into its own TMEM columns (no cross-warp hand-off per tile)
+// At the end the page accumulators of each M tile go to shared memory as
+// [H][R] fp32, and CTA r of the cluster sums channel slice r over the cluster
+// (distributed shared memory) into the partial.
+__global__ void __launch_bounds__(kVThreads, 1)
     decode_values_kernel(const __grid_constant__ CUtensorMap s_map, const ValueArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + a.off_bar);
-  uint64_t* cfull = bar;                         // [kVStages]
-  uint64_t* cempty = cfull + kVStages;           // [kVStages]
-  uint64_t* zfull = cempty + kVStages;           // [kZBufs]
-  uint64_t* zempty = zfull + kZBufs;             // [kZBufs]
-  uint64_t* pfull = zempty + kZBufs;             // [2]
-  uint64_t* pempty = pfull + 2;                  // [2]
-  uint64_t* dfull = pempty + 2;                  // [1]
+  uint64_t* cfull = bar;                     // [NS] stage landed
+  uint64_t* cempty = cfull + kVMaxStages;    // [NS] stage read (P warp + dequant warps)
+  uint64_t* pfull = cempty + kVMaxStages;    // [NS] P tile written
+  uint64_t* pempty = pfull + kVMaxStages;    // [NS] MMAs reading the P tile done
+  uint64_t* zempty = pempty + kVMaxStages;   // [nW] MMA reading warp w's Z tile done
+  uint64_t* dfull = zempty + kVMaxWarps;     // every accumulator final
   uint32_t* tslot = reinterpret_cast<uint32_t*>(dfull + 1);
-  int* failed = reinterpret_cast<int*>(dfull + 2);
-  int* flags = reinterpret_cast<int*>(sm + a.off_flags);   // [kVStages][kVPages]
-  float* Mh = reinterpret_cast<float*>(sm + a.off_m);      // [N]
-  float* Lh = reinterpret_cast<float*>(sm + a.off_l);      // [N]
-  int* bt_s = reinterpret_cast<int*>(sm + a.off_bt);       // this split's block-table entries
+  int* flags = reinterpret_cast<int*>(sm + a.off_flags);  // [NS][PS] page ids, -1 = skip
+  int* bt_s = reinterpret_cast<int*>(sm + a.off_bt);      // this split's block-table entries
+  float* Mh = reinterpret_cast<float*>(sm + a.off_m);     // [H]
+  float* Lh = reinterpret_cast<float*>(sm + a.off_l);     // [H] this CTA's l
+  float* accs = reinterpret_cast<float*>(sm);             // [H][R] this CTA's sums (after the pipeline)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, b = blockIdx.y;
   const LatentGeom& V = a.val;
+  const int NS = a.NS, PS = a.PS, ST = a.ST;
 
   int L = a.seq_lens[b];
   const bool bad_len = L < 0 || L > a.max_pages * kPage || L > a.max_position;
@@ -656,261 +688,309 @@ __global__ void __launch_bounds__(kBThreads, 1)
     if (split == 0 && tid == 0) set_status(a.status, STARKV_DEV_BAD_SEQ_LEN);
     L = 0;
   }
+  const int seq_stages = (L + ST - 1) / ST;
+  const int clust = split / a.CS;
+  // a cluster none of whose splits has tokens leaves as a whole (no partial)
+  if ((int)((int64_t)clust * a.CS * a.stages_total / a.splits) >= seq_stages) return;
   const int st_lo = (int)((int64_t)split * a.stages_total / a.splits);
-  const int st_hi0 = (int)((int64_t)(split + 1) * a.stages_total / a.splits);
-  const int st_hi = min(st_hi0, (L + kVT - 1) / kVT);
-  const int nst = st_hi - st_lo;
-  if (nst <= 0) return;  // nothing of this sequence here (uniform across the CTA)
+  const int st_hi = min((int)((int64_t)(split + 1) * a.stages_total / a.splits), seq_stages);
+  const int nst = st_hi > st_lo ? st_hi - st_lo : 0;
+  const bool work = nst > 0;  // uniform across the CTA
 
-  if (warp == 1) tmem_alloc(tslot, a.tmem_cols);
+  if (work && warp == 1) tmem_alloc(tslot, a.tmem_cols);
   if (tid == 0) {
-    for (int s = 0; s < kVStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&cfull[s], 1);
-      mbar_init(&cempty[s], kVWarps);
+      mbar_init(&cempty[s], a.nW + 1);
+      mbar_init(&pfull[s], 1);
+      mbar_init(&pempty[s], a.nW);
     }
-    for (int s = 0; s < kZBufs; ++s) {
-      mbar_init(&zfull[s], kVWarps);
-      mbar_init(&zempty[s], 1);
-    }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&pfull[s], kVWarps);
-      mbar_init(&pempty[s], 1);
-    }
-    mbar_init(dfull, 1);
-    *failed = 0;
+    for (int w = 0; w < a.nW; ++w) mbar_init(&zempty[w], 1);
+    mbar_init(dfull, a.nW);
     fence_mbar_init();
   }
-  // sequence-wide maxima per head (common reference of every split; one warp
-  // per head, lanes over the 32-token block maxima), l = 0, this split's page
-  // ids, P buffers zeroed once (rows >= H stay zero)
-  {
-    const int nblk = (L + 31) / 32;
-    for (int h = warp; h < a.N; h += kBThreads / 32) {
-      float m = -INFINITY;
-      if (h < a.H) {
-        const float* sm_row = a.Smax + ((int64_t)b * a.H + h) * (a.tpad / 32);
-        for (int i = lane; i < nblk; i += 32) m = fmaxf(m, sm_row[i]);
-      }
-      m = warp_max(m);
-      if (lane == 0) {
-        Mh[h] = m;
-        Lh[h] = 0.f;
-      }
-    }
-    const int p0 = st_lo * kVPages;
-    const int np_split = min(nst * kVPages, (L + kPage - 1) / kPage - p0);
-    for (int e = tid; e < np_split; e += blockDim.x) bt_s[e] = a.block_table[(int64_t)b * a.max_pages + p0 + e];
+  // sequence-wide maxima per head (the common reference of every split; a
+  // sequence with no finite score uses 0), this split's page ids, P tiles
+  // zeroed once (rows >= H stay zero)
+  for (int h = tid; h < a.H; h += blockDim.x) {
+    const unsigned int o = a.Mx[b * a.H + h];
+    const float m = o ? ordered_float(o) : -INFINITY;
+    Mh[h] = m == -INFINITY ? 0.f : m;
+    Lh[h] = 0.f;
   }
-  for (int i = tid; i < (int)(2 * kPBytes / 16); i += blockDim.x)
-    reinterpret_cast<uint4*>(sm + a.off_p)[i] = make_uint4(0, 0, 0, 0);
+  if (work) {
+    const int p0 = st_lo * PS;
+    const int np_split = min(nst * PS, (L + kPage - 1) / kPage - p0);
+    for (int e = tid; e < np_split; e += blockDim.x) bt_s[e] = a.block_table[(int64_t)b * a.max_pages + p0 + e];
+    for (int i = tid; i < (int)(NS * a.p_stage / 16); i += blockDim.x)
+      reinterpret_cast<uint4*>(sm + a.off_p)[i] = make_uint4(0, 0, 0, 0);
+  }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tslot;
+  bool ok = true;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- producer: value codes + metadata of 4 pages per stage
-      for (int k = 0; k < nst; ++k) {
-        const int cs = k % kVStages;
-        const uint32_t ph = (k / kVStages) & 1;
-        if (!mbar_wait(&cempty[cs], ph ^ 1)) {
-          set_status(a.status, kDevWaitTimeout);
-          *failed = 1;
-          break;
-        }
-        const int j0 = (st_lo + k) * kVT;
-        const int nval = min(kVT, L - j0);
-        const int np = (nval + kPage - 1) / kPage;
-        int* fl = flags + cs * kVPages;
-        uint32_t bytes = 0;
-        for (int p = 0; p < kVPages; ++p) {
-          int pid = -1;
-          if (p < np) {
-            pid = bt_s[k * kVPages + p];
-            if (pid < 0 || pid >= a.n_pages) {
-              set_status(a.status, STARKV_DEV_BAD_PAGE);
-              pid = -1;
-            } else {
-              bytes += a.codes_page + a.meta_page;
-            }
-          }
-          fl[p] = pid;
-        }
-        // score rows of the stage: one 2-D TMA box of H rows x 64 tokens (fp32)
-        bytes += a.s_stage;
-        mbar_arrive_expect_tx(&cfull[cs], bytes);
-        tma_load_2d(sm + a.off_s + cs * a.s_stage, &s_map, j0, b * a.H, &cfull[cs]);
-        for (int p = 0; p < np; ++p) {
-          const int pid = fl[p];
-          if (pid < 0) continue;
-          bulk_g2s(sm + a.off_codes + cs * a.codes_stage + p * a.codes_pitch,
-                   a.v_codes + (int64_t)pid * V.region_bytes, a.codes_page, &cfull[cs]);
-          bulk_g2s(sm + a.off_meta + cs * a.meta_stage + p * a.meta_pitch,
-                   a.v_meta + (int64_t)pid * V.groups * kPage, a.meta_page, &cfull[cs]);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer: D[mt] += Z[mt]^T P^T
-      const uint32_t idesc = make_idesc_f16(128, a.N, true, false);
-      uint32_t zc = 0;
-      bool ok = true;
-      for (int k = 0; k < nst && ok; ++k) {
-        const int ps = k & 1;
-        if (!mbar_wait(&pfull[ps], (k >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-        const uint32_t p_addr = smem_u32(sm + a.off_p + ps * kPBytes);
-        for (int mt = 0; mt < a.MT; ++mt, ++zc) {
-          const uint32_t zs = zc % kZBufs, zph = (zc / kZBufs) & 1;
-          if (!mbar_wait(&zfull[zs], zph)) {
+  if (work) {
+    const uint32_t tmem = *tslot;
+    if (warp == 0) {
+      if (lane == 0) {
+        // ---------------- producer
+        for (int k = 0; k < nst; ++k) {
+          const int cs = k % NS;
+          if (!mbar_wait(&cempty[cs], ((k / NS) & 1) ^ 1)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t z_addr = smem_u32(sm + a.off_z + zs * kZBytes);
-          for (int ks = 0; ks < kVT / 16; ++ks) {
-            const uint64_t ad = make_sdesc(z_addr + ks * 4096, 1024, 2048, 2);
-            const uint64_t bd = make_sdesc(p_addr + ks * 32, 16, 1024, 2);
-            mma_f16(tmem + mt * a.N, ad, bd, idesc, (k > 0 || ks > 0) ? 1u : 0u);
-          }
-          mma_commit(&zempty[zs]);
-        }
-        if (ok) mma_commit(&pempty[ps]);
-      }
-      if (!ok) {
-        set_status(a.status, kDevWaitTimeout);
-        *failed = 1;
-      }
-      mma_commit(dfull);
-    }
-  } else {
-    // ---------------- P and Z producers (CUDA cores), then the accumulator drain
-    const int wt = tid - 64;  // 0..255
-    uint32_t zc = 0;
-    bool ok = true;
-    for (int k = 0; k < nst && ok; ++k) {
-      const int cs = k % kVStages;
-      const int ps = k & 1;
-      if (!mbar_wait(&cfull[cs], (k / kVStages) & 1) || !mbar_wait(&pempty[ps], ((k >> 1) & 1) ^ 1)) {
-        ok = false;
-        break;
-      }
-      const int j0 = (st_lo + k) * kVT;
-      const int* fl = flags + cs * kVPages;
-      // P[h][t] = exp2(s - M_h) as fp16, K-major (row = head, 64 tokens); one item
-      // = 8 consecutive tokens of one head; l sums the fp16 values the MMA uses
-      uint8_t* pbuf = sm + a.off_p + ps * kPBytes;
-      for (int e = wt; e < a.H * (kVT / 8); e += kVWarps * 32) {
-        const int h = e / (kVT / 8), t0 = (e % (kVT / 8)) * 8;
-        uint32_t w4[4];
-        float lsum8 = 0.f;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          float pv[2];
-#pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            const int t = t0 + 2 * u + v;
-            const int j = j0 + t;
-            float p = 0.f;
-            if (j < L && fl[t / kPage] >= 0) {
-              const float sc = reinterpret_cast<const float*>(sm + a.off_s + cs * a.s_stage)[h * kVT + t];
-              if (sc != -INFINITY) p = exp2f(sc - Mh[h]);
+          const int j0 = (st_lo + k) * ST;
+          const int np = min(PS, (L - j0 + kPage - 1) / kPage);
+          int* fl = flags + cs * PS;
+          uint32_t bytes = (uint32_t)(ST / 32) * a.s_box_bytes;
+          for (int p = 0; p < PS; ++p) {
+            int pid = -1;
+            if (p < np) {
+              pid = bt_s[k * PS + p];
+              if (pid < 0 || pid >= a.n_pages) {
+                set_status(a.status, STARKV_DEV_BAD_PAGE);
+                pid = -1;
+              } else {
+                bytes += a.codes_page + a.meta_page;
+              }
             }
-            pv[v] = p;
+            fl[p] = pid;
           }
-          const __half2 h2 = __floats2half2_rn(pv[0], pv[1]);
-          lsum8 += __low2float(h2) + __high2float(h2);
-          w4[u] = *reinterpret_cast<const uint32_t*>(&h2);
+          mbar_arrive_expect_tx(&cfull[cs], bytes);
+          uint8_t* sdst = sm + a.off_s + cs * a.s_stage;
+          for (int i = 0; i < ST / 32; ++i) tma_load_2d(sdst + i * a.s_box, &s_map, j0 + 32 * i, b * a.H, &cfull[cs]);
+          for (int p = 0; p < np; ++p) {
+            const int pid = fl[p];
+            if (pid < 0) continue;
+            bulk_g2s(sm + a.off_codes + cs * a.codes_stage + p * a.codes_pitch,
+                     a.v_codes + (int64_t)pid * V.region_bytes, a.codes_page, &cfull[cs]);
+            bulk_g2s(sm + a.off_meta + cs * a.meta_stage + p * a.meta_pitch,
+                     a.v_meta + (int64_t)pid * V.groups * kPage, a.meta_page, &cfull[cs]);
+          }
         }
-        *reinterpret_cast<uint4*>(pbuf + sw128_kmajor_offset(h, t0, 64)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-        atomicAdd(&Lh[h], lsum8);
       }
-      fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&pfull[ps]);
-      // Z tiles: 64 tokens x 128 channels, MN-major (channels contiguous), fp16
-      const int q8 = (warp - 2) & 7, t = ((warp - 2) >> 3) * 32 + lane;  // warp: 16-channel group; lane: token
-      const int j = j0 + t;
-      const int pg = t / kPage, t16 = t % kPage;
-      const bool tvalid = j < L && fl[pg] >= 0;
-      const uint8_t* region = sm + a.off_codes + cs * a.codes_stage + pg * a.codes_pitch;
-      const uint32_t* meta = reinterpret_cast<const uint32_t*>(sm + a.off_meta + cs * a.meta_stage + pg * a.meta_pitch);
-      for (int mt = 0; mt < a.MT; ++mt, ++zc) {
-        const uint32_t zs = zc % kZBufs, zph = (zc / kZBufs) & 1;
-        if (!mbar_wait(&zempty[zs], zph ^ 1)) {
+    } else if (warp == 1) {
+      // ---------------- P: lane = head (and head + 32)
+      float2 lacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      float mh[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) mh[i] = lane + 32 * i < a.H ? Mh[lane + 32 * i] : 0.f;
+      for (int k = 0; k < nst && ok; ++k) {
+        const int cs = k % NS;
+        const uint32_t ph = (k / NS) & 1;
+        const bool got = mbar_wait(&cfull[cs], ph) && mbar_wait(&pempty[cs], ph ^ 1);
+        if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
-        uint8_t* zbuf = sm + a.off_z + zs * kZBytes;
-        {
-          const int m0 = q8 * 16;                    // first M position of this 16-channel group
-          const int gi = (mt * 128 + m0) >> 4;
-          uint4 c0 = make_uint4(0, 0, 0, 0), c1 = make_uint4(0, 0, 0, 0);
-          if (tvalid && gi < V.groups) {
-            const uint32_t mw = meta[gi * kPage + t16];
-            if (gi < V.top_groups)
-              dequant16_4bit(region + gi * 128 + 8 * t16, mw, c0, c1);
-            else
-              dequant16_3bit(region + V.top_groups * 128 + (gi - V.top_groups) * 96, t16, mw, c0, c1);
+        const int j0 = (st_lo + k) * ST;
+        const int* fl = flags + cs * PS;
+        bool full = j0 + ST <= L;
+        for (int p = 0; p < PS; ++p) full = full && fl[p] >= 0;
+        const uint8_t* sst = sm + a.off_s + cs * a.s_stage;
+        uint8_t* pt = sm + a.off_p + cs * a.p_stage;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int h = lane + 32 * i;
+          if (h < a.H) {
+            for (int bx = 0; bx < ST / 32; ++bx) {
+              const uint8_t* row = sst + bx * a.s_box + h * 128;  // 32 fp32 scores, 16-byte chunks swizzled by h % 8
+#pragma unroll
+              for (int c = 0; c < 8; c += 2) {
+                const float4 v0 = *reinterpret_cast<const float4*>(row + ((c ^ (h & 7)) << 4));
+                const float4 v1 = *reinterpret_cast<const float4*>(row + (((c + 1) ^ (h & 7)) << 4));
+                const int t0 = bx * 32 + 4 * c;  // first of 8 tokens, all in one page
+                float pv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+                for (int u = 0; u < 8; ++u) pv[u] = ex2_approx(pv[u] - mh[i]);
+                if (!full) {
+                  const int lim = fl[t0 >> 4] >= 0 ? L - (j0 + t0) : 0;  // tokens t0 + u valid for u < lim
+#pragma unroll
+                  for (int u = 0; u < 8; ++u) pv[u] = u < lim ? pv[u] : 0.f;
+                }
+                uint32_t w4[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  w4[u] = h2bits(__floats2half2_rn(pv[2 * u], pv[2 * u + 1]));
+                  lacc[i].x += pv[2 * u];
+                  lacc[i].y += pv[2 * u + 1];
+                }
+                *reinterpret_cast<uint4*>(pt + sw128_kmajor_offset(h, t0, a.N)) =
+                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
+              }
+            }
           }
-          *reinterpret_cast<uint4*>(zbuf + sw128_mnmajor_offset(t, m0, 2)) = c0;
-          *reinterpret_cast<uint4*>(zbuf + sw128_mnmajor_offset(t, m0 + 8, 2)) = c1;
         }
         fence_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&zfull[zs]);
+        if (lane == 0) {
+          mbar_arrive(&pfull[cs]);
+          mbar_arrive(&cempty[cs]);
+        }
       }
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        if (lane + 32 * i < a.H) Lh[lane + 32 * i] = lacc[i].x + lacc[i].y;
+    } else if (warp - 2 < a.nW) {
+      // ---------------- dequant + MMA: 16 tokens x 128 channels per stage
+      const int w = warp - 2;
+      const int mt = w % a.MT, pg = w / a.MT;
+      const int t16 = lane & 15, gsel = lane >> 4;
+      uint8_t* zt = sm + a.off_z + w * kZTile;
+      const uint32_t zaddr = smem_u32(zt);
+      const uint32_t idesc = make_idesc_f16(128, a.N, true, false);
+      const uint32_t dcol = tmem + (uint32_t)(w * a.N);
+      for (int k = 0; k < nst && ok; ++k) {
+        const int cs = k % NS;
+        const uint32_t ph = (k / NS) & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&cfull[cs], ph))) {
+          ok = false;
+          break;
+        }
+        const int j0 = (st_lo + k) * ST;
+        const bool tvalid = flags[cs * PS + pg] >= 0 && j0 + pg * kPage + t16 < L;
+        const uint8_t* region = sm + a.off_codes + cs * a.codes_stage + pg * a.codes_pitch;
+        const uint32_t* meta =
+            reinterpret_cast<const uint32_t*>(sm + a.off_meta + cs * a.meta_stage + pg * a.meta_pitch);
+        uint4 cz[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int gi = mt * 8 + gsel + 2 * i;
+          cz[2 * i] = make_uint4(0, 0, 0, 0);
+          cz[2 * i + 1] = make_uint4(0, 0, 0, 0);
+          if (tvalid && gi < V.groups) {
+            const uint32_t mw = meta[gi * kPage + t16];
+            if (gi < V.top_groups)
+              dequant16_4bit(region + gi * 128 + 8 * t16, mw, cz[2 * i], cz[2 * i + 1]);
+            else
+              dequant16_3bit(region + V.top_groups * 128 + (gi - V.top_groups) * 96, t16, mw, cz[2 * i],
+                             cz[2 * i + 1]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cempty[cs]);
+        if (!__all_sync(0xffffffffu, mbar_wait(&zempty[w], (k & 1) ^ 1))) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m0 = (gsel + 2 * i) * 16;
+          *reinterpret_cast<uint4*>(zt + sw128_mnmajor_offset(t16, m0, 2)) = cz[2 * i];
+          *reinterpret_cast<uint4*>(zt + sw128_mnmajor_offset(t16, m0 + 8, 2)) = cz[2 * i + 1];
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (mbar_wait(&pfull[cs], ph)) {
+            tc_fence_after();
+            const int kofs = pg * kPage;  // this page's tokens within the stage's P tile
+            const uint32_t pa =
+                smem_u32(sm + a.off_p + cs * a.p_stage) + (uint32_t)((kofs >> 6) * a.N * 128 + (kofs & 63) * 2);
+            mma_f16(dcol, make_sdesc(zaddr, 1024, 2048, 2), make_sdesc(pa, 16, 1024, 2), idesc, k > 0 ? 1u : 0u);
+            mma_commit(&zempty[w]);
+            mma_commit(&pempty[cs]);
+          } else {
+            ok = false;
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      }
+      if (lane == 0) mma_commit(dfull);  // arrives once this warp's MMAs are complete
       __syncwarp();
-      if (lane == 0) mbar_arrive(&cempty[cs]);
     }
-    if (!ok && lane == 0) {
-      set_status(a.status, kDevWaitTimeout);
-      *failed = 1;
-    }
-    // drain D (TMEM) into this split's partial sums (plain coalesced stores)
-    if (mbar_wait(dfull, 0)) {
-      tc_fence_after();
-      const int q4 = warp & 3, hsel = (warp - 2) >> 2;
-      float* prow = a.part + ((int64_t)b * a.splits + split) * a.H * a.R;
-      for (int mt = hsel; mt < a.MT; mt += kVWarps / 4) {
+    if (!ok && lane == 0) set_status(a.status, kDevWaitTimeout);
+
+    // ---------------- drain: page accumulators of each M tile, summed, into accs[h][ch]
+    const bool drained = __all_sync(0xffffffffu, mbar_wait_poll(dfull, 0));
+    tc_fence_after();
+    const int groups4 = (int)(blockDim.x / 32) / 4;
+    if ((warp >> 2) < groups4) {
+      const int q4 = warp & 3;
+      for (int mt = warp >> 2; mt < a.MT; mt += groups4) {
         const int mpos = mt * 128 + q4 * 32 + lane;
         const int gidx = mpos >> 4;
         const int ch = gidx * 16 + value_channel_of_position(mpos & 15, gidx < V.top_groups);
         for (int c0 = 0; c0 < a.N; c0 += 16) {
-          uint32_t r[16];
-          asm volatile(
-              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
-              "[%16];"
-              : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-                "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-                "=r"(r[15])
-              : "r"(tmem + mt * a.N + c0 + ((uint32_t)(q4 * 32) << 16)));
-          tmem_wait_row<16>(r);
+          float acc[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+          if (drained) {
+            for (int ps = 0; ps < PS; ++ps) {
+              uint32_t r[16];
+              asm volatile(
+                  "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
+                  "[%16];"
+                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                    "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                    "=r"(r[15])
+                  : "r"(tmem + (uint32_t)((mt + a.MT * ps) * a.N + c0) + ((uint32_t)(q4 * 32) << 16)));
+              tmem_wait_row<16>(r);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(r[i]);
+            }
+          }
           if (ch < a.R) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int h = c0 + i;
-              if (h < a.H) prow[(int64_t)h * a.R + ch] = __uint_as_float(r[i]);
+              if (h < a.H) accs[h * a.R + ch] = acc[i];
             }
           }
         }
       }
-    } else if (lane == 0) {
-      set_status(a.status, kDevWaitTimeout);
+    }
+    if (!drained && lane == 0) set_status(a.status, kDevWaitTimeout);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem, a.tmem_cols);
+    }
+  } else {
+    // no tokens in this split: contribute zeros to the cluster sum
+    for (int i = tid; i < a.H * a.R / 4; i += blockDim.x) reinterpret_cast<float4*>(accs)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+
+  // ---------------- cluster sum: CTA r adds channel slice r over the cluster
+  cluster_sync();
+  {
+    const uint32_t r = cluster_rank();
+    const int slice = a.R / a.CS;  // multiple of 4
+    const int per_h = slice / 4;
+    float* prow = a.part + ((int64_t)b * a.nclust + clust) * a.H * a.R;
+    for (int e = tid; e < a.H * per_h; e += blockDim.x) {
+      const int h = e / per_h, c4 = (e % per_h) * 4 + (int)r * slice;
+      const float* src = accs + h * a.R + c4;
+      float4 v[8];  // every peer's value in flight at once (cluster size <= 8)
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (q < a.CS) v[q] = dsmem_ld_f4(dsmem_addr(src, (uint32_t)q));
+      float4 sum = v[0];
+#pragma unroll
+      for (int q = 1; q < 8; ++q) {
+        if (q < a.CS) {
+          sum.x += v[q].x;
+          sum.y += v[q].y;
+          sum.z += v[q].z;
+          sum.w += v[q].w;
+        }
+      }
+      *reinterpret_cast<float4*>(prow + (int64_t)h * a.R + c4) = sum;
+    }
+    if (r == 0) {
+      for (int h = tid; h < a.H; h += blockDim.x) {
+        float l = 0.f;
+        for (int q = 0; q < a.CS; ++q) l += dsmem_ld_f32(dsmem_addr(Lh + h, (uint32_t)q));
+        a.lpart[((int64_t)b * a.nclust + clust) * a.H + h] = l;
+      }
     }
   }
-  tc_fence_before();
-  __syncthreads();
-  for (int h = tid; h < a.H; h += blockDim.x) a.lpart[((int64_t)b * a.splits + split) * a.H + h] = Lh[h];
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, a.tmem_cols);
-  }
+  cluster_sync();  // peers' shared memory stays in place until every CTA has read it
 }
 
 // ===========================================================================
@@ -918,12 +998,12 @@ __global__ void __launch_bounds__(kBThreads, 1)
 // ===========================================================================
 struct ProjArgs {
   int H, h_kv, group, d, R;
-  int splits, stages_total;
+  int splits, stages_total, st;  // value-kernel splits, stages and tokens per stage
+  int cs, nclust;                // splits per cluster, clusters (partials) per sequence
   const float* part;     // [B][splits][H][R]
   const float* lpart;    // [B][splits][H]
   float* oacc;           // [B][H][d] fp32 sums (zeroed by the score kernel)
   unsigned int* ocnt;    // [H][ceil(B/16)] arrival counters (zeroed by the score kernel)
-  const float* Smax;
   const int32_t* seq_lens;
   int tpad, max_pages, max_position;
   const __half* Bv16;
@@ -977,18 +1057,20 @@ __global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, i
         *reinterpret_cast<const uint4*>(a.Bv16 + (int64_t)(ch0 + r) * ldg + kv * d + q * 8);
   }
   // l per sequence = sum of its splits' l
+  // partials of sequence b: clusters whose first split has tokens (a prefix)
   auto n_splits = [&](int b) {
     int L = a.seq_lens[b];
     if (L < 0 || L > a.max_pages * kPage || L > a.max_position) L = 0;
-    const int nst = (L + kVT - 1) / kVT;
-    return nst > 0 ? min(a.splits, (int)(((int64_t)nst * a.splits - 1) / a.stages_total) + 1) : 0;
+    const int nst = (L + a.st - 1) / a.st;
+    const int nsp = nst > 0 ? min(a.splits, (int)(((int64_t)nst * a.splits - 1) / a.stages_total) + 1) : 0;
+    return (nsp + a.cs - 1) / a.cs;
   };
   if (tid < kProjM) {
     const int b = b0 + tid;
     float l = 0.f;
     if (b < batch) {
       const int nsp = n_splits(b);
-      for (int sp = 0; sp < nsp; ++sp) l += a.lpart[((int64_t)b * a.splits + sp) * a.H + h];
+      for (int sp = 0; sp < nsp; ++sp) l += a.lpart[((int64_t)b * a.nclust + sp) * a.H + h];
     }
     linv[tid] = l > 0.f ? 1.f / l : 0.f;
   }
@@ -1000,7 +1082,7 @@ __global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, i
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (b < batch) {
       const int nsp = n_splits(b);
-      const float* base = a.part + ((int64_t)b * a.splits * a.H + h) * R + ch0 + c4;
+      const float* base = a.part + ((int64_t)b * a.nclust * a.H + h) * R + ch0 + c4;
       const int64_t stride = (int64_t)a.H * R;
 #pragma unroll 3
       for (int sp = 0; sp < nsp; ++sp) {
@@ -1072,6 +1154,10 @@ bool tc_decode_supported(const starkv_config& cfg) {
   if (group > hpc) return false;  // a CTA's heads must cover whole KV heads
   if (cfg.num_q_heads > 64) return false;
   if (cfg.rank_v % 64 != 0) return false;  // projection stages 64-channel slices
+  // value kernel: at least two pages per stage with one N-column accumulator per warp
+  const int N = ((cfg.num_q_heads + 15) / 16) * 16;
+  const int nw_max = (512 / N) < kVMaxWarps ? 512 / N : kVMaxWarps;
+  if (((cfg.rank_v + 127) / 128) * 2 > nw_max) return false;
   return true;
 }
 
@@ -1087,9 +1173,108 @@ int sm_count() {
   return n;
 }
 
+// Shared-memory layout of the value kernel for a given split count.
+struct VSmem {
+  int NS;
+  uint32_t off_z, off_p, off_s, off_codes, off_meta, off_flags, off_bt, off_m, off_l, off_bar;
+  uint32_t p_stage, s_box, s_box_bytes, s_stage, codes_page, meta_page, codes_pitch, meta_pitch, codes_stage,
+      meta_stage, tmem_cols;
+  size_t smem;
+};
+
+bool value_smem(const Ctx& c, int N, int nW, int PS, int ST, int stages_total, int splits, VSmem& v) {
+  const starkv_config& f = c.cfg;
+  v.codes_page = c.val.region_bytes;
+  v.meta_page = c.val.groups * kPage * 4;
+  v.codes_pitch = v.codes_page + 64;
+  v.meta_pitch = v.meta_page + 64;
+  v.codes_stage = PS * v.codes_pitch;
+  v.meta_stage = PS * v.meta_pitch;
+  v.s_box_bytes = (uint32_t)f.num_q_heads * 128;       // 32 fp32 scores x H rows
+  v.s_box = (v.s_box_bytes + 1023) / 1024 * 1024;      // swizzled boxes start 1024-aligned
+  v.s_stage = (uint32_t)(ST / 32) * v.s_box;
+  v.p_stage = (uint32_t)N * (ST > 64 ? ST : 64) * 2;   // K-major fp16, 64-token rows
+  uint32_t cols = 32;
+  while (cols < (uint32_t)(nW * N)) cols <<= 1;
+  v.tmem_cols = cols;
+  const uint32_t bt_bytes = (uint32_t)(((stages_total + splits - 1) / splits + 1) * PS * 4);
+  const uint32_t fixed = (uint32_t)nW * kZTile + kVMaxStages * PS * 4 + bt_bytes + N * 8 + 64 * 8 + 1024 + 64;
+  const uint32_t per_stage = v.p_stage + v.s_stage + v.codes_stage + v.meta_stage;
+  const uint32_t budget = 227u * 1024u;
+  int ns = fixed < budget ? (int)((budget - fixed) / per_stage) : 0;
+  if (ns > kVMaxStages) ns = kVMaxStages;
+  if (ns < 2) return false;
+  v.NS = ns;
+  uint32_t o = 0;
+  v.off_z = o;
+  o += nW * kZTile;
+  v.off_p = o;
+  o += ns * v.p_stage;
+  v.off_s = o;
+  o += ns * v.s_stage;
+  v.off_codes = o;
+  o += ns * v.codes_stage;
+  v.off_meta = o;
+  o += ns * v.meta_stage;
+  v.off_flags = o;
+  o += kVMaxStages * PS * 4;
+  v.off_bt = (o + 15) / 16 * 16;
+  o = v.off_bt + bt_bytes;
+  v.off_m = (o + 15) / 16 * 16;
+  o = v.off_m + N * 4;
+  v.off_l = o;
+  o += N * 4;
+  v.off_bar = (o + 15) / 16 * 16;
+  o = v.off_bar + 64 * 8;
+  v.smem = o + 1024;
+  // the CTA's [H][R] sums reuse the pipeline's buffers, below the page table and barriers
+  return (size_t)f.num_q_heads * f.rank_v * 4 <= v.off_flags;
+}
+
+// Clusters of `cs` value CTAs that fit on the device at once (cached per device).
+int value_max_clusters(int cs, int threads, size_t smem) {
+  struct Entry {
+    int dev, cs, threads;
+    size_t smem;
+    int n;
+  };
+  static Entry cache[64];
+  static int used = 0;
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].dev == dev && cache[i].cs == cs && cache[i].threads == threads && cache[i].smem == smem)
+      return cache[i].n;
+  int n = 0;
+  if (cudaFuncSetAttribute(decode_values_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+      cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cs);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, decode_values_kernel, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  if (used < 64) cache[used++] = Entry{dev, cs, threads, smem, n};
+  return n;
+}
+
 struct TcLayout {
   int hpc, kvpc, ncols, HG, tiles_per_seq, tpad, splits, stages_total, N, MT;
-  size_t off_S, off_Smax, off_acc, off_l, off_w, off_oacc, off_ocnt, w_bytes, ws;
+  int PS, nW, ST;  // value kernel: pages per stage, dequant warps, tokens per stage
+  int CS, nclust;  // value kernel: CTAs per cluster (splits reduced on chip), clusters per sequence
+  VSmem vs;        // value kernel shared memory
+  bool ok;         // a valid value-kernel configuration exists
+  size_t off_S, off_mx, off_acc, off_l, off_w, off_oacc, off_ocnt, w_bytes, ws;
 };
 
 TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
@@ -1101,23 +1286,69 @@ TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
   t.HG = f.num_q_heads / t.hpc;
   t.tiles_per_seq = (max_pages * kPage + kT - 1) / kT;
   t.tpad = t.tiles_per_seq * kT;
-  t.stages_total = t.tpad / kVT;
-  int splits = sm_count() / (batch > 0 ? batch : 1);  // one CTA per SM: stay within a single wave
-  if (splits > t.stages_total) splits = t.stages_total;
-  if (splits < 1) splits = 1;
-  t.splits = splits;
   t.N = ((f.num_q_heads + 15) / 16) * 16;
   t.MT = (f.rank_v + 127) / 128;
+  {
+    // dequant warps = M tiles x pages per stage, each with N TMEM columns (<= 512 in all)
+    const int nw_max = (512 / t.N) < kVMaxWarps ? 512 / t.N : kVMaxWarps;
+    int ps = 1;
+    while (t.MT * ps * 2 <= nw_max) ps *= 2;
+    t.PS = ps;
+    t.nW = t.MT * ps;
+    t.ST = kPage * ps;
+  }
+  t.stages_total = (t.tpad + t.ST - 1) / t.ST;
+  {
+    // Splits per sequence (one CTA per SM: stay within a single wave) and
+    // cluster size: clusters of CS splits add their sums on chip, so only
+    // splits / CS partials per sequence cross HBM (written, then read by the
+    // projection).  A cluster must fit in one GPC, so fewer clusters of 8 than
+    // of 2 are resident at once; the split count keeps every cluster of the
+    // grid resident.  Pick the pair with the least estimated time: value bytes
+    // over the SMs in use plus the partials' traffic.
+    const int sms = sm_count();
+    const int bt = batch > 0 ? batch : 1;
+    int s0 = sms / bt;
+    if (s0 > t.stages_total) s0 = t.stages_total;
+    if (s0 < 1) s0 = 1;
+    const double tok_bytes = (double)c.val.region_bytes / kPage + c.val.groups * 4.0 + f.num_q_heads * 4.0;
+    const double work = (double)bt * t.tpad * tok_bytes;
+    const double part_unit = 2.0 * f.num_q_heads * f.rank_v * 4.0;
+    const int threads = (2 + t.nW) * 32;
+    VSmem probe;
+    t.ok = value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, 1, probe);  // largest page table
+    double best = -1.0;
+    t.splits = 1;
+    t.CS = 1;
+    for (int cs = 8; cs >= 1 && t.ok; cs >>= 1) {
+      int sp = (s0 / cs) * cs;
+      if (cs > 1 && bt * (sp / cs) > 0) {
+        const int resident = value_max_clusters(cs, threads, probe.smem);
+        const int per_seq = resident / bt;  // clusters per sequence that stay resident
+        if (sp / cs > per_seq) sp = per_seq * cs;
+      }
+      if (sp < cs || sp == 0) continue;
+      const double used = (double)bt * sp < sms ? (double)bt * sp / sms : 1.0;
+      const double cost = work / used + (double)bt * (sp / cs) * part_unit;
+      if (best < 0.0 || cost < best) {
+        best = cost;
+        t.splits = sp;
+        t.CS = cs;
+      }
+    }
+    t.nclust = t.splits / t.CS;
+    if (t.ok) t.ok = value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, t.splits, t.vs);
+  }
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
   size_t o = 0;
   t.off_S = o;
   o += al((size_t)batch * f.num_q_heads * t.tpad * 4);
-  t.off_Smax = o;
-  o += al((size_t)batch * f.num_q_heads * (t.tpad / 32) * 4);
+  t.off_mx = o;
+  o += al((size_t)batch * f.num_q_heads * 4);
   t.off_acc = o;
-  o += al((size_t)batch * t.splits * f.num_q_heads * f.rank_v * 4);
+  o += al((size_t)batch * t.nclust * f.num_q_heads * f.rank_v * 4);
   t.off_l = o;
-  o += al((size_t)batch * t.splits * f.num_q_heads * 4);
+  o += al((size_t)batch * t.nclust * f.num_q_heads * 4);
   t.w_bytes = (size_t)t.ncols * f.head_dim * 2;
   t.off_w = o;
   o += al((size_t)batch * t.HG * t.w_bytes);
@@ -1177,7 +1408,7 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   const TcLayout t = tc_layout(c, batch, max_pages);
   char* w = (char*)ws;
   float* S = (float*)(w + t.off_S);
-  float* Smax = (float*)(w + t.off_Smax);
+  unsigned int* Mx = (unsigned int*)(w + t.off_mx);
   float* acc = (float*)(w + t.off_acc);
   float* lsum = (float*)(w + t.off_l);
   uint8_t* wimg = (uint8_t*)(w + t.off_w);
@@ -1190,15 +1421,15 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
     dim3 g(f.num_q_heads, batch);
     switch (f.rank_k) {
       case 16:
-        decode_wprep_kernel<16><<<g, 64, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, f.num_q_heads, c.group, d, t.hpc,
+        decode_wprep_kernel<16><<<g, 64, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, Mx, f.num_q_heads, c.group, d, t.hpc,
                                                 t.ncols, max_pages, f.max_position);
         break;
       case 32:
-        decode_wprep_kernel<32><<<g, 64, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, f.num_q_heads, c.group, d, t.hpc,
+        decode_wprep_kernel<32><<<g, 64, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, Mx, f.num_q_heads, c.group, d, t.hpc,
                                                 t.ncols, max_pages, f.max_position);
         break;
       default:
-        decode_wprep_kernel<64><<<g, 64, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, f.num_q_heads, c.group, d, t.hpc,
+        decode_wprep_kernel<64><<<g, 64, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, Mx, f.num_q_heads, c.group, d, t.hpc,
                                                 t.ncols, max_pages, f.max_position);
         break;
     }
@@ -1235,7 +1466,7 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   A.Bk = c.Bk;
   A.rope = c.rope;
   A.S = S;
-  A.Smax = Smax;
+  A.Mx = Mx;
   A.oacc = oacc;
   A.ocnt = ocnt;
   A.oacc_elems = (int64_t)batch * f.num_q_heads * d;
@@ -1282,7 +1513,11 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   B.N = t.N;
   B.R = f.rank_v;
   B.MT = t.MT;
-  B.d = d;
+  B.PS = t.PS;
+  B.nW = t.nW;
+  B.ST = t.ST;
+  B.CS = t.CS;
+  B.nclust = t.nclust;
   B.max_pages = max_pages;
   B.tpad = t.tpad;
   B.splits = t.splits;
@@ -1293,52 +1528,55 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   B.seq_lens = seq_lens;
   B.v_codes = (const uint8_t*)cache.v_codes;
   B.v_meta = (const uint32_t*)cache.v_meta;
-  B.Smax = Smax;
+  B.Mx = Mx;
   B.part = acc;
   B.lpart = lsum;
   B.status = c.status;
-  B.codes_page = c.val.region_bytes;
-  B.meta_page = c.val.groups * kPage * 4;
-  B.codes_pitch = B.codes_page + 64;
-  B.meta_pitch = B.meta_page + 64;
-  B.codes_stage = kVPages * B.codes_pitch;
-  B.meta_stage = kVPages * B.meta_pitch;
-  B.s_stage = f.num_q_heads * kVT * 4;
-  uint32_t cols = 32;
-  while (cols < (uint32_t)(t.MT * t.N)) cols <<= 1;
-  B.tmem_cols = cols;
+  if (!t.ok) return cudaErrorInvalidConfiguration;
   {
-    uint32_t o = 0;
-    B.off_z = o;
-    o += kZBufs * kZBytes;
-    B.off_p = o;
-    o += 2 * kPBytes;
-    B.off_codes = o;
-    o += kVStages * B.codes_stage;
-    B.off_meta = o;
-    o += kVStages * B.meta_stage;
-    o = (o + 127) / 128 * 128;  // TMA destination
-    B.off_s = o;
-    o += kVStages * B.s_stage;
-    B.off_flags = o;
-    o += kVStages * kVPages * 4;
-    B.off_bt = (o + 15) / 16 * 16;
-    o = B.off_bt + ((t.stages_total + t.splits - 1) / t.splits + 1) * kVPages * 4;
-    B.off_m = (o + 15) / 16 * 16;
-    o = B.off_m + t.N * 4;
-    B.off_l = o;
-    o += t.N * 4;
-    B.off_bar = (o + 15) / 16 * 16;
-    o = B.off_bar + 32 * 8;
-    const size_t smem = o + 1024;
+    const VSmem& v = t.vs;
+    B.NS = v.NS;
+    B.off_z = v.off_z;
+    B.off_p = v.off_p;
+    B.off_s = v.off_s;
+    B.off_codes = v.off_codes;
+    B.off_meta = v.off_meta;
+    B.off_flags = v.off_flags;
+    B.off_bt = v.off_bt;
+    B.off_m = v.off_m;
+    B.off_l = v.off_l;
+    B.off_bar = v.off_bar;
+    B.p_stage = v.p_stage;
+    B.s_box = v.s_box;
+    B.s_box_bytes = v.s_box_bytes;
+    B.s_stage = v.s_stage;
+    B.codes_page = v.codes_page;
+    B.meta_page = v.meta_page;
+    B.codes_pitch = v.codes_pitch;
+    B.meta_pitch = v.meta_pitch;
+    B.codes_stage = v.codes_stage;
+    B.meta_stage = v.meta_stage;
+    B.tmem_cols = v.tmem_cols;
+    const size_t smem = v.smem;
     CUtensorMap s_map;
     if (!encode_map_2d(&s_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, S, (uint64_t)t.tpad, (uint64_t)batch * f.num_q_heads,
-                       (uint64_t)t.tpad * 4, kVT, (uint32_t)f.num_q_heads, CU_TENSOR_MAP_SWIZZLE_NONE))
+                       (uint64_t)t.tpad * 4, 32, (uint32_t)f.num_q_heads, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(decode_values_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    decode_values_kernel<<<dim3(t.splits, batch), kBThreads, smem, s>>>(s_map, B);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(t.splits, batch);
+    cfg.blockDim = dim3((2 + t.nW) * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = t.CS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_values_kernel, s_map, B);
     if (e != cudaSuccess) return e;
   }
 
@@ -1351,9 +1589,11 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   P.R = f.rank_v;
   P.splits = t.splits;
   P.stages_total = t.stages_total;
+  P.st = t.ST;
+  P.cs = t.CS;
+  P.nclust = t.nclust;
   P.part = acc;
   P.lpart = lsum;
-  P.Smax = Smax;
   P.seq_lens = seq_lens;
   P.tpad = t.tpad;
   P.max_pages = max_pages;

@@ -44,11 +44,48 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
-// Wait for phase `parity` to complete, giving up after `limit` polls.
-// Returns false on time-out (the caller records the failure and bails out).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = (1u << 22)) {
-  for (uint32_t i = 0; i < limit; ++i) {
+// One test that may suspend the thread for up to `ns` nanoseconds while the
+// phase is incomplete (the thread resumes as soon as the phase completes), so a
+// waiting warp takes no issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_test_suspend(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait by polling without suspending (for a barrier that a tcgen05.commit
+// completes, where a suspended thread may resume late), giving up after about
+// `limit_ns` nanoseconds.
+__device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 0; i < (1u << 30); ++i) {
     if (mbar_test(bar, parity)) return true;
+    if ((i & 63) == 63 && global_ns() - t0 > limit_ns) return false;
+  }
+  return false;
+}
+
+// Wait for phase `parity` to complete, giving up after about `limit_ns`
+// nanoseconds (and at most `limit` suspended tests).  Returns false on
+// time-out; the caller records the failure and winds down.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 2000000000ull,
+                                          uint32_t limit = (1u << 22)) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 0; i < limit; ++i) {
+    if (mbar_test_suspend(bar, parity, 100000u)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
   }
   return false;
 }
@@ -76,6 +113,42 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 
 // Make generic-proxy shared-memory writes visible to the async proxy (MMA / TMA reads).
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
+// Thread-block clusters: rank, barrier, distributed shared memory loads
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Every thread of every CTA in the cluster arrives (release) and waits (acquire).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ float4 dsmem_ld_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
 
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory, MMA, commit, loads

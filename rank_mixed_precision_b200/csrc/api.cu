@@ -197,14 +197,31 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
     cudaFree(c->rope);
     cudaFree(c->trig);
     cudaFree(c->Bv16);
-    cudaFree(c->zacc);
+    cudaFree(c->zpart);
     cudaFree(c->status);
     delete c;
   };
+  // small appends: K splits of the projection so that about every SM streams a
+  // slice of A (slices of 64..512 rows, 128 output columns per CTA)
+  {
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, c->device);
+    const int col_blocks = (c->lat_cols + 127) / 128;
+    c->app_splits = 0;
+    if (cfg->hidden % 64 == 0 && c->lat_cols % 8 == 0) {
+      for (int kl = 512; kl >= 64; kl >>= 1) {
+        if (cfg->hidden % kl != 0) continue;
+        if (cfg->hidden / kl > 16) break;  // the quantiser adds at most 16 split sums
+        c->app_splits = cfg->hidden / kl;
+        if ((int64_t)c->app_splits * col_blocks * 4 >= (int64_t)sms * 3) break;
+      }
+    }
+  }
   if ((e = cudaMalloc(&c->A, a_bytes)) != cudaSuccess || (e = cudaMalloc(&c->Bk, bk_bytes)) != cudaSuccess ||
       (e = cudaMalloc(&c->Bv, bv_bytes)) != cudaSuccess || (e = cudaMalloc(&c->rope, rope_bytes)) != cudaSuccess ||
       (e = cudaMalloc(&c->trig, trig_bytes)) != cudaSuccess || (e = cudaMalloc(&c->Bv16, bv_bytes / 2)) != cudaSuccess ||
-      (e = cudaMalloc(&c->zacc, (size_t)kSmallAppend * c->lat_cols * 4)) != cudaSuccess ||
+      (e = cudaMalloc(&c->zpart, (size_t)(c->app_splits > 0 ? c->app_splits : 1) * kSmallAppend * c->lat_cols * 4)) !=
+          cudaSuccess ||
       (e = cudaMalloc(&c->status, sizeof(unsigned int))) != cudaSuccess) {
     cleanup();
     return cuda_fail(e, "cudaMalloc (context factors)");
@@ -218,7 +235,6 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
   if (e == cudaSuccess) e = launch_prepare_factors(*c, (const __nv_bfloat16*)B_k, (const __nv_bfloat16*)B_v, s);
   if (e == cudaSuccess) e = launch_prepare_tc_factors(*c, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->status, 0, sizeof(unsigned int), s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(c->zacc, 0, (size_t)kSmallAppend * c->lat_cols * 4, s);
   // RoPE table: angle p * base^(-2i/d) in fp64, cos/sin in fp64, stored as fp32
   // and the same angles as an fp16 [cos.. | sin..] row per position (tensor-core operand)
   std::vector<float2> rope((size_t)cfg->max_position * half);
@@ -243,6 +259,13 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
   const char* path = getenv("STARKV_DECODE_PATH");
   const bool want_simt = path && strcmp(path, "simt") == 0;
   c->tc = !want_simt && tc_decode_supported(c->cfg) && c->val.g == 16 && make_trig_map(c);
+  if (c->app_splits > 0) {
+    const int kl = cfg->hidden / c->app_splits;
+    if (!starkv::encode_map_2d(&c->a_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->A, (uint64_t)c->lat_cols,
+                               (uint64_t)cfg->hidden, (uint64_t)c->lat_cols * 2, 64, kl < 256 ? kl : 256,
+                               CU_TENSOR_MAP_SWIZZLE_128B))
+      c->app_splits = 0;  // the general append kernel serves every size
+  }
   *out = reinterpret_cast<starkv_ctx*>(c);
   return ok();
 }
@@ -257,7 +280,7 @@ starkv_status starkv_destroy(starkv_ctx* ctx) {
   cudaFree(c->rope);
   cudaFree(c->trig);
   cudaFree(c->Bv16);
-  cudaFree(c->zacc);
+  cudaFree(c->zpart);
   cudaFree(c->status);
   delete c;
   return ok();
@@ -406,7 +429,6 @@ starkv_status starkv_read_device_status(starkv_ctx* ctx, starkv_stream_t stream,
   unsigned int h = 0;
   cudaError_t e = cudaMemcpyAsync(&h, c->status, sizeof(h), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->status, 0, sizeof(unsigned int), s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(c->zacc, 0, (size_t)kSmallAppend * c->lat_cols * 4, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "read_device_status");
   *status = h;

@@ -93,47 +93,74 @@ struct ScoreArgs {
 };
 
 // ---------------------------------------------------------------------------
-// W prep: one CTA per (sequence, head), thread i owns the frequency pair
-// (i, i + d/2) for every latent channel c:
+// W prep: one CTA per (head, 4 sequences).  With q~ the query rotated to its
+// position and i < d/2 a frequency pair (i, i + d/2), for every latent channel c
 //   W[c][i]       = (q~_i B'[c,i] + q~_{i+d/2} B'[c,i+d/2]) * log2(e)/sqrt(d)
 //   W[c][i + d/2] = (q~_{i+d/2} B'[c,i] - q~_i B'[c,i+d/2]) * log2(e)/sqrt(d)
-// with q~ the query rotated to its position.  Written as fp16 directly in the
-// score kernel's shared-memory image (K-major, 128-byte swizzle).
+// A thread owns (c, 8 consecutive i): it reads those B' values once, reuses them
+// for the 4 sequences and writes 16-byte fp16 chunks straight into the score
+// kernel's shared-memory image (K-major, 128-byte swizzle).  The CTA also zeroes
+// the running score maxima of its (sequence, head) pairs.
 // ---------------------------------------------------------------------------
+constexpr int kWpSeq = 4;  // sequences per W-prep CTA
+
 template <int RK>
-__global__ void __launch_bounds__(64) decode_wprep_kernel(const __nv_bfloat16* __restrict__ q,
-                                                          const int32_t* __restrict__ seq_lens,
-                                                          const float* __restrict__ Bk, const float2* __restrict__ rope,
-                                                          uint8_t* __restrict__ wimg, unsigned int* __restrict__ Mx,
-                                                          int H, int group, int d, int hpc, int ncols, int max_pages,
-                                                          int max_position) {
-  const int h = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
+__global__ void __launch_bounds__(128) decode_wprep_kernel(const __nv_bfloat16* __restrict__ q,
+                                                           const int32_t* __restrict__ seq_lens,
+                                                           const float* __restrict__ Bk, const float2* __restrict__ rope,
+                                                           uint8_t* __restrict__ wimg, unsigned int* __restrict__ Mx,
+                                                           int H, int group, int d, int hpc, int ncols, int batch,
+                                                           int max_pages, int max_position) {
+  __shared__ float qs[kWpSeq][2][64];  // rotated, scaled (q~_i, q~_{i+d/2}) per sequence
+  const int h = blockIdx.x, b0 = blockIdx.y * kWpSeq, tid = threadIdx.x;
   const int half = d / 2;
-  if (i == 0) Mx[b * H + h] = 0u;
-  if (i >= half) return;
-  int L = seq_lens[b];
-  if (L <= 0 || L > max_pages * kPage || L > max_position) L = 1;  // unused (no tiles), keep reads in range
   const int kv = h / group, hg = h / hpc, hl = h % hpc;
-  const float2 cs = rope[(int64_t)(L - 1) * half + i];
-  const __nv_bfloat16* qv = q + ((int64_t)b * H + h) * d;
   const float scale = kLog2e * rsqrtf((float)d);
-  const float x0 = __bfloat162float(qv[i]), x1 = __bfloat162float(qv[i + half]);
-  const float qa = (x0 * cs.x - x1 * cs.y) * scale;
-  const float qb = (x1 * cs.x + x0 * cs.y) * scale;
-  const float* B = Bk + (int64_t)kv * RK * d;
-  float ba[RK], bb[RK];
-#pragma unroll
-  for (int c = 0; c < RK; ++c) {
-    ba[c] = B[c * d + i];
-    bb[c] = B[c * d + i + half];
+  for (int e = tid; e < kWpSeq * half; e += blockDim.x) {
+    const int sb = e / half, i = e % half, b = b0 + sb;
+    float qa = 0.f, qb = 0.f;
+    if (b < batch) {
+      int L = seq_lens[b];
+      if (L <= 0 || L > max_pages * kPage || L > max_position) L = 1;  // unused (no tiles), keep reads in range
+      const float2 cs = rope[(int64_t)(L - 1) * half + i];
+      const __nv_bfloat16* qv = q + ((int64_t)b * H + h) * d;
+      const float x0 = __bfloat162float(qv[i]), x1 = __bfloat162float(qv[i + half]);
+      qa = (x0 * cs.x - x1 * cs.y) * scale;
+      qb = (x1 * cs.x + x0 * cs.y) * scale;
+      if (i == 0) Mx[b * H + h] = 0u;
+    }
+    qs[sb][0][i] = qa;
+    qs[sb][1][i] = qb;
   }
-  uint8_t* img = wimg + ((int64_t)b * (H / hpc) + hg) * ((int64_t)ncols * d * 2);
-#pragma unroll
-  for (int c = 0; c < RK; ++c) {
+  __syncthreads();
+  const float* B = Bk + (int64_t)kv * RK * d;
+  for (int e = tid; e < RK * (half / 8); e += blockDim.x) {
+    const int c = e / (half / 8), i0 = (e % (half / 8)) * 8;
+    const float4 a0 = __ldg(reinterpret_cast<const float4*>(B + c * d + i0));
+    const float4 a1 = __ldg(reinterpret_cast<const float4*>(B + c * d + i0 + 4));
+    const float4 c0 = __ldg(reinterpret_cast<const float4*>(B + c * d + half + i0));
+    const float4 c1 = __ldg(reinterpret_cast<const float4*>(B + c * d + half + i0 + 4));
+    const float ba[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float bb[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
     const int n = hl * RK + c;
-    *reinterpret_cast<__half*>(img + sw128_kmajor_offset(n, i, ncols)) = __float2half_rn(fmaf(qa, ba[c], qb * bb[c]));
-    *reinterpret_cast<__half*>(img + sw128_kmajor_offset(n, i + half, ncols)) =
-        __float2half_rn(fmaf(qb, ba[c], -qa * bb[c]));
+    for (int sb = 0; sb < kWpSeq; ++sb) {
+      const int b = b0 + sb;
+      if (b >= batch) break;
+      uint32_t lo[4], hi[4];
+#pragma unroll
+      for (int j = 0; j < 8; j += 2) {
+        const float qa0 = qs[sb][0][i0 + j], qb0 = qs[sb][1][i0 + j];
+        const float qa1 = qs[sb][0][i0 + j + 1], qb1 = qs[sb][1][i0 + j + 1];
+        const __half2 wl = __floats2half2_rn(fmaf(qa0, ba[j], qb0 * bb[j]), fmaf(qa1, ba[j + 1], qb1 * bb[j + 1]));
+        const __half2 wh = __floats2half2_rn(fmaf(qb0, ba[j], -qa0 * bb[j]), fmaf(qb1, ba[j + 1], -qa1 * bb[j + 1]));
+        lo[j / 2] = *reinterpret_cast<const uint32_t*>(&wl);
+        hi[j / 2] = *reinterpret_cast<const uint32_t*>(&wh);
+      }
+      uint8_t* img = wimg + ((int64_t)b * (H / hpc) + hg) * ((int64_t)ncols * d * 2);
+      *reinterpret_cast<uint4*>(img + sw128_kmajor_offset(n, i0, ncols)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(img + sw128_kmajor_offset(n, i0 + half, ncols)) =
+          make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    }
   }
 }
 
@@ -412,43 +439,52 @@ __global__ void __launch_bounds__(kAThreads, 1)
     if (*failed) break;
     const int ntile = t1 - t0;
     if (warp == 0) {
-      if (lane == 0) {
-        // ---------------- producer ----------------
-        for (int k = 0; k < ntile; ++k) {
-          const uint32_t c = it + k, s = c & 1, ph = (c >> 1) & 1;
-          if (!mbar_wait(&empty[s], ph ^ 1)) {
+      // ---------------- producer: one lane per copy (issued in parallel) ----------------
+      const int nsub = d / 64;
+      for (int k = 0; k < ntile; ++k) {
+        const uint32_t c = it + k, s = c & 1, ph = (c >> 1) & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1))) {
+          if (lane == 0) {
             set_status(a.status, kDevWaitTimeout);
             *failed = 1;
-            break;
           }
-          const int j0 = (t0 + k) * kT;
-          const int nval = min(kT, L - j0);
-          const int np = (nval + kPage - 1) / kPage;
-          uint32_t bytes = a.trig_stage;
-          int* fl = flags + s * kPagesPerTile;
-          for (int p = 0; p < kPagesPerTile; ++p) {
-            int pid = -1;
-            if (p < np) {
-              pid = bt_s[(j0 / kPage + p) - t0 * kPagesPerTile];
-              if (pid < 0 || pid >= a.n_pages) {
-                set_status(a.status, STARKV_DEV_BAD_PAGE);
-                pid = -1;
-              } else {
-                bytes += a.codes_page + a.meta_page;
-              }
+          break;
+        }
+        const int j0 = (t0 + k) * kT;
+        const int nval = min(kT, L - j0);
+        const int np = (nval + kPage - 1) / kPage;
+        int* fl = flags + s * kPagesPerTile;
+        if (lane < kPagesPerTile) {
+          int pid = -1;
+          if (lane < np) {
+            pid = bt_s[(j0 / kPage + lane) - t0 * kPagesPerTile];
+            if (pid < 0 || pid >= a.n_pages) {
+              set_status(a.status, STARKV_DEV_BAD_PAGE);
+              pid = -1;
             }
-            fl[p] = pid;
           }
-          mbar_arrive_expect_tx(&full[s], bytes);
-          uint8_t* trig_dst = sm + a.off_trig + s * a.trig_stage;
-          for (int sub = 0; sub < d / 64; ++sub) tma_load_2d(trig_dst + sub * 16384, &trig_map, sub * 64, j0, &full[s]);
-          for (int p = 0; p < np; ++p) {
+          fl[lane] = pid;
+        }
+        __syncwarp();
+        const int nvalid =
+            __popc(__ballot_sync(0xffffffffu, lane < kPagesPerTile && fl[lane < kPagesPerTile ? lane : 0] >= 0));
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], a.trig_stage + (uint32_t)nvalid * (a.codes_page + a.meta_page));
+        __syncwarp();
+        uint8_t* trig_dst = sm + a.off_trig + s * a.trig_stage;
+        for (int i = lane; i < nsub + 2 * kPagesPerTile; i += 32) {
+          if (i < nsub) {
+            tma_load_2d(trig_dst + i * 16384, &trig_map, i * 64, j0, &full[s]);
+          } else {
+            const int p = (i - nsub) >> 1;
             const int pid = fl[p];
-            if (pid < 0) continue;
-            bulk_g2s(sm + a.off_codes + s * a.codes_stage + p * a.codes_pitch,
-                     a.k_codes + ((int64_t)pid * a.h_kv + kv0) * a.key.region_bytes, a.codes_page, &full[s]);
-            bulk_g2s(sm + a.off_meta + s * a.meta_stage + p * a.meta_pitch,
-                     a.k_meta + ((int64_t)pid * a.h_kv + kv0) * a.key.groups * kPage, a.meta_page, &full[s]);
+            if (pid >= 0) {
+              if (((i - nsub) & 1) == 0)
+                bulk_g2s(sm + a.off_codes + s * a.codes_stage + p * a.codes_pitch,
+                         a.k_codes + ((int64_t)pid * a.h_kv + kv0) * a.key.region_bytes, a.codes_page, &full[s]);
+              else
+                bulk_g2s(sm + a.off_meta + s * a.meta_stage + p * a.meta_pitch,
+                         a.k_meta + ((int64_t)pid * a.h_kv + kv0) * a.key.groups * kPage, a.meta_page, &full[s]);
+            }
           }
         }
       }
@@ -648,9 +684,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 // One CTA per (token split, sequence); the CS splits of a cluster add their
 // sums on chip and write one partial.  Warp roles:
-//   warp 0, lane 0   producer: per stage of ST tokens, the score rows (TMA boxes
+//   warp 0           producer: per stage of ST tokens, the score rows (TMA boxes
 //                    of 32 tokens x H heads, 128-byte swizzle) and the value
-//                    codes + metadata of its PS pages (bulk copies), NS stages deep
+//                    codes + metadata of its PS pages (bulk copies, one lane per
+//                    copy), NS stages deep
 //   warp 1           P: lane = head; P[h, t] = exp2(s - M_h) as fp16 into a
 //                    K-major tile, l_h summed in registers
 //   warps 2..nW+1    dequant warp w = (M tile w % MT, page w / MT of the stage):
@@ -734,45 +771,52 @@ __global__ void __launch_bounds__(kVThreads, 1)
   if (work) {
     const uint32_t tmem = *tslot;
     if (warp == 0) {
-      if (lane == 0) {
-        // ---------------- producer
-        for (int k = 0; k < nst; ++k) {
-          const int cs = k % NS;
-          if (!mbar_wait(&cempty[cs], ((k / NS) & 1) ^ 1)) {
-            ok = false;
-            break;
-          }
-          const int j0 = (st_lo + k) * ST;
-          const int np = min(PS, (L - j0 + kPage - 1) / kPage);
-          int* fl = flags + cs * PS;
-          uint32_t bytes = (uint32_t)(ST / 32) * a.s_box_bytes;
-          for (int p = 0; p < PS; ++p) {
-            int pid = -1;
-            if (p < np) {
-              pid = bt_s[k * PS + p];
-              if (pid < 0 || pid >= a.n_pages) {
-                set_status(a.status, STARKV_DEV_BAD_PAGE);
-                pid = -1;
-              } else {
-                bytes += a.codes_page + a.meta_page;
-              }
+      // ---------------- producer: one lane per copy (a bulk copy costs its issuing
+      // thread about as long as the next copy's latency would, so issue in parallel)
+      const int nbox = ST / 32;
+      for (int k = 0; k < nst; ++k) {
+        const int cs = k % NS;
+        if (!__all_sync(0xffffffffu, mbar_wait(&cempty[cs], ((k / NS) & 1) ^ 1))) {
+          ok = false;
+          break;
+        }
+        const int j0 = (st_lo + k) * ST;
+        const int np = min(PS, (L - j0 + kPage - 1) / kPage);
+        int* fl = flags + cs * PS;
+        if (lane < PS) {
+          int pid = -1;
+          if (lane < np) {
+            pid = bt_s[k * PS + lane];
+            if (pid < 0 || pid >= a.n_pages) {
+              set_status(a.status, STARKV_DEV_BAD_PAGE);
+              pid = -1;
             }
-            fl[p] = pid;
           }
-          mbar_arrive_expect_tx(&cfull[cs], bytes);
-          uint8_t* sdst = sm + a.off_s + cs * a.s_stage;
-          for (int i = 0; i < ST / 32; ++i) tma_load_2d(sdst + i * a.s_box, &s_map, j0 + 32 * i, b * a.H, &cfull[cs]);
-          for (int p = 0; p < np; ++p) {
+          fl[lane] = pid;
+        }
+        __syncwarp();
+        const int nvalid = __popc(__ballot_sync(0xffffffffu, lane < PS && fl[lane < PS ? lane : 0] >= 0));
+        if (lane == 0)
+          mbar_arrive_expect_tx(&cfull[cs], (uint32_t)nbox * a.s_box_bytes + (uint32_t)nvalid * (a.codes_page + a.meta_page));
+        __syncwarp();
+        uint8_t* sdst = sm + a.off_s + cs * a.s_stage;
+        for (int i = lane; i < nbox + 2 * PS; i += 32) {
+          if (i < nbox) {
+            tma_load_2d(sdst + i * a.s_box, &s_map, j0 + 32 * i, b * a.H, &cfull[cs]);
+          } else {
+            const int p = (i - nbox) >> 1;
             const int pid = fl[p];
-            if (pid < 0) continue;
-            bulk_g2s(sm + a.off_codes + cs * a.codes_stage + p * a.codes_pitch,
-                     a.v_codes + (int64_t)pid * V.region_bytes, a.codes_page, &cfull[cs]);
-            bulk_g2s(sm + a.off_meta + cs * a.meta_stage + p * a.meta_pitch,
-                     a.v_meta + (int64_t)pid * V.groups * kPage, a.meta_page, &cfull[cs]);
+            if (pid >= 0) {
+              if (((i - nbox) & 1) == 0)
+                bulk_g2s(sm + a.off_codes + cs * a.codes_stage + p * a.codes_pitch,
+                         a.v_codes + (int64_t)pid * V.region_bytes, a.codes_page, &cfull[cs]);
+              else
+                bulk_g2s(sm + a.off_meta + cs * a.meta_stage + p * a.meta_pitch,
+                         a.v_meta + (int64_t)pid * V.groups * kPage, a.meta_page, &cfull[cs]);
+            }
           }
         }
       }
-      __syncwarp();
     } else if (warp == 1) {
       // ---------------- P: lane = head (and head + 32)
       float2 lacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -1010,98 +1054,92 @@ struct ProjArgs {
   __nv_bfloat16* out;
 };
 
-constexpr int kProjM = 16;    // sequences per projection CTA (the MMA's M)
-constexpr int kProjK = 64;    // channels per staged B'_v slice
+constexpr int kProjM = 16;   // sequences per projection CTA (the MMA's M)
+constexpr int kProjC = 128;  // latent channels per projection CTA
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t& r0, uint32_t& r1) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
-}
-__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// grid (H, R / kProjK, ceil(B / 16)), 256 threads; warp w owns output columns
-// [16 w, 16 w + 16) (d = 64: warps 4..7 idle in the MMA).  Each CTA multiplies a
-// 64-channel slice, o_lat[16 seq x 64] (fp16, = acc / l) . B'_v[64 x d], adds it
-// into the fp32 sums and the last CTA of a (head, sequence block) to arrive
-// writes the bf16 output (arrival counter, no waiting).
-constexpr int kProjC = 256;  // channels per projection CTA
-
-__global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, int batch, int slices) {
-  extern __shared__ __align__(16) uint8_t proj_smem[];
-  __half(*As)[kProjC + 8] = reinterpret_cast<__half(*)[kProjC + 8]>(proj_smem);                 // [16][256 + 8]
-  __half(*Bs)[128 + 8] = reinterpret_cast<__half(*)[128 + 8]>(proj_smem + kProjM * (kProjC + 8) * 2);  // [256][136]
+// grid (H, R / kc, ceil(B / 16)), 256 threads, kc = 128 channels (64 when R is
+// not a multiple of 128).  Every load of the CTA (its
+// B'_v slice, the partial sums and l of its sequences) is issued up front; then
+// o_lat[16 seq x 128] (fp16, = acc / l) . B'_v[128 x d] on mma.sync (warp w owns
+// output columns [16 w, 16 w + 16); d = 64 leaves warps 4..7 idle), added into
+// the fp32 sums, and the last CTA of a (head, sequence block) to arrive writes
+// the bf16 output (arrival counter, no waiting).
+__global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, int batch, int kc) {
+  __shared__ __align__(16) __half As[kProjM][kProjC + 8];
+  __shared__ __align__(16) __half Bs[kProjC][128 + 8];
   __shared__ float linv[kProjM];
+  __shared__ int nparts_s[kProjM];
   __shared__ int last;
   const int R = a.R, d = a.d;
-  const int h = blockIdx.x, kc = blockIdx.y, bc = blockIdx.z;
+  const int h = blockIdx.x, ch0 = blockIdx.y * kc, bc = blockIdx.z;
   const int b0 = bc * kProjM;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int kv = h / a.group;
   const int ldg = a.h_kv * d;
-  const int nch = slices * kProjK;           // channels of this CTA (<= 256)
-  const int ch0 = kc * nch;
-  // B'_v rows of this chunk: issue every load first
-  for (int e = tid; e < nch * (d / 8); e += 256) {
-    const int r = e / (d / 8), q = e % (d / 8);
-    *reinterpret_cast<uint4*>(&Bs[r][q * 8]) =
-        *reinterpret_cast<const uint4*>(a.Bv16 + (int64_t)(ch0 + r) * ldg + kv * d + q * 8);
-  }
-  // l per sequence = sum of its splits' l
   // partials of sequence b: clusters whose first split has tokens (a prefix)
-  auto n_splits = [&](int b) {
-    int L = a.seq_lens[b];
-    if (L < 0 || L > a.max_pages * kPage || L > a.max_position) L = 0;
-    const int nst = (L + a.st - 1) / a.st;
-    const int nsp = nst > 0 ? min(a.splits, (int)(((int64_t)nst * a.splits - 1) / a.stages_total) + 1) : 0;
-    return (nsp + a.cs - 1) / a.cs;
-  };
+  if (tid < kProjM) {
+    const int b = b0 + tid;
+    int np = 0;
+    if (b < batch) {
+      int L = a.seq_lens[b];
+      if (L < 0 || L > a.max_pages * kPage || L > a.max_position) L = 0;
+      const int nst = (L + a.st - 1) / a.st;
+      const int nsp = nst > 0 ? min(a.splits, (int)(((int64_t)nst * a.splits - 1) / a.stages_total) + 1) : 0;
+      np = (nsp + a.cs - 1) / a.cs;
+    }
+    nparts_s[tid] = np;
+  }
+  // B'_v rows of this slice straight into shared memory
+  for (int e = tid; e < kc * (d / 8); e += 256) {
+    const int r = e / (d / 8), q8 = e % (d / 8);
+    *reinterpret_cast<uint4*>(&Bs[r][q8 * 8]) =
+        __ldg(reinterpret_cast<const uint4*>(a.Bv16 + (int64_t)(ch0 + r) * ldg + kv * d + q8 * 8));
+  }
+  __syncthreads();
   if (tid < kProjM) {
     const int b = b0 + tid;
     float l = 0.f;
-    if (b < batch) {
-      const int nsp = n_splits(b);
-      for (int sp = 0; sp < nsp; ++sp) l += a.lpart[((int64_t)b * a.nclust + sp) * a.H + h];
-    }
+    for (int sp = 0; sp < nparts_s[tid]; ++sp) l += __ldcg(a.lpart + ((int64_t)b * a.nclust + sp) * a.H + h);
     linv[tid] = l > 0.f ? 1.f / l : 0.f;
   }
-  __syncthreads();
-  // o_lat = (sum over splits of the partials) / l, four channels per item
-  for (int e = tid; e < kProjM * (nch / 4); e += 256) {
-    const int r = e / (nch / 4), c4 = (e % (nch / 4)) * 4;
+  // o_lat sums: 2 items of 4 channels per thread (16 sequences x 32 quads)
+  float4 acc[2];
+  const int items = kProjM * (kc / 4);
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int e = tid + it * 256;
+    const int r = e / (kc / 4), c4 = (e % (kc / 4)) * 4;
     const int b = b0 + r;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (b < batch) {
-      const int nsp = n_splits(b);
+    acc[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e < items && b < batch) {
+      const int np = nparts_s[r];
       const float* base = a.part + ((int64_t)b * a.nclust * a.H + h) * R + ch0 + c4;
       const int64_t stride = (int64_t)a.H * R;
-#pragma unroll 3
-      for (int sp = 0; sp < nsp; ++sp) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(base + sp * stride));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+#pragma unroll 4
+      for (int sp = 0; sp < np; ++sp) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(base + sp * stride));
+        acc[it].x += v.x;
+        acc[it].y += v.y;
+        acc[it].z += v.z;
+        acc[it].w += v.w;
       }
     }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int e = tid + it * 256;
+    if (e >= items) break;
+    const int r = e / (kc / 4), c4 = (e % (kc / 4)) * 4;
     const float li = linv[r];
-    *reinterpret_cast<__half2*>(&As[r][c4]) = __floats2half2_rn(acc.x * li, acc.y * li);
-    *reinterpret_cast<__half2*>(&As[r][c4 + 2]) = __floats2half2_rn(acc.z * li, acc.w * li);
+    *reinterpret_cast<__half2*>(&As[r][c4]) = __floats2half2_rn(acc[it].x * li, acc[it].y * li);
+    *reinterpret_cast<__half2*>(&As[r][c4 + 2]) = __floats2half2_rn(acc[it].z * li, acc[it].w * li);
   }
   __syncthreads();
   float c[2][4] = {};
   if (warp * 16 < d) {
 #pragma unroll 4
-    for (int kk = 0; kk < nch; kk += 16) {
+    for (int kk = 0; kk < kc; kk += 16) {
       uint32_t a0, a1, a2, a3;
       ldsm_x4(sm100::smem_u32(&As[lane & 15][kk + (lane >> 4) * 8]), a0, a1, a2, a3);
 #pragma unroll
@@ -1111,8 +1149,6 @@ __global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, i
         mma16816(c[nt], a0, a1, a2, a3, b0r, b1r);
       }
     }
-  }
-  if (warp * 16 < d) {
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       const int col = warp * 16 + nt * 8 + (lane & 3) * 2;
@@ -1153,7 +1189,7 @@ bool tc_decode_supported(const starkv_config& cfg) {
   if (hpc % group != 0 && group % hpc != 0) return false;
   if (group > hpc) return false;  // a CTA's heads must cover whole KV heads
   if (cfg.num_q_heads > 64) return false;
-  if (cfg.rank_v % 64 != 0) return false;  // projection stages 64-channel slices
+  if (cfg.rank_v % 64 != 0) return false;  // projection CTAs own 128- or 64-channel slices
   // value kernel: at least two pages per stage with one N-column accumulator per warp
   const int N = ((cfg.num_q_heads + 15) / 16) * 16;
   const int nw_max = (512 / N) < kVMaxWarps ? 512 / N : kVMaxWarps;
@@ -1418,19 +1454,19 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
 
   // ---------------- W images: rotated query folded into B'_k, per (sequence, head)
   {
-    dim3 g(f.num_q_heads, batch);
+    dim3 g(f.num_q_heads, (batch + kWpSeq - 1) / kWpSeq);
     switch (f.rank_k) {
       case 16:
-        decode_wprep_kernel<16><<<g, 64, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, Mx, f.num_q_heads, c.group, d, t.hpc,
-                                                t.ncols, max_pages, f.max_position);
+        decode_wprep_kernel<16><<<g, 128, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, Mx, f.num_q_heads, c.group, d, t.hpc,
+                                                 t.ncols, batch, max_pages, f.max_position);
         break;
       case 32:
-        decode_wprep_kernel<32><<<g, 64, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, Mx, f.num_q_heads, c.group, d, t.hpc,
-                                                t.ncols, max_pages, f.max_position);
+        decode_wprep_kernel<32><<<g, 128, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, Mx, f.num_q_heads, c.group, d, t.hpc,
+                                                 t.ncols, batch, max_pages, f.max_position);
         break;
       default:
-        decode_wprep_kernel<64><<<g, 64, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, Mx, f.num_q_heads, c.group, d, t.hpc,
-                                                t.ncols, max_pages, f.max_position);
+        decode_wprep_kernel<64><<<g, 128, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, Mx, f.num_q_heads, c.group, d, t.hpc,
+                                                 t.ncols, batch, max_pages, f.max_position);
         break;
     }
     cudaError_t e = cudaGetLastError();
@@ -1602,14 +1638,8 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   P.out = out;
   P.oacc = oacc;
   P.ocnt = ocnt;
-  const int slices = f.rank_v % (4 * kProjK) == 0 ? 4 : (f.rank_v % (2 * kProjK) == 0 ? 2 : 1);
-  const size_t psmem = (size_t)kProjM * (kProjC + 8) * 2 + (size_t)kProjC * (128 + 8) * 2;
-  {
-    cudaError_t e = cudaFuncSetAttribute(decode_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
-    if (e != cudaSuccess) return e;
-  }
-  decode_project_kernel<<<dim3(f.num_q_heads, f.rank_v / (kProjK * slices), (batch + kProjM - 1) / kProjM), 256, psmem,
-                          s>>>(P, batch, slices);
+  const int kc = f.rank_v % kProjC == 0 ? kProjC : 64;
+  decode_project_kernel<<<dim3(f.num_q_heads, f.rank_v / kc, (batch + kProjM - 1) / kProjM), 256, 0, s>>>(P, batch, kc);
   return cudaGetLastError();
 }
 

@@ -42,7 +42,9 @@ struct Ctx {
   float2* rope;           // [max_position][d_h/2] (cos, sin), built in fp64
   __half* trig;           // [max_position][d_h] fp16: cos(p th_0..), sin(p th_0..) (tensor-core operand)
   __half* Bv16;           // [R][h_kv*d_h] fp16, B'_v
-  float* zacc;            // [kSmallAppend][h_kv*r_k + R] fp32 split-K sums of small appends (kept zero)
+  float* zpart;           // [app_splits][kSmallAppend][lat_cols] fp32 split-K sums of small appends
+  int app_splits;         // K splits of the small-append projection (0: that path is off)
+  CUtensorMap a_map;      // TMA map of `A`: box 64 columns x min(256, hidden / app_splits) rows, 128-byte swizzle
   unsigned int* status;   // device status word
   CUtensorMap trig_map;   // TMA map of `trig`: box 64 x 128, 128-byte swizzle
   bool tc;                // tensor-core decode available for this shape

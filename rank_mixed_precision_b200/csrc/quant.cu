@@ -7,6 +7,7 @@
 // eq. 13 (block-diagonal orthogonal rotation, absorbed by the up-projection)
 // and eq. 14 (4-bit leading channels, 3-bit the rest).
 #include "internal.cuh"
+#include "sm100.cuh"
 
 namespace starkv {
 
@@ -236,98 +237,154 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
 
 // ---------------------------------------------------------------------------
 // Small appends (a decode step adds one token per sequence): the projection is
-// a thin GEMM bound by reading A once.  Split K over 128-row slices so the whole
-// GPU streams A: each CTA owns 64 columns x 128 rows of A and adds its n x 64
-// partial sums into the context's fp32 buffer; a second kernel rotates,
-// quantises and packs each (token, group) and returns the buffer to zero.
+// a thin GEMM bound by reading A once.  Split K so the whole GPU streams A: a
+// CTA owns 128 columns x KL rows of A, fetched as a few 128-byte-swizzled TMA
+// boxes that are all in flight at once, multiplies the n x KL slice of X into
+// them (mma.sync, fp32 accumulators) and writes its n x 128 partial sums to
+// its own slot of the context's split buffer; the quantise kernel adds the
+// splits in a fixed order (deterministic), rotates, quantises and packs.
 // ---------------------------------------------------------------------------
-constexpr int kSkRows = 128, kSkCols = 64;
+constexpr int kAgCols = 128;  // output columns per CTA: 8 warps x 16
 
-constexpr int kSkSub = 4;  // 128-row sub-slices per CTA
-
-__global__ void __launch_bounds__(256) append_splitk_kernel(AppendArgs a, float* zacc) {
-  __shared__ __align__(16) __nv_bfloat16 As[kSkRows][kSkCols];   // 16 KB
-  __shared__ __nv_bfloat16 Xs[kSmallAppend][kSkRows];             // 16 KB
-  const int tid = threadIdx.x;
-  const int col0 = blockIdx.x * kSkCols;
-  const int n = (int)a.n;
-  const int cq = (tid % 16) * 4;
-  float acc[kSmallAppend / 16][4] = {};
-  for (int sub = 0; sub < kSkSub; ++sub) {
-    const int k0 = (blockIdx.y * kSkSub + sub) * kSkRows;
-    if (k0 >= a.hidden) break;
-    __syncthreads();
-    for (int e = tid; e < kSkRows * (kSkCols / 8); e += 256) {
-      const int r = e / (kSkCols / 8), q = e % (kSkCols / 8);
-      const int col = col0 + q * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (col < a.lat_cols) v = *reinterpret_cast<const uint4*>(a.A + (int64_t)(k0 + r) * a.lat_cols + col);
-      *reinterpret_cast<uint4*>(&As[r][q * 8]) = v;
+__global__ void __launch_bounds__(256, 1)
+    append_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const AppendArgs a, int KL, float* zpart) {
+  extern __shared__ uint8_t ag_smem[];
+  uint8_t* sm = ag_smem + ((1024u - (sm100::smem_u32(ag_smem) & 1023u)) & 1023u);
+  __shared__ uint64_t bar;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c0 = blockIdx.x * kAgCols, ks = blockIdx.y, k0 = ks * KL;
+  const int n = (int)a.n, mtiles = (n + 15) / 16;
+  const int box_rows = KL < 256 ? KL : 256;
+  const int nbox = 2 * (KL / box_rows);
+  if (tid == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  // A slice: two 64-column halves of KL rows (128-byte rows, 128-byte swizzle)
+  if (warp == 0) {
+    if (lane == 0) sm100::mbar_arrive_expect_tx(&bar, (uint32_t)KL * kAgCols * 2);
+    __syncwarp();
+    for (int i = lane; i < nbox; i += 32) {
+      const int half = i & 1, rb = i >> 1;
+      sm100::tma_load_2d(sm + half * KL * 128 + rb * box_rows * 128, &a_map, c0 + half * 64, k0 + rb * box_rows, &bar);
     }
-    for (int e = tid; e < n * kSkRows; e += 256) {
-      const int i = e / kSkRows, k = e % kSkRows;
-      Xs[i][k] = a.X[(int64_t)i * a.hidden + k0 + k];
-    }
-    __syncthreads();
+  }
+  // X slice (rows >= n are zero), row stride KL + 8 elements against bank conflicts
+  __nv_bfloat16* Xs = reinterpret_cast<__nv_bfloat16*>(sm + 2 * KL * 128);
+  const int xs = KL + 8;
+  for (int e = tid; e < mtiles * 16 * (KL / 8); e += blockDim.x) {
+    const int r = e / (KL / 8), q = e % (KL / 8);
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < n) v = *reinterpret_cast<const uint4*>(a.X + (int64_t)r * a.hidden + k0 + q * 8);
+    *reinterpret_cast<uint4*>(Xs + r * xs + q * 8) = v;
+  }
+  __syncthreads();
+  if (!__all_sync(0xffffffffu, sm100::mbar_wait(&bar, 0))) {
+    if (lane == 0) set_status(a.status, kDevWaitTimeout);
+    return;
+  }
+  const int half = warp >> 2, wc = (warp & 3) * 16;  // this warp's 16 columns inside its 64-column half
+  const uint8_t* At = sm + half * KL * 128;
+  float acc[kSmallAppend / 16][2][4] = {};
+  for (int kk = 0; kk < KL; kk += 16) {
+    uint32_t b[2][2];
 #pragma unroll
-    for (int ii = 0; ii < kSmallAppend / 16; ++ii) {
-      const int i = tid / 16 + 16 * ii;
-      if (i >= n) break;
-      for (int k = 0; k < kSkRows; ++k) {
-        const float x = __bfloat162float(Xs[i][k]);
-        const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&As[k][cq]);
-        const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&As[k][cq + 2]);
-        acc[ii][0] = fmaf(x, __low2float(w01), acc[ii][0]);
-        acc[ii][1] = fmaf(x, __high2float(w01), acc[ii][1]);
-        acc[ii][2] = fmaf(x, __low2float(w23), acc[ii][2]);
-        acc[ii][3] = fmaf(x, __high2float(w23), acc[ii][3]);
+    for (int nt = 0; nt < 2; ++nt) {
+      const int k = kk + (lane & 15);
+      const int chunk = ((wc + nt * 8) >> 3) ^ (k & 7);
+      sm100::ldsm_x2_t(sm100::smem_u32(At + k * 128 + chunk * 16), b[nt][0], b[nt][1]);
+    }
+#pragma unroll
+    for (int mt = 0; mt < kSmallAppend / 16; ++mt) {
+      if (mt < mtiles) {
+        uint32_t a0, a1, a2, a3;
+        sm100::ldsm_x4(sm100::smem_u32(Xs + (mt * 16 + (lane & 15)) * xs + kk + (lane >> 4) * 8), a0, a1, a2, a3);
+        sm100::mma16816_bf16(acc[mt][0], a0, a1, a2, a3, b[0][0], b[0][1]);
+        sm100::mma16816_bf16(acc[mt][1], a0, a1, a2, a3, b[1][0], b[1][1]);
       }
     }
   }
+  float* zp = zpart + (int64_t)ks * kSmallAppend * a.lat_cols;
 #pragma unroll
-  for (int ii = 0; ii < kSmallAppend / 16; ++ii) {
-    const int i = tid / 16 + 16 * ii;
-    if (i >= n) break;
+  for (int mt = 0; mt < kSmallAppend / 16; ++mt) {
+    if (mt >= mtiles) break;
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (col0 + cq + j < a.lat_cols) atomicAdd(&zacc[(int64_t)i * a.lat_cols + col0 + cq + j], acc[ii][j]);
+    for (int nt = 0; nt < 2; ++nt) {
+      const int col = c0 + half * 64 + wc + nt * 8 + (lane & 3) * 2;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int r = mt * 16 + (lane >> 2) + hf * 8;
+        if (r < n && col < a.lat_cols)
+          *reinterpret_cast<float2*>(zp + (int64_t)r * a.lat_cols + col) =
+              make_float2(acc[mt][nt][hf * 2], acc[mt][nt][hf * 2 + 1]);
+      }
+    }
   }
 }
 
-// one thread per (token, 4-column unit); the unit that starts a group quantises it
-__global__ void append_quant_kernel(AppendArgs a, float* zacc) {
+// One thread per (token, 4 columns): it adds its columns' split sums (every
+// load in flight at once), then the group's leader gathers the group's g values
+// from its neighbours by shuffles (groups never straddle a warp: they start on
+// multiples of g <= 16 columns and a warp covers 128) and rotates, quantises and
+// packs them.
+constexpr int kMaxAppSplits = 16;
+
+__global__ void __launch_bounds__(128) append_quant_kernel(AppendArgs a, const float* zpart, int splits) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int units = a.lat_cols / 4;
-  if (idx >= a.n * units) return;
-  const int64_t row = idx / units;
-  const int col = (int)(idx % units) * 4;
-  float* z = zacc + row * a.lat_cols + col;
+  const bool active = idx < a.n * units;
+  const int64_t row = active ? idx / units : 0;
+  const int col = active ? (int)(idx % units) * 4 : 0;
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (active) {
+    float4 part[kMaxAppSplits];
+#pragma unroll
+    for (int sp = 0; sp < kMaxAppSplits; ++sp)
+      if (sp < splits)
+        part[sp] = __ldcg(reinterpret_cast<const float4*>(zpart + ((int64_t)sp * kSmallAppend + row) * a.lat_cols + col));
+#pragma unroll
+    for (int sp = 0; sp < kMaxAppSplits; ++sp) {  // fixed order: deterministic sums
+      if (sp < splits) {
+        v.x += part[sp].x;
+        v.y += part[sp].y;
+        v.z += part[sp].z;
+        v.w += part[sp].w;
+      }
+    }
+  }
   const int key_cols = a.h_kv * a.key.r;
   const bool is_key = col < key_cols;
   const LatentGeom& L = is_key ? a.key : a.val;
   const int cin = is_key ? col % a.key.r : col - key_cols;
-  if (cin % L.g == 0) {
-    float x[16];
-    for (int i = 0; i < L.g; ++i) x[i] = z[i];
-    if (a.lat_out)
-      for (int i = 0; i < L.g; ++i) a.lat_out[row * a.lat_cols + col + i] = x[i];
-    const int64_t slot = a.slots[row];
-    if (slot >= a.n_pages * kPage) {
-      set_status(a.status, STARKV_DEV_BAD_SLOT);
-    } else if (slot >= 0) {
-      const int64_t page = slot / kPage;
-      const int t = (int)(slot % kPage);
-      const int gi = cin / L.g;
-      if (is_key) {
-        const int kv = col / a.key.r;
-        rotate_quantize_store_any(x, L, gi, a.k_codes + (page * a.h_kv + kv) * L.region_bytes,
-                                  a.k_meta + (page * a.h_kv + kv) * L.groups * kPage, t, a.status);
-      } else {
-        rotate_quantize_store_any(x, L, gi, a.v_codes + page * L.region_bytes, a.v_meta + page * L.groups * kPage,
-                                  t, a.status);
-      }
+  const int lane = threadIdx.x & 31;
+  float x[16];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {  // units lane .. lane + 3 (a group spans g / 4 <= 4 of them)
+    const int src = lane + j < 32 ? lane + j : 31;
+    x[4 * j] = __shfl_sync(0xffffffffu, v.x, src);
+    x[4 * j + 1] = __shfl_sync(0xffffffffu, v.y, src);
+    x[4 * j + 2] = __shfl_sync(0xffffffffu, v.z, src);
+    x[4 * j + 3] = __shfl_sync(0xffffffffu, v.w, src);
+  }
+  if (!active || cin % L.g != 0) return;
+  if (a.lat_out)
+    for (int i = 0; i < L.g; ++i) a.lat_out[row * a.lat_cols + col + i] = x[i];
+  const int64_t slot = a.slots[row];
+  if (slot >= a.n_pages * kPage) {
+    set_status(a.status, STARKV_DEV_BAD_SLOT);
+  } else if (slot >= 0) {
+    const int64_t page = slot / kPage;
+    const int t = (int)(slot % kPage);
+    const int gi = cin / L.g;
+    if (is_key) {
+      const int kv = col / a.key.r;
+      rotate_quantize_store_any(x, L, gi, a.k_codes + (page * a.h_kv + kv) * L.region_bytes,
+                                a.k_meta + (page * a.h_kv + kv) * L.groups * kPage, t, a.status);
+    } else {
+      rotate_quantize_store_any(x, L, gi, a.v_codes + page * L.region_bytes, a.v_meta + page * L.groups * kPage,
+                                t, a.status);
     }
-    for (int i = 0; i < L.g; ++i) z[i] = 0.f;  // leave the buffer zeroed for the next call
   }
 }
 
@@ -351,12 +408,15 @@ cudaError_t launch_append(const Ctx& c, const starkv_cache& cache, const __nv_bf
   a.k_meta = (uint32_t*)cache.k_meta;
   a.v_meta = (uint32_t*)cache.v_meta;
   a.status = c.status;
-  if (n <= kSmallAppend && c.cfg.hidden % kSkRows == 0) {
-    dim3 g1((unsigned)((c.lat_cols + kSkCols - 1) / kSkCols),
-            (unsigned)((c.cfg.hidden / kSkRows + kSkSub - 1) / kSkSub));
-    append_splitk_kernel<<<g1, 256, 0, s>>>(a, c.zacc);
+  if (n <= kSmallAppend && c.app_splits > 0 && (reinterpret_cast<uintptr_t>(X) & 15) == 0) {
+    const int KL = c.cfg.hidden / c.app_splits;
+    const size_t smem = (size_t)2 * KL * 128 + (size_t)((n + 15) / 16) * 16 * (KL + 8) * 2 + 1024;
+    cudaError_t e = cudaFuncSetAttribute(append_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 g1((unsigned)((c.lat_cols + kAgCols - 1) / kAgCols), (unsigned)c.app_splits);
+    append_gemm_kernel<<<g1, 256, smem, s>>>(c.a_map, a, KL, c.zpart);
     const int64_t units = n * (c.lat_cols / 4);
-    append_quant_kernel<<<(unsigned)((units + 127) / 128), 128, 0, s>>>(a, c.zacc);
+    append_quant_kernel<<<(unsigned)((units + 127) / 128), 128, 0, s>>>(a, c.zpart, c.app_splits);
     return cudaGetLastError();
   }
   dim3 grid((unsigned)((n + kAppBM - 1) / kAppBM), (unsigned)((c.lat_cols + kAppBN - 1) / kAppBN));

@@ -89,6 +89,7 @@ struct ScoreArgs {
   unsigned int* status;
   uint32_t off_trig, off_codes, off_meta, off_flags, off_bt, off_bar;
   uint32_t trig_stage, codes_page, meta_page, codes_stage, meta_stage, w_bytes;
+  int NK;  // key-stage ring depth (the position tiles use two stages)
   uint32_t codes_pitch, meta_pitch;  // shared-memory page strides (padded against bank conflicts)
 };
 
@@ -166,6 +167,7 @@ __global__ void __launch_bounds__(128) decode_wprep_kernel(const __nv_bfloat16* 
 
 // TMEM columns of the score accumulators: two buffers of up to 256 columns.
 constexpr uint32_t kScoreTmemCols = 512;
+constexpr int kMaxKeyStages = 6;  // deepest key-stage ring
 
 // Issue the TMEM loads of one RK-column row into raw registers (no wait).
 template <int RK>
@@ -227,113 +229,111 @@ __device__ __forceinline__ void tmem_load_row(uint32_t taddr, float (&G)[RK]) {
 // Key dot product on packed codes (one token, one head), compile-time layout.
 //
 // Codes become floats by writing their bits into the mantissa of 1.0:
-// x = 1 + code / 2^k exactly (k = 4 for a 4-bit nibble; for 3-bit codes the
-// 2-bit low plane gives 1 + lo/4 and the high bit 1 + hi/2).  With
-// gs = sum_c G_c over the group:
-//   4-bit:  sum_c code_c G_c = 16 (sum_c x_c G_c - gs)
-//   3-bit:  sum_c code_c G_c = 4 sum_c xlo_c G_c + 8 sum_c xhi_c G_c - 12 gs
+// x = 1 + code / 16 exactly, for a 4-bit code and for a 3-bit code whose two
+// planes were first rebuilt into a nibble.  With gs = sum_c G_c over the group,
+//   sum_c code_c G_c = 16 (sum_c x_c G_c - gs)
 // and the group's contribution is s * sum code G + zp * gs.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float mant(uint32_t bits) { return __uint_as_float(0x3F800000u | bits); }
 
-// field of `width` bits at bit `pos` of w, moved to mantissa bits [23 - width, 23)
-template <int POS, int WIDTH>
-__device__ __forceinline__ float field_as_unit(uint32_t w) {
-  constexpr int dst = 23 - WIDTH;
-  constexpr uint32_t mask = ((1u << WIDTH) - 1u) << dst;
-  if constexpr (POS <= dst) return mant((w << (dst - POS)) & mask);
-  else return mant((w >> (POS - dst)) & mask);
+// 3-bit codes of one token as 4-bit nibbles: the 2-bit plane's fields (bits
+// 2c..2c+1) and the 1-bit plane's bits (bit c) spread to nibble c (bits 4c..4c+3).
+__device__ __forceinline__ uint32_t spread2_to_nibbles8(uint32_t x) {  // 8 fields of 2 bits
+  x = (x | (x << 8)) & 0x00FF00FFu;
+  x = (x | (x << 4)) & 0x0F0F0F0Fu;
+  return (x | (x << 2)) & 0x33333333u;
 }
-
-// Packed fp32 pairs (sm_100a f32x2 arithmetic: two lanes of fp32 per instruction).
-typedef unsigned long long f32x2_t;
-__device__ __forceinline__ f32x2_t pk2(float x, float y) {
-  f32x2_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
-  return r;
-}
-__device__ __forceinline__ float2 upk2(f32x2_t r) {
-  float2 v;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
-  return v;
-}
-__device__ __forceinline__ f32x2_t ffma2(f32x2_t a, f32x2_t b, f32x2_t c) {
-  f32x2_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ f32x2_t fadd2(f32x2_t a, f32x2_t b) {
-  f32x2_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ float hsum2(f32x2_t r) {
-  const float2 v = upk2(r);
-  return v.x + v.y;
+__device__ __forceinline__ uint32_t spread1_to_nibbles8(uint32_t y) {  // 8 single bits
+  y = (y | (y << 12)) & 0x000F000Fu;
+  y = (y | (y << 6)) & 0x03030303u;
+  return (y | (y << 3)) & 0x11111111u;
 }
 
 template <int G>
 struct KeyGroup {
-  // 4-bit tile: token t16's G nibbles; 3-bit tile: its 2-bit and 1-bit planes
-  __device__ __forceinline__ static float dot4(const uint8_t* tile, int t16, const float* Gv, float& gs) {
-    f32x2_t a2 = 0ull, g2 = 0ull;
-    if constexpr (G == 4) {
-      const uint32_t w = *reinterpret_cast<const uint16_t*>(tile + 2 * t16);
+  // sum_c x_c G_c and sum_c G_c over up to 8 channels whose codes are the
+  // nibbles of w (x_c = 1 + code_c / 16); two accumulators each
+  template <int N>
+  __device__ __forceinline__ static void nib_dot(uint32_t w, const float* Gv, float (&acc)[2], float (&gs)[2]) {
 #pragma unroll
-      for (int c = 0; c < 4; c += 2) {
-        const f32x2_t gp = pk2(Gv[c], Gv[c + 1]);
-        a2 = ffma2(pk2(field_as_unit<0, 4>(w >> (4 * c)), field_as_unit<0, 4>(w >> (4 * c + 4))), gp, a2);
-        g2 = fadd2(g2, gp);
-      }
+    for (int c = 0; c < N; ++c) {
+      const float x = mant(((c >= 5 ? (w >> (4 * c - 19)) : (w << (19 - 4 * c)))) & 0x00780000u);
+      acc[c & 1] = fmaf(x, Gv[c], acc[c & 1]);
+      gs[c & 1] += Gv[c];
+    }
+  }
+  // sum_c code_c G_c of a 4-bit group (16 (sum x G - sum G)), sum_c G_c in gsum
+  __device__ __forceinline__ static float dot4(const uint8_t* tile, int t16, const float* Gv, float& gsum) {
+    float acc[2] = {0.f, 0.f}, gs[2] = {0.f, 0.f};
+    if constexpr (G == 4) {
+      nib_dot<4>(*reinterpret_cast<const uint16_t*>(tile + 2 * t16), Gv, acc, gs);
     } else {
       const uint32_t* wp = reinterpret_cast<const uint32_t*>(tile + (G / 2) * t16);
 #pragma unroll
-      for (int q = 0; q < G / 8; ++q) {
-        const uint32_t w = wp[q];
-        const float* g8 = Gv + 8 * q;
-        f32x2_t gp = pk2(g8[0], g8[1]);
-        a2 = ffma2(pk2(field_as_unit<0, 4>(w), field_as_unit<4, 4>(w)), gp, a2);
-        g2 = fadd2(g2, gp);
-        gp = pk2(g8[2], g8[3]);
-        a2 = ffma2(pk2(field_as_unit<8, 4>(w), field_as_unit<12, 4>(w)), gp, a2);
-        g2 = fadd2(g2, gp);
-        gp = pk2(g8[4], g8[5]);
-        a2 = ffma2(pk2(field_as_unit<16, 4>(w), field_as_unit<20, 4>(w)), gp, a2);
-        g2 = fadd2(g2, gp);
-        gp = pk2(g8[6], g8[7]);
-        a2 = ffma2(pk2(field_as_unit<24, 4>(w), field_as_unit<28, 4>(w)), gp, a2);
-        g2 = fadd2(g2, gp);
-      }
+      for (int q = 0; q < G / 8; ++q) nib_dot<8>(wp[q], Gv + 8 * q, acc, gs);
     }
-    gs = hsum2(g2);
-    return 16.f * (hsum2(a2) - gs);
+    gsum = gs[0] + gs[1];
+    return 16.f * (acc[0] + acc[1] - gsum);
   }
-  __device__ __forceinline__ static float dot3(const uint8_t* tile, int t16, const float* Gv, float& gs) {
-    uint32_t lo, hi;
+  // the same for a 3-bit group: planes rebuilt into nibbles first
+  __device__ __forceinline__ static float dot3(const uint8_t* tile, int t16, const float* Gv, float& gsum) {
+    float acc[2] = {0.f, 0.f}, gs[2] = {0.f, 0.f};
     if constexpr (G == 4) {
-      lo = tile[t16];
-      hi = (uint32_t)(tile[16 + (t16 >> 1)] >> ((t16 & 1) * 4));
+      const uint32_t lo = tile[t16];
+      const uint32_t hi = (uint32_t)(tile[16 + (t16 >> 1)] >> ((t16 & 1) * 4)) & 0xFu;
+      nib_dot<4>(spread2_to_nibbles8(lo) | (spread1_to_nibbles8(hi) << 2), Gv, acc, gs);
     } else if constexpr (G == 8) {
-      lo = *reinterpret_cast<const uint16_t*>(tile + 2 * t16);
-      hi = tile[32 + t16];
+      const uint32_t lo = *reinterpret_cast<const uint16_t*>(tile + 2 * t16);
+      const uint32_t hi = tile[32 + t16];
+      nib_dot<8>(spread2_to_nibbles8(lo) | (spread1_to_nibbles8(hi) << 2), Gv, acc, gs);
     } else {
-      lo = *reinterpret_cast<const uint32_t*>(tile + 4 * t16);
-      hi = *reinterpret_cast<const uint16_t*>(tile + 64 + 2 * t16);
+      const uint32_t lo = *reinterpret_cast<const uint32_t*>(tile + 4 * t16);
+      const uint32_t hi = *reinterpret_cast<const uint16_t*>(tile + 64 + 2 * t16);
+      nib_dot<8>(spread2_to_nibbles8(lo & 0xFFFFu) | (spread1_to_nibbles8(hi & 0xFFu) << 2), Gv, acc, gs);
+      nib_dot<8>(spread2_to_nibbles8(lo >> 16) | (spread1_to_nibbles8(hi >> 8) << 2), Gv + 8, acc, gs);
     }
-    f32x2_t al = 0ull, ah = 0ull, g2 = 0ull;
-#pragma unroll
-    for (int c = 0; c < G; c += 2) {
-      const f32x2_t gp = pk2(Gv[c], Gv[c + 1]);
-      al = ffma2(pk2(field_as_unit<0, 2>(lo >> (2 * c)), field_as_unit<0, 2>(lo >> (2 * c + 2))), gp, al);
-      ah = ffma2(pk2(field_as_unit<0, 1>(hi >> c), field_as_unit<0, 1>(hi >> (c + 1))), gp, ah);
-      g2 = fadd2(g2, gp);
-    }
-    gs = hsum2(g2);
-    return 4.f * hsum2(al) + 8.f * hsum2(ah) - 12.f * gs;
+    gsum = gs[0] + gs[1];
+    return 16.f * (acc[0] + acc[1] - gsum);
   }
 };
 
 // sum_c z_hat_c G_c over one token's key latent in a staged page region.
+template <int RK, int G>
+__device__ __forceinline__ float key_dot(const uint8_t* region, const uint32_t* meta, int top_groups, int t16,
+                                         const uint32_t (&raw)[RK]);
+
+// Two heads' scores at once: the groups of both are independent, so their
+// dependency chains interleave.
+template <int RK, int G>
+__device__ __forceinline__ void key_dot2(const uint8_t* regA, const uint32_t* metaA, const uint8_t* regB,
+                                         const uint32_t* metaB, int top_groups, int t16, const uint32_t (&rA)[RK],
+                                         const uint32_t (&rB)[RK], float& sA, float& sB) {
+  const float* GA = reinterpret_cast<const float*>(rA);
+  const float* GB = reinterpret_cast<const float*>(rB);
+  float accA = 0.f, accB = 0.f;
+#pragma unroll
+  for (int gi = 0; gi < RK / G; ++gi) {
+    const uint32_t mA = metaA[gi * kPage + t16], mB = metaB[gi * kPage + t16];
+    float gsA, gsB, cA, cB;
+    if (gi < top_groups) {
+      cA = KeyGroup<G>::dot4(regA + gi * 8 * G, t16, GA + gi * G, gsA);
+      cB = KeyGroup<G>::dot4(regB + gi * 8 * G, t16, GB + gi * G, gsB);
+    } else {
+      const int o = top_groups * 8 * G + (gi - top_groups) * 6 * G;
+      cA = KeyGroup<G>::dot3(regA + o, t16, GA + gi * G, gsA);
+      cB = KeyGroup<G>::dot3(regB + o, t16, GB + gi * G, gsB);
+    }
+    const float sa = __half2float(__ushort_as_half((unsigned short)(mA & 0xFFFF)));
+    const float za = __half2float(__ushort_as_half((unsigned short)(mA >> 16)));
+    const float sb = __half2float(__ushort_as_half((unsigned short)(mB & 0xFFFF)));
+    const float zb = __half2float(__ushort_as_half((unsigned short)(mB >> 16)));
+    accA = fmaf(sa, cA, fmaf(za, gsA, accA));
+    accB = fmaf(sb, cB, fmaf(zb, gsB, accB));
+  }
+  sA = accA;
+  sB = accB;
+}
+
 template <int RK, int G>
 __device__ __forceinline__ float key_dot(const uint8_t* region, const uint32_t* meta, int top_groups, int t16,
                                          const uint32_t (&raw)[RK]) {
@@ -362,15 +362,19 @@ __global__ void __launch_bounds__(kAThreads, 1)
   uint8_t* sm = align1024(smem_raw);
   uint8_t* Wsm = sm;                                         // [ncols x d] K-major, 128B swizzle
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + a.off_bar);
-  uint64_t* full = bar;        // [2] stage loaded (TMA + bulk)
-  uint64_t* empty = bar + 2;   // [2] stage free (MMA commit + epilogue warps)
-  uint64_t* tfull = bar + 4;   // [2] accumulator ready
-  uint64_t* tempty = bar + 6;  // [2] accumulator drained
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 8);
-  int* failed = reinterpret_cast<int*>(bar + 9);
-  int* flags = reinterpret_cast<int*>(sm + a.off_flags);    // [2][8] page ids (-1 = invalid)
+  // Two rings: position tiles (needed by the MMA only, freed by its commit) and
+  // key codes + metadata (read by the epilogue, freed by it), NK stages deep.
+  uint64_t* trfull = bar;                       // [2] position tile loaded
+  uint64_t* trempty = bar + 2;                  // [2] position tile read by the MMA
+  uint64_t* tfull = bar + 4;                    // [2] accumulator ready
+  uint64_t* tempty = bar + 6;                   // [2] accumulator drained
+  uint64_t* kfull = bar + 8;                    // [NK] key stage loaded
+  uint64_t* kempty = kfull + kMaxKeyStages;     // [NK] key stage read by the epilogue
+  uint64_t* wbar = kempty + kMaxKeyStages;      // W image loaded
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(wbar + 1);
+  int* failed = reinterpret_cast<int*>(wbar + 2);
+  int* flags = reinterpret_cast<int*>(sm + a.off_flags);    // [NK][8] page ids (-1 = invalid)
   int* bt_s = reinterpret_cast<int*>(sm + a.off_bt);        // this job's block-table entries
-  uint64_t* wbar = bar + 10;                                 // W image loaded
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int d = a.d;
 
@@ -382,10 +386,14 @@ __global__ void __launch_bounds__(kAThreads, 1)
   if (warp == 1) tmem_alloc(tslot, kScoreTmemCols);
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + kEpiWarps);
+      mbar_init(&trfull[s], 1);
+      mbar_init(&trempty[s], 1);
       mbar_init(&tfull[s], 1);
       mbar_init(&tempty[s], kEpiWarps);
+    }
+    for (int s = 0; s < a.NK; ++s) {
+      mbar_init(&kfull[s], 1);
+      mbar_init(&kempty[s], kEpiWarps);
     }
     mbar_init(wbar, 1);
     *failed = 0;
@@ -442,18 +450,32 @@ __global__ void __launch_bounds__(kAThreads, 1)
       // ---------------- producer: one lane per copy (issued in parallel) ----------------
       const int nsub = d / 64;
       for (int k = 0; k < ntile; ++k) {
-        const uint32_t c = it + k, s = c & 1, ph = (c >> 1) & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1))) {
+        const uint32_t c = it + k, ts = c & 1, tph = (c >> 1) & 1;
+        const uint32_t ks = c % a.NK, kph = (c / a.NK) & 1;
+        const int j0 = (t0 + k) * kT;
+        // position rows of the tile
+        if (!__all_sync(0xffffffffu, mbar_wait(&trempty[ts], tph ^ 1))) {
           if (lane == 0) {
             set_status(a.status, kDevWaitTimeout);
             *failed = 1;
           }
           break;
         }
-        const int j0 = (t0 + k) * kT;
+        if (lane == 0) mbar_arrive_expect_tx(&trfull[ts], a.trig_stage);
+        __syncwarp();
+        uint8_t* trig_dst = sm + a.off_trig + ts * a.trig_stage;
+        if (lane < nsub) tma_load_2d(trig_dst + lane * 16384, &trig_map, lane * 64, j0, &trfull[ts]);
+        // key codes and metadata of its pages
+        if (!__all_sync(0xffffffffu, mbar_wait(&kempty[ks], kph ^ 1))) {
+          if (lane == 0) {
+            set_status(a.status, kDevWaitTimeout);
+            *failed = 1;
+          }
+          break;
+        }
         const int nval = min(kT, L - j0);
         const int np = (nval + kPage - 1) / kPage;
-        int* fl = flags + s * kPagesPerTile;
+        int* fl = flags + ks * kPagesPerTile;
         if (lane < kPagesPerTile) {
           int pid = -1;
           if (lane < np) {
@@ -468,23 +490,18 @@ __global__ void __launch_bounds__(kAThreads, 1)
         __syncwarp();
         const int nvalid =
             __popc(__ballot_sync(0xffffffffu, lane < kPagesPerTile && fl[lane < kPagesPerTile ? lane : 0] >= 0));
-        if (lane == 0) mbar_arrive_expect_tx(&full[s], a.trig_stage + (uint32_t)nvalid * (a.codes_page + a.meta_page));
+        if (lane == 0) mbar_arrive_expect_tx(&kfull[ks], (uint32_t)nvalid * (a.codes_page + a.meta_page));
         __syncwarp();
-        uint8_t* trig_dst = sm + a.off_trig + s * a.trig_stage;
-        for (int i = lane; i < nsub + 2 * kPagesPerTile; i += 32) {
-          if (i < nsub) {
-            tma_load_2d(trig_dst + i * 16384, &trig_map, i * 64, j0, &full[s]);
-          } else {
-            const int p = (i - nsub) >> 1;
-            const int pid = fl[p];
-            if (pid >= 0) {
-              if (((i - nsub) & 1) == 0)
-                bulk_g2s(sm + a.off_codes + s * a.codes_stage + p * a.codes_pitch,
-                         a.k_codes + ((int64_t)pid * a.h_kv + kv0) * a.key.region_bytes, a.codes_page, &full[s]);
-              else
-                bulk_g2s(sm + a.off_meta + s * a.meta_stage + p * a.meta_pitch,
-                         a.k_meta + ((int64_t)pid * a.h_kv + kv0) * a.key.groups * kPage, a.meta_page, &full[s]);
-            }
+        if (lane < 2 * kPagesPerTile) {
+          const int p = lane >> 1;
+          const int pid = fl[p];
+          if (pid >= 0) {
+            if ((lane & 1) == 0)
+              bulk_g2s(sm + a.off_codes + ks * a.codes_stage + p * a.codes_pitch,
+                       a.k_codes + ((int64_t)pid * a.h_kv + kv0) * a.key.region_bytes, a.codes_page, &kfull[ks]);
+            else
+              bulk_g2s(sm + a.off_meta + ks * a.meta_stage + p * a.meta_pitch,
+                       a.k_meta + ((int64_t)pid * a.h_kv + kv0) * a.key.groups * kPage, a.meta_page, &kfull[ks]);
           }
         }
       }
@@ -492,8 +509,8 @@ __global__ void __launch_bounds__(kAThreads, 1)
       if (lane == 0) {
         // ---------------- MMA issuer ----------------
         for (int k = 0; k < ntile; ++k) {
-          const uint32_t c = it + k, s = c & 1, ph = (c >> 1) & 1;
-          if (!mbar_wait(&full[s], ph) || !mbar_wait(&tempty[s], ph ^ 1)) {
+          const uint32_t c = it + k, s = c & 1, ph = (c >> 1) & 1;  // position stage = accumulator = c & 1
+          if (!mbar_wait(&trfull[s], ph) || !mbar_wait(&tempty[s], ph ^ 1)) {
             set_status(a.status, kDevWaitTimeout);
             *failed = 1;
             break;
@@ -509,7 +526,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
             mma_f16(dt, ad, bd, idesc, ks > 0);
           }
           mma_commit(&tfull[s]);
-          mma_commit(&empty[s]);
+          mma_commit(&trempty[s]);
         }
       }
     } else {
@@ -517,10 +534,12 @@ __global__ void __launch_bounds__(kAThreads, 1)
       const int q4 = warp & 3, hq = (warp - 2) >> 2;   // TMEM lane quarter, head quarter
       const int t = q4 * 32 + lane;
       const int t16 = t % kPage, p = t / kPage;
-      const int hper = a.hpc / 4;
+      const int hper = a.hpc / 4;  // heads per thread (<= 4)
+      float mloc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // running maxima of this thread's heads
       for (int k = 0; k < ntile; ++k) {
         const uint32_t c = it + k, s = c & 1, ph = (c >> 1) & 1;
-        if (!mbar_wait(&tfull[s], ph) || !mbar_wait(&full[s], ph)) {
+        const uint32_t ks = c % a.NK, kph = (c / a.NK) & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&tfull[s], ph) && mbar_wait(&kfull[ks], kph))) {
           if (lane == 0) {
             set_status(a.status, kDevWaitTimeout);
             *failed = 1;
@@ -530,52 +549,70 @@ __global__ void __launch_bounds__(kAThreads, 1)
         tc_fence_after();
         const int tile = t0 + k;
         const int j = tile * kT + t;
-        const int pid = flags[s * kPagesPerTile + p];
+        const int pid = flags[ks * kPagesPerTile + p];
         const bool valid = j < L && pid >= 0;
-        const uint8_t* cstage = sm + a.off_codes + s * a.codes_stage + p * a.codes_pitch;
-        const uint32_t* mstage = reinterpret_cast<const uint32_t*>(sm + a.off_meta + s * a.meta_stage + p * a.meta_pitch);
+        const uint8_t* cstage = sm + a.off_codes + ks * a.codes_stage + p * a.codes_pitch;
+        const uint32_t* mstage =
+            reinterpret_cast<const uint32_t*>(sm + a.off_meta + ks * a.meta_stage + p * a.meta_pitch);
         const uint32_t trow = tmem + s * 256 + ((uint32_t)(q4 * 32) << 16);
-        auto head = [&](int hl, const uint32_t(&raw)[RK]) {
-          const int h = h0 + hl;
-          const int kvl = h / a.group - kv0;
-          float score = -INFINITY;
-          if (valid)
-            score = key_dot<RK, G>(cstage + kvl * a.key.region_bytes, mstage + kvl * a.key.groups * kPage,
-                                   a.key.top_groups, t16, raw);
+        auto finish = [&](int i, float score) {  // i: this thread's head index (static)
+          const int h = h0 + hq * hper + i;
           if (j < L) a.S[((int64_t)b * a.H + h) * a.tpad + j] = score;
-          const float m = warp_max(score);
-          if (lane == 0 && m != -INFINITY) atomicMax(&a.Mx[b * a.H + h], ordered_bits(m));
+          mloc[i] = fmaxf(mloc[i], score);
         };
         const int hl0 = hq * hper;
         if constexpr (RK >= 64) {
           // one 64-column row per head (a 256-column accumulator holds 4 heads: one per warp)
-          for (int hh = 0; hh < hper; ++hh) {
+#pragma unroll
+          for (int hh = 0; hh < 4; ++hh) {
+            if (hh >= hper) break;
             uint32_t rA[RK];
             tmem_issue_row<RK>(trow + (hl0 + hh) * RK, rA);
             tmem_wait_row<RK>(rA);
-            head(hl0 + hh, rA);
+            float sc = -INFINITY;
+            if (valid) {
+              const int kA = (h0 + hl0 + hh) / a.group - kv0;
+              sc = key_dot<RK, G>(cstage + kA * a.key.region_bytes, mstage + kA * a.key.groups * kPage,
+                                  a.key.top_groups, t16, rA);
+            }
+            finish(hh, sc);
           }
         } else {
-          // ping-pong: the next head's accumulator row lands while this one computes
-          uint32_t rA[RK], rB[RK];
-          tmem_issue_row<RK>(trow + hl0 * RK, rA);
-          for (int hh = 0; hh < hper; hh += 2) {
+#pragma unroll
+          for (int hh = 0; hh < 4; hh += 2) {
+            if (hh >= hper) break;
+            const int hA = hl0 + hh;
+            const bool two = hh + 1 < hper;
+            const int hB = two ? hA + 1 : hA;
+            uint32_t rA[RK], rB[RK];
+            tmem_issue_row<RK>(trow + hA * RK, rA);
+            tmem_issue_row<RK>(trow + hB * RK, rB);
             tmem_wait_row<RK>(rA);
-            if (hh + 1 < hper) tmem_issue_row<RK>(trow + (hl0 + hh + 1) * RK, rB);
-            head(hl0 + hh, rA);
-            if (hh + 1 < hper) {
-              tmem_wait_row<RK>(rB);
-              if (hh + 2 < hper) tmem_issue_row<RK>(trow + (hl0 + hh + 2) * RK, rA);
-              head(hl0 + hh + 1, rB);
+            tmem_wait_row<RK>(rB);
+            float sA = -INFINITY, sB = -INFINITY;
+            if (valid) {
+              const int kA = (h0 + hA) / a.group - kv0, kB = (h0 + hB) / a.group - kv0;
+              key_dot2<RK, G>(cstage + kA * a.key.region_bytes, mstage + kA * a.key.groups * kPage,
+                              cstage + kB * a.key.region_bytes, mstage + kB * a.key.groups * kPage, a.key.top_groups,
+                              t16, rA, rB, sA, sB);
             }
+            finish(hh, sA);
+            if (two) finish(hh + 1, sB);
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&tempty[s]);
-          mbar_arrive(&empty[s]);
+          mbar_arrive(&kempty[ks]);
         }
+      }
+      // this job's running maxima: one warp reduction and one atomic per head
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (i >= hper) break;
+        const float m = warp_max(mloc[i]);
+        if (lane == 0 && m != -INFINITY) atomicMax(&a.Mx[b * a.H + h0 + hq * hper + i], ordered_bits(m));
       }
     }
     it += ntile;
@@ -1522,16 +1559,24 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
     o = (o + 1023) / 1024 * 1024;
     A.off_trig = o;
     o += 2 * A.trig_stage;
+    // as many key stages as fit (page table, flags, barriers and alignment slack after them)
+    const uint32_t tail = (uint32_t)(A.items_per_cta * kPagesPerTile * 4) + kMaxKeyStages * kPagesPerTile * 4 +
+                          (2 * kMaxKeyStages + 16) * 8 + 1024 + 64;
+    const uint32_t per_key = A.codes_stage + A.meta_stage;
+    int nk = (int)((227u * 1024u - o - tail) / per_key);
+    if (nk > kMaxKeyStages) nk = kMaxKeyStages;
+    if (nk < 2) return cudaErrorInvalidConfiguration;
+    A.NK = nk;
     A.off_codes = o;
-    o += 2 * A.codes_stage;
+    o += nk * A.codes_stage;
     A.off_meta = o;
-    o += 2 * A.meta_stage;
+    o += nk * A.meta_stage;
     A.off_flags = o;
-    o += 2 * kPagesPerTile * 4;
+    o += kMaxKeyStages * kPagesPerTile * 4;
     A.off_bt = (o + 15) / 16 * 16;
     o = A.off_bt + A.items_per_cta * kPagesPerTile * 4;
     A.off_bar = (o + 15) / 16 * 16;
-    o = A.off_bar + 16 * 8;
+    o = A.off_bar + (2 * kMaxKeyStages + 16) * 8;
     const size_t smem = o + 1024;  // alignment slack
     cudaError_t e;
     switch (f.rank_k) {

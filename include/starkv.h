@@ -272,6 +272,14 @@ STARKV_API starkv_status starkv_dequantize(starkv_ctx* ctx, int32_t which, const
 STARKV_API starkv_status starkv_read_device_status(starkv_ctx* ctx, starkv_stream_t stream,
                                         uint32_t* status);
 
+/* Test-only failure detection check (no counterpart on the pages): queue one
+ * block that waits on a shared-memory barrier nothing ever completes, with the
+ * bounded wait every pipelined kernel of this library uses, given `limit_ns`
+ * nanoseconds (1e3 .. 1e9) instead of the kernels' own limit.  The wait gives up,
+ * sets STARKV_DEV_WAIT_TIMEOUT in the status word and the block exits; the
+ * context stays usable.  Errors: INVALID_ARG (limit out of range), CUDA. */
+STARKV_API starkv_status starkv_selftest_wait_timeout(starkv_ctx* ctx, uint64_t limit_ns, starkv_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -422,6 +422,15 @@ starkv_status starkv_dequantize(starkv_ctx* ctx, int32_t which, const void* code
   return ok();
 }
 
+starkv_status starkv_selftest_wait_timeout(starkv_ctx* ctx, uint64_t limit_ns, starkv_stream_t stream) {
+  if (!ctx) return fail(STARKV_ERR_INVALID_ARG, "NULL context");
+  if (limit_ns < 1000ull || limit_ns > 1000000000ull) return fail(STARKV_ERR_INVALID_ARG, "limit_ns out of range");
+  Ctx* c = reinterpret_cast<Ctx*>(ctx);
+  cudaError_t e = starkv::launch_wait_timeout_selftest(c->status, limit_ns, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  return ok();
+}
+
 starkv_status starkv_read_device_status(starkv_ctx* ctx, starkv_stream_t stream, uint32_t* status) {
   if (!ctx || !status) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
   Ctx* c = reinterpret_cast<Ctx*>(ctx);

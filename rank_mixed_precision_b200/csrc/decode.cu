@@ -19,6 +19,7 @@
 #include <mutex>
 
 #include "internal.cuh"
+#include "sm100.cuh"
 
 namespace starkv {
 
@@ -396,6 +397,23 @@ cudaError_t noalloc_scratch(void** out) {
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
+}
+
+// Failure-detection check: the same bounded mbarrier wait the pipelined
+// kernels use, on a barrier whose single expected arrival never comes.
+__global__ void wait_timeout_selftest_kernel(unsigned int* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  if (!__all_sync(0xffffffffu, sm100::mbar_wait(&bar, 0, limit_ns)) && threadIdx.x == 0) set_status(status, kDevWaitTimeout);
+}
+
+cudaError_t launch_wait_timeout_selftest(unsigned int* status, uint64_t limit_ns, cudaStream_t s) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+  return cudaGetLastError();
 }
 
 }  // namespace starkv

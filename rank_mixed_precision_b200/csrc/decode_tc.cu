@@ -709,7 +709,9 @@ __device__ __forceinline__ int value_channel_of_position(int p, bool top) {
 }
 
 constexpr int kVMaxWarps = 16;                      // dequant warps at most
-constexpr int kVThreads = (2 + kVMaxWarps) * 32;
+constexpr int kVPWarps = 2;                         // P warps (each half of a stage's tokens)
+constexpr int kVRoleWarps = 1 + kVPWarps;           // producer + P warps
+constexpr int kVThreads = (kVRoleWarps + kVMaxWarps) * 32;
 constexpr int kVMaxStages = 8;
 constexpr uint32_t kZTile = kPage * 128 * 2;        // one page x one 128-channel M tile, fp16
 
@@ -725,9 +727,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
 //                    of 32 tokens x H heads, 128-byte swizzle) and the value
 //                    codes + metadata of its PS pages (bulk copies, one lane per
 //                    copy), NS stages deep
-//   warp 1           P: lane = head; P[h, t] = exp2(s - M_h) as fp16 into a
-//                    K-major tile, l_h summed in registers
-//   warps 2..nW+1    dequant warp w = (M tile w % MT, page w / MT of the stage):
+//   warps 1..2       P: lane = head, each warp half of the stage's tokens;
+//                    P[h, t] = exp2(s - M_h) as fp16 into a K-major tile, l_h
+//                    summed in registers
+//   warps 3..nW+2    dequant warp w = (M tile w % MT, page w / MT of the stage):
 //                    dequantises its 16 tokens x 128 channels into its own Z tile
 //                    and issues its own MMA  D_w[ch, h] += sum_t Z[t, ch] P[h, t]
 //                    into its own TMEM columns (no cross-warp hand-off per tile)
@@ -740,7 +743,7 @@ __global__ void __launch_bounds__(kVThreads, 1)
   uint8_t* sm = align1024(smem_raw);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + a.off_bar);
   uint64_t* cfull = bar;                     // [NS] stage landed
-  uint64_t* cempty = cfull + kVMaxStages;    // [NS] stage read (P warp + dequant warps)
+  uint64_t* cempty = cfull + kVMaxStages;    // [NS] stage read (P warps + dequant warps)
   uint64_t* pfull = cempty + kVMaxStages;    // [NS] P tile written
   uint64_t* pempty = pfull + kVMaxStages;    // [NS] MMAs reading the P tile done
   uint64_t* zempty = pempty + kVMaxStages;   // [nW] MMA reading warp w's Z tile done
@@ -775,8 +778,8 @@ __global__ void __launch_bounds__(kVThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&cfull[s], 1);
-      mbar_init(&cempty[s], a.nW + 1);
-      mbar_init(&pfull[s], 1);
+      mbar_init(&cempty[s], a.nW + kVPWarps);
+      mbar_init(&pfull[s], kVPWarps);
       mbar_init(&pempty[s], a.nW);
     }
     for (int w = 0; w < a.nW; ++w) mbar_init(&zempty[w], 1);
@@ -854,8 +857,10 @@ __global__ void __launch_bounds__(kVThreads, 1)
           }
         }
       }
-    } else if (warp == 1) {
-      // ---------------- P: lane = head (and head + 32)
+    } else if (warp < kVRoleWarps) {
+      // ---------------- P: lane = head (and head + 32), this warp's half of the tokens
+      const int pw = warp - 1;
+      const int tspan = ST / kVPWarps;  // a multiple of 8
       float2 lacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       float mh[2];
 #pragma unroll
@@ -878,31 +883,28 @@ __global__ void __launch_bounds__(kVThreads, 1)
         for (int i = 0; i < 2; ++i) {
           const int h = lane + 32 * i;
           if (h < a.H) {
-            for (int bx = 0; bx < ST / 32; ++bx) {
-              const uint8_t* row = sst + bx * a.s_box + h * 128;  // 32 fp32 scores, 16-byte chunks swizzled by h % 8
+            for (int t0 = pw * tspan; t0 < (pw + 1) * tspan; t0 += 8) {
+              // 8 tokens t0..t0+7 (one page): two 16-byte chunks of the swizzled 32-token score row
+              const uint8_t* row = sst + (t0 >> 5) * a.s_box + h * 128;
+              const int c = (t0 & 31) >> 2;
+              const float4 v0 = *reinterpret_cast<const float4*>(row + ((c ^ (h & 7)) << 4));
+              const float4 v1 = *reinterpret_cast<const float4*>(row + (((c + 1) ^ (h & 7)) << 4));
+              float pv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-              for (int c = 0; c < 8; c += 2) {
-                const float4 v0 = *reinterpret_cast<const float4*>(row + ((c ^ (h & 7)) << 4));
-                const float4 v1 = *reinterpret_cast<const float4*>(row + (((c + 1) ^ (h & 7)) << 4));
-                const int t0 = bx * 32 + 4 * c;  // first of 8 tokens, all in one page
-                float pv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+              for (int u = 0; u < 8; ++u) pv[u] = ex2_approx(pv[u] - mh[i]);
+              if (!full) {
+                const int lim = fl[t0 >> 4] >= 0 ? L - (j0 + t0) : 0;  // tokens t0 + u valid for u < lim
 #pragma unroll
-                for (int u = 0; u < 8; ++u) pv[u] = ex2_approx(pv[u] - mh[i]);
-                if (!full) {
-                  const int lim = fl[t0 >> 4] >= 0 ? L - (j0 + t0) : 0;  // tokens t0 + u valid for u < lim
-#pragma unroll
-                  for (int u = 0; u < 8; ++u) pv[u] = u < lim ? pv[u] : 0.f;
-                }
-                uint32_t w4[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  w4[u] = h2bits(__floats2half2_rn(pv[2 * u], pv[2 * u + 1]));
-                  lacc[i].x += pv[2 * u];
-                  lacc[i].y += pv[2 * u + 1];
-                }
-                *reinterpret_cast<uint4*>(pt + sw128_kmajor_offset(h, t0, a.N)) =
-                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                for (int u = 0; u < 8; ++u) pv[u] = u < lim ? pv[u] : 0.f;
               }
+              uint32_t w4[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                w4[u] = h2bits(__floats2half2_rn(pv[2 * u], pv[2 * u + 1]));
+                lacc[i].x += pv[2 * u];
+                lacc[i].y += pv[2 * u + 1];
+              }
+              *reinterpret_cast<uint4*>(pt + sw128_kmajor_offset(h, t0, a.N)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
           }
         }
@@ -915,10 +917,10 @@ __global__ void __launch_bounds__(kVThreads, 1)
       }
 #pragma unroll
       for (int i = 0; i < 2; ++i)
-        if (lane + 32 * i < a.H) Lh[lane + 32 * i] = lacc[i].x + lacc[i].y;
-    } else if (warp - 2 < a.nW) {
+        if (lane + 32 * i < a.H) atomicAdd(&Lh[lane + 32 * i], lacc[i].x + lacc[i].y);
+    } else if (warp - kVRoleWarps < a.nW) {
       // ---------------- dequant + MMA: 16 tokens x 128 channels per stage
-      const int w = warp - 2;
+      const int w = warp - kVRoleWarps;
       const int mt = w % a.MT, pg = w / a.MT;
       const int t16 = lane & 15, gsel = lane >> 4;
       uint8_t* zt = sm + a.off_z + w * kZTile;
@@ -1387,7 +1389,7 @@ TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
     const double tok_bytes = (double)c.val.region_bytes / kPage + c.val.groups * 4.0 + f.num_q_heads * 4.0;
     const double work = (double)bt * t.tpad * tok_bytes;
     const double part_unit = 2.0 * f.num_q_heads * f.rank_v * 4.0;
-    const int threads = (2 + t.nW) * 32;
+    const int threads = (kVRoleWarps + t.nW) * 32;
     VSmem probe;
     t.ok = value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, 1, probe);  // largest page table
     double best = -1.0;
@@ -1550,8 +1552,8 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   A.trig_stage = kT * d * 2;
   A.codes_page = t.kvpc * c.key.region_bytes;
   A.meta_page = t.kvpc * c.key.groups * kPage * 4;
-  A.codes_pitch = A.codes_page + 64;
-  A.meta_pitch = A.meta_page + 64;
+  A.codes_pitch = (A.codes_page + 64 + 127) / 128 * 128 - 64;  // = 64 mod 128: the two pages a warp reads
+  A.meta_pitch = (A.meta_page + 64 + 127) / 128 * 128 - 64;    // fall on different banks
   A.codes_stage = kPagesPerTile * A.codes_pitch;
   A.meta_stage = kPagesPerTile * A.meta_pitch;
   {
@@ -1647,7 +1649,7 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(t.splits, batch);
-    cfg.blockDim = dim3((2 + t.nW) * 32);
+    cfg.blockDim = dim3((kVRoleWarps + t.nW) * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

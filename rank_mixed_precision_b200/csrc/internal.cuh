@@ -60,6 +60,9 @@ constexpr int kSmallAppend = 64;
 // Extra device status bit: a pipeline wait in a tensor-core kernel gave up.
 constexpr unsigned int kDevWaitTimeout = STARKV_DEV_WAIT_TIMEOUT;
 
+// One block waiting on a barrier that nothing completes (bounded; sets kDevWaitTimeout).
+cudaError_t launch_wait_timeout_selftest(unsigned int* status, uint64_t limit_ns, cudaStream_t s);
+
 // ---------------------------------------------------------------------------
 // Device helpers
 // ---------------------------------------------------------------------------

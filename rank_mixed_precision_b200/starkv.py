@@ -27,6 +27,7 @@ EXPORTS = [
     "starkv_get_config", "starkv_append", "starkv_workspace_bytes", "starkv_decode_attn",
     "starkv_decode_attn_noalloc",
     "starkv_prefill_attn", "starkv_quantize_pack", "starkv_dequantize", "starkv_read_device_status",
+    "starkv_selftest_wait_timeout",
 ]
 
 
@@ -77,6 +78,7 @@ _SIGS = {
     "starkv_quantize_pack": ([_vp, _i32, _vp, _i64, _vp, _vp, _vp], _i32),
     "starkv_dequantize": ([_vp, _i32, _vp, _vp, _i64, _vp, _vp], _i32),
     "starkv_read_device_status": ([_vp, _vp, ctypes.POINTER(ctypes.c_uint32)], _i32),
+    "starkv_selftest_wait_timeout": ([_vp, ctypes.c_uint64, _vp], _i32),
 }
 
 
@@ -244,6 +246,10 @@ def starkv_dequantize(ctx, which: int, codes, meta, n: int, z_out, stream=None):
     _need(meta, torch.int32, "meta")
     _need(z_out, torch.float32, "z_out", 2)
     _check(lib().starkv_dequantize(ctx, which, _p(codes), _p(meta), n, _p(z_out), _stream(stream)))
+
+
+def starkv_selftest_wait_timeout(ctx, limit_ns: int, stream=None) -> None:
+    _check(lib().starkv_selftest_wait_timeout(ctx, int(limit_ns), _stream(stream)))
 
 
 def starkv_read_device_status(ctx, stream=None) -> int:

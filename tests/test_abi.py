@@ -94,3 +94,8 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(starkv, "LIB_PATH", "/nonexistent/libstarkv.so")
     with pytest.raises(ImportError):
         starkv.starkv_version()
+
+
+def test_selftest_wait_timeout_checks_arguments_on_the_host(S):
+    # raw call (no stream lookup): the context and the limit are checked before any launch
+    assert S.lib().starkv_selftest_wait_timeout(None, 1_000_000, None) == S.ERR_INVALID_ARG

@@ -114,6 +114,9 @@ __global__ void __launch_bounds__(128) decode_wprep_kernel(const __nv_bfloat16* 
                                                            int max_pages, int max_position) {
   __shared__ float qs[kWpSeq][2][64];  // rotated, scaled (q~_i, q~_{i+d/2}) per sequence
   const int h = blockIdx.x, b0 = blockIdx.y * kWpSeq, tid = threadIdx.x;
+  // first kernel of a decode call: its inputs may come from any earlier kernel
+  pdl_wait();
+  pdl_launch_dependents();
   const int half = d / 2;
   const int kv = h / group, hg = h / hpc, hl = h % hpc;
   const float scale = kLog2e * rsqrtf((float)d);
@@ -378,6 +381,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int d = a.d;
 
+  // (before the wait: every kernel earlier than the query fold has completed)
   // zero the projection's sums and arrival counters (grid-stride over all CTAs)
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + tid; i < a.oacc_elems; i += (int64_t)gridDim.x * blockDim.x)
     a.oacc[i] = 0.f;
@@ -399,6 +403,8 @@ __global__ void __launch_bounds__(kAThreads, 1)
     *failed = 0;
     fence_mbar_init();
   }
+  pdl_wait();  // W images and zeroed maxima (query fold), appended codes
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -758,6 +764,8 @@ __global__ void __launch_bounds__(kVThreads, 1)
   const int split = blockIdx.x, b = blockIdx.y;
   const LatentGeom& V = a.val;
   const int NS = a.NS, PS = a.PS, ST = a.ST;
+  pdl_wait();  // scores, their maxima and the appended codes (every CTA, even one that leaves early)
+  pdl_launch_dependents();
 
   int L = a.seq_lens[b];
   const bool bad_len = L < 0 || L > a.max_pages * kPage || L > a.max_position;
@@ -1128,12 +1136,15 @@ __global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, i
     }
     nparts_s[tid] = np;
   }
-  // B'_v rows of this slice straight into shared memory
+  // B'_v rows of this slice straight into shared memory (they do not depend on
+  // the kernels before, so this overlaps the value kernel's tail)
   for (int e = tid; e < kc * (d / 8); e += 256) {
     const int r = e / (d / 8), q8 = e % (d / 8);
     *reinterpret_cast<uint4*>(&Bs[r][q8 * 8]) =
         __ldg(reinterpret_cast<const uint4*>(a.Bv16 + (int64_t)(ch0 + r) * ldg + kv * d + q8 * 8));
   }
+  pdl_wait();  // partial sums, l and the zeroed accumulators
+  pdl_launch_dependents();
   __syncthreads();
   if (tid < kProjM) {
     const int b = b0 + tid;
@@ -1462,7 +1473,8 @@ static cudaError_t launch_scores_g(const Ctx& c, const ScoreArgs& a, int grid, s
   cudaError_t e =
       cudaFuncSetAttribute(decode_scores_kernel<RK, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  decode_scores_kernel<RK, G><<<grid, kAThreads, smem, s>>>(c.trig_map, a);
+  e = launch_chained(decode_scores_kernel<RK, G>, dim3(grid), dim3(kAThreads), smem, s, 1u, c.trig_map, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -1494,20 +1506,22 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   // ---------------- W images: rotated query folded into B'_k, per (sequence, head)
   {
     dim3 g(f.num_q_heads, (batch + kWpSeq - 1) / kWpSeq);
+    cudaError_t e0 = cudaSuccess;
     switch (f.rank_k) {
       case 16:
-        decode_wprep_kernel<16><<<g, 128, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, Mx, f.num_q_heads, c.group, d, t.hpc,
-                                                 t.ncols, batch, max_pages, f.max_position);
+        e0 = launch_chained(decode_wprep_kernel<16>, g, dim3(128), 0, s, 1u, q, seq_lens, (const float*)c.Bk, (const float2*)c.rope, wimg, Mx,
+                            (int)f.num_q_heads, c.group, d, t.hpc, t.ncols, batch, max_pages, (int)f.max_position);
         break;
       case 32:
-        decode_wprep_kernel<32><<<g, 128, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, Mx, f.num_q_heads, c.group, d, t.hpc,
-                                                 t.ncols, batch, max_pages, f.max_position);
+        e0 = launch_chained(decode_wprep_kernel<32>, g, dim3(128), 0, s, 1u, q, seq_lens, (const float*)c.Bk, (const float2*)c.rope, wimg, Mx,
+                            (int)f.num_q_heads, c.group, d, t.hpc, t.ncols, batch, max_pages, (int)f.max_position);
         break;
       default:
-        decode_wprep_kernel<64><<<g, 128, 0, s>>>(q, seq_lens, c.Bk, c.rope, wimg, Mx, f.num_q_heads, c.group, d, t.hpc,
-                                                 t.ncols, batch, max_pages, f.max_position);
+        e0 = launch_chained(decode_wprep_kernel<64>, g, dim3(128), 0, s, 1u, q, seq_lens, (const float*)c.Bk, (const float2*)c.rope, wimg, Mx,
+                            (int)f.num_q_heads, c.group, d, t.hpc, t.ncols, batch, max_pages, (int)f.max_position);
         break;
     }
+    if (e0 != cudaSuccess) return e0;
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -1647,19 +1661,8 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
       return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(decode_values_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(t.splits, batch);
-    cfg.blockDim = dim3((kVRoleWarps + t.nW) * 32);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = t.CS;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_values_kernel, s_map, B);
+    e = launch_chained(decode_values_kernel, dim3(t.splits, batch), dim3((kVRoleWarps + t.nW) * 32), smem, s,
+                       (unsigned)t.CS, s_map, B);
     if (e != cudaSuccess) return e;
   }
 
@@ -1686,7 +1689,11 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   P.oacc = oacc;
   P.ocnt = ocnt;
   const int kc = f.rank_v % kProjC == 0 ? kProjC : 64;
-  decode_project_kernel<<<dim3(f.num_q_heads, f.rank_v / kc, (batch + kProjM - 1) / kProjM), 256, 0, s>>>(P, batch, kc);
+  {
+    cudaError_t e = launch_chained(decode_project_kernel, dim3(f.num_q_heads, f.rank_v / kc, (batch + kProjM - 1) / kProjM),
+                                   dim3(256), 0, s, 1u, P, batch, kc);
+    if (e != cudaSuccess) return e;
+  }
   return cudaGetLastError();
 }
 

@@ -254,6 +254,7 @@ __global__ void __launch_bounds__(256, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c0 = blockIdx.x * kAgCols, ks = blockIdx.y, k0 = ks * KL;
   const int n = (int)a.n, mtiles = (n + 15) / 16;
+  sm100::pdl_launch_dependents();
   const int box_rows = KL < 256 ? KL : 256;
   const int nbox = 2 * (KL / box_rows);
   if (tid == 0) {
@@ -331,6 +332,8 @@ __global__ void __launch_bounds__(256, 1)
 constexpr int kMaxAppSplits = 16;
 
 __global__ void __launch_bounds__(128) append_quant_kernel(AppendArgs a, const float* zpart, int splits) {
+  sm100::pdl_wait();  // the split sums of the projection kernel
+  sm100::pdl_launch_dependents();
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int units = a.lat_cols / 4;
   const bool active = idx < a.n * units;
@@ -416,7 +419,9 @@ cudaError_t launch_append(const Ctx& c, const starkv_cache& cache, const __nv_bf
     dim3 g1((unsigned)((c.lat_cols + kAgCols - 1) / kAgCols), (unsigned)c.app_splits);
     append_gemm_kernel<<<g1, 256, smem, s>>>(c.a_map, a, KL, c.zpart);
     const int64_t units = n * (c.lat_cols / 4);
-    append_quant_kernel<<<(unsigned)((units + 127) / 128), 128, 0, s>>>(a, c.zpart, c.app_splits);
+    e = launch_chained(append_quant_kernel, dim3((unsigned)((units + 127) / 128)), dim3(128), 0, s, 1u, a,
+                       (const float*)c.zpart, c.app_splits);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
   dim3 grid((unsigned)((n + kAppBM - 1) / kAppBM), (unsigned)((c.lat_cols + kAppBN - 1) / kAppBN));

@@ -38,7 +38,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) of one decode call, summed over its four kernels,
 # from one ncu capture of the current kernels (profiles/decode_kernels_*.md);
 # None for a workload without a capture.  Reset whenever a decode kernel changes.
-DECODE_TRAFFIC_NCU = {"longchat7b_decode_b16_t4096": 133_788_000}
+DECODE_TRAFFIC_NCU = {"longchat7b_decode_b16_t4096": 134_520_000}
 
 
 # ---------------------------------------------------------------------------
@@ -251,6 +251,118 @@ class DecodeState:
             ev[1].record()
 
 
+class PrefillState:
+    """Chunked prefill: each sequence holds `ctx` packed tokens; a step appends the
+    next `chunk` tokens (their hidden states through the projection, rotation,
+    quantiser and packer) and runs causal attention of those `chunk` queries over
+    all ctx + chunk positions."""
+
+    def __init__(self, w, seed, device):
+        import torch
+        from rank_mixed_precision_b200 import starkv as S
+        self.S = S
+        bf = lambda a: torch.from_numpy(gen.bf16_bits(a).view(np.int16).copy()).view(torch.bfloat16).to(device)
+        f = gen.make_factors(w, seed)
+        B, T0, C = w.batch, w.ctx, w.chunk
+        self.total = T0 + C
+        cfg = S.make_config(w.H, w.h_kv, w.d_h, w.hidden, w.r_k, w.R, self.total + 16, w.top_fraction, w.rope_base)
+        self.kv = S.StarKV(cfg, bf(f.A_k), bf(f.A_v), bf(f.B_k), bf(f.B_v))
+        bt, n_pages = gen.make_block_table(np.full(B, self.total, np.int32), seed)
+        self.cache = self.kv.new_cache(n_pages)
+        step = 4096
+        for b in range(B):
+            for s0 in range(0, T0, step):
+                n = min(step, T0 - s0)
+                X = bf(gen.make_hidden(n, w.hidden, seed, name="X", sub=1000 * b + s0 // step))
+                slots = torch.from_numpy(gen.slots_for(bt, b, np.arange(s0, s0 + n))).to(device)
+                self.kv.append(self.cache, X, slots)
+        torch.cuda.synchronize()
+        self.X = bf(gen.make_hidden(B * C, w.hidden, seed, name="X_chunk"))
+        self.slots = torch.from_numpy(np.concatenate([gen.slots_for(bt, b, np.arange(T0, T0 + C))
+                                                      for b in range(B)])).to(device)
+        self.q = bf(gen.make_queries(B * C, w.H, w.d_h, seed, name="q_chunk"))
+        self.cu_q = torch.tensor(np.arange(B + 1, dtype=np.int32) * C).to(device)
+        self.bt = torch.from_numpy(bt).to(device)
+        self.sl = torch.full((B,), self.total, dtype=torch.int32, device=device)
+        self.out = torch.empty_like(self.q)
+        self.ws = self.kv.workspace(S.OP_PREFILL, B, bt.shape[1], B * C)
+        st = self.kv.status()
+        if st:
+            raise RuntimeError(f"device status {st:#x} after cache fill")
+
+    def step(self, ev=None):
+        S = self.S
+        S.starkv_append(self.kv.ctx, self.cache.struct, self.X, self.slots)
+        if ev is not None:
+            ev[0].record()
+        S.starkv_prefill_attn(self.kv.ctx, self.cache.struct, self.q, self.cu_q, self.bt, self.sl,
+                              self.q.shape[0] // self.sl.shape[0], self.out, self.ws)
+        if ev is not None:
+            ev[1].record()
+
+
+def prefill_flops(w) -> dict:
+    """Algorithmic flops of one prefill step (causal QK and PV, values and keys
+    re-expanded once per position and KV head, the chunk's projection)."""
+    T0, C = w.ctx, w.chunk
+    pairs = C * T0 + C * (C + 1) // 2                       # (query, key) pairs of one sequence
+    attn = pairs * w.H * 4 * w.d_h
+    vexp = (T0 + C) * w.h_kv * w.R * w.d_h * 2
+    kexp = (T0 + C) * w.h_kv * w.r_k * w.d_h * 2
+    proj = C * w.hidden * (w.h_kv * w.r_k + w.R) * 2
+    per = {"attention": attn, "value_reexpansion": vexp, "key_reexpansion": kexp, "projection": proj}
+    return {k: v * w.batch for k, v in per.items()}
+
+
+def run_prefill(args, w, rank, world, local):
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    st = PrefillState(w, args.seed, device)
+    for _ in range(args.warmup):
+        st.step()
+    torch.cuda.synchronize()
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record()
+        for i in range(args.steps):
+            st.step(pairs[i])
+        t1.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    if st.kv.status():
+        raise RuntimeError("device status set during the timed region")
+    fl = prefill_flops(w)
+    total = sum(fl.values())
+    value, ms_max = job_throughput(total * args.steps / 1e12, t0.elapsed_time(t1), world, device)
+    attn_ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+    if rank != 0:
+        return None
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        pass
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+    achieved = (total - fl["projection"]) / (attn_ms / 1e3) / 1e12
+    return {
+        "metric": "prefill TFLOP/s (algorithmic)", "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32 (CUDA-core prefill)", "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "batch": w.batch, "ctx": w.ctx, "chunk": w.chunk,
+                   "step": "append the chunk + causal prefill attention of its queries"},
+        "flops_per_step": fl,
+        "roofline": {"bound": "tensor", "kernel": "starkv_prefill_attn (expand + attention kernels)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": None, "launch_ms": attn_ms},
+        "clocks": clk.summary(),
+    }
+
+
 def run_starkv(args, w, rank, world, local):
     import torch
     torch.cuda.set_device(local)
@@ -443,6 +555,8 @@ def main(argv=None):
     w = gen.workload(args.workload)
     if args.impl == "reference":
         line = run_reference(args, w, rank, world)
+    elif w.chunk > 0:
+        line = run_prefill(args, w, rank, world, local)
     else:
         line = run_starkv(args, w, rank, world, local)
     if line is not None:

@@ -94,16 +94,16 @@ struct ScoreArgs {
 };
 
 // ---------------------------------------------------------------------------
-// W prep: one CTA per (head, 4 sequences).  With q~ the query rotated to its
+// W prep: one CTA per (head, sequence).  With q~ the query rotated to its
 // position and i < d/2 a frequency pair (i, i + d/2), for every latent channel c
 //   W[c][i]       = (q~_i B'[c,i] + q~_{i+d/2} B'[c,i+d/2]) * log2(e)/sqrt(d)
 //   W[c][i + d/2] = (q~_{i+d/2} B'[c,i] - q~_i B'[c,i+d/2]) * log2(e)/sqrt(d)
-// A thread owns (c, 8 consecutive i): it reads those B' values once, reuses them
-// for the 4 sequences and writes 16-byte fp16 chunks straight into the score
-// kernel's shared-memory image (K-major, 128-byte swizzle).  The CTA also zeroes
-// the running score maxima of its (sequence, head) pairs.
+// A thread owns (c, 8 consecutive i): it reads those B' values (L2-resident) and
+// writes 16-byte fp16 chunks straight into the score kernel's shared-memory
+// image (K-major, 128-byte swizzle).  The CTA also zeroes the running score
+// maxima of its (sequence, head) pairs.
 // ---------------------------------------------------------------------------
-constexpr int kWpSeq = 4;  // sequences per W-prep CTA
+constexpr int kWpSeq = 1;  // sequences per W-prep CTA
 
 template <int RK>
 __global__ void __launch_bounds__(128) decode_wprep_kernel(const __nv_bfloat16* __restrict__ q,

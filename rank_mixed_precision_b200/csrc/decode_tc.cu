@@ -205,29 +205,6 @@ __device__ __forceinline__ void tmem_wait_row(uint32_t (&r)[RK]) {
   }
 }
 
-template <int RK>
-__device__ __forceinline__ void tmem_load_row(uint32_t taddr, float (&G)[RK]) {
-  uint32_t r[32];
-  if constexpr (RK == 16) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 16; ++i) G[i] = __uint_as_float(r[i]);
-  } else {
-#pragma unroll
-    for (int h = 0; h < RK / 32; ++h) {
-      tmem_ld32(taddr + h * 32, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) G[h * 32 + i] = __uint_as_float(r[i]);
-    }
-  }
-}
-
 // ---------------------------------------------------------------------------
 // Key dot product on packed codes (one token, one head), compile-time layout.
 //
@@ -301,10 +278,6 @@ struct KeyGroup {
 };
 
 // sum_c z_hat_c G_c over one token's key latent in a staged page region.
-template <int RK, int G>
-__device__ __forceinline__ float key_dot(const uint8_t* region, const uint32_t* meta, int top_groups, int t16,
-                                         const uint32_t (&raw)[RK]);
-
 // Two heads' scores at once: the groups of both are independent, so their
 // dependency chains interleave.
 template <int RK, int G>

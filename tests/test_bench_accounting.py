@@ -1,0 +1,56 @@
+"""The bench's roofline denominators against closed forms.
+
+Algorithmic bytes of a decode call and algorithmic flops of a prefill step
+are what the reported fractions divide by; these tests recompute them from the
+shapes alone (packed bits per channel, metadata per group, factor sizes,
+causal pair counts) so a change to either side shows up here.
+"""
+import pytest
+
+import bench
+from harness import gen
+
+
+def _closed_form_bytes_per_token(w):
+    def region(r):
+        n_top = int(round(w.top_fraction * r))
+        return 2 * (4 * n_top + 3 * (r - n_top))  # one page (16 tokens) of one latent region
+
+    def groups(r):
+        import math
+        n_top = int(round(w.top_fraction * r))
+        g = math.gcd(16, math.gcd(n_top, r - n_top))
+        return r // g
+
+    key = w.h_kv * (region(w.r_k) / 16 + 4 * groups(w.r_k))
+    val = region(w.R) / 16 + 4 * groups(w.R)
+    return key + val
+
+
+@pytest.mark.parametrize("name,expect", [("longchat7b_decode_b16_t4096", 1600), ("llama3_8b_gqa_decode_b32_t4096to8192", 672)])
+def test_bytes_per_token_is_payload_plus_metadata(name, expect):
+    w = gen.workload(name)
+    assert bench.bytes_per_token(w) == expect
+    assert _closed_form_bytes_per_token(w) == expect
+
+
+def test_decode_algorithmic_bytes_on_the_bench_workload():
+    w = gen.workload("longchat7b_decode_b16_t4096")
+    tokens, max_pages = w.batch * w.ctx, w.ctx // 16 + 1
+    got = bench.decode_algorithmic_bytes(w, tokens, w.batch, max_pages)
+    factors = 2 * (32 * 32 * 128 + 1024 * 32 * 128)  # bf16 B_k and B_v
+    assert got == tokens * 1600 + factors + 2 * 2 * 16 * 32 * 128 + 4 * 16 * max_pages + 4 * 16
+    assert 113e6 < got < 114.5e6  # the scope table quotes 113.5 MB (cache 104.86 MB + B_v 8.39 MB + B_k 0.26 MB)
+
+
+def test_prefill_flops_match_the_scope_table():
+    w = gen.workload("longchat7b_prefill_b4_t30720_c2048")
+    fl = bench.prefill_flops(w)
+    # per sequence: causal pairs of 2048 queries at positions 30720.. over all earlier keys
+    pairs = 2048 * 30720 + 2048 * 2049 // 2
+    assert fl["attention"] == 4 * pairs * 32 * 4 * 128
+    assert fl["attention"] / 4 == pytest.approx(1.065e12, rel=1e-3)
+    assert fl["value_reexpansion"] / 4 == pytest.approx(0.275e12, rel=1e-3)
+    assert fl["key_reexpansion"] / 4 == pytest.approx(8.6e9, rel=1e-2)
+    assert fl["projection"] / 4 == pytest.approx(34e9, rel=2e-2)
+    assert sum(fl.values()) == pytest.approx(5.53e12, rel=1e-3)

@@ -99,3 +99,31 @@ def test_missing_library_fails_loudly(monkeypatch):
 def test_selftest_wait_timeout_checks_arguments_on_the_host(S):
     # raw call (no stream lookup): the context and the limit are checked before any launch
     assert S.lib().starkv_selftest_wait_timeout(None, 1_000_000, None) == S.ERR_INVALID_ARG
+
+
+def test_every_entry_point_rejects_a_null_context_before_any_device_work(S):
+    """Raw C calls with NULL handles: each returns INVALID_ARG (and sets a message)
+    from the host-side checks, without a device or a CUDA call."""
+    L = S.lib()
+    sz = ctypes.c_size_t()
+    u32 = ctypes.c_uint32()
+    calls = {
+        "starkv_append": lambda: L.starkv_append(None, None, None, None, 0, None, None),
+        "starkv_decode_attn": lambda: L.starkv_decode_attn(None, None, None, None, None, 1, 1, None, None, 0, None),
+        "starkv_decode_attn_noalloc": lambda: L.starkv_decode_attn_noalloc(None, None, None, None, None, 1, 1, None, None),
+        "starkv_prefill_attn": lambda: L.starkv_prefill_attn(None, None, None, None, None, None, 1, 1, 1, 1, None, None,
+                                                            0, None),
+        "starkv_workspace_bytes": lambda: L.starkv_workspace_bytes(None, 0, 1, 1, 0, ctypes.byref(sz)),
+        "starkv_quantize_pack": lambda: L.starkv_quantize_pack(None, 0, None, 0, None, None, None),
+        "starkv_dequantize": lambda: L.starkv_dequantize(None, 0, None, None, 0, None, None),
+        "starkv_read_device_status": lambda: L.starkv_read_device_status(None, None, ctypes.byref(u32)),
+        "starkv_get_config": lambda: L.starkv_get_config(None, None),
+        "starkv_cache_layout": lambda: L.starkv_cache_layout(None, 1, None),
+        "starkv_create": lambda: L.starkv_create(None, None, None, None, None, None, None),
+        "starkv_selftest_wait_timeout": lambda: L.starkv_selftest_wait_timeout(None, 1_000_000, None),
+    }
+    assert set(calls) | {"starkv_version", "starkv_last_error", "starkv_destroy"} == set(S.EXPORTS)
+    for name, call in calls.items():
+        assert call() == S.ERR_INVALID_ARG, name
+        assert S.starkv_last_error(), name
+    assert L.starkv_destroy(None) == S.OK  # destroying nothing is allowed

@@ -161,6 +161,22 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def pack_layout(tensors, align: int = 256):
+    """Byte offsets that lay `tensors` out back to back in one buffer, each
+    start rounded up to `align`, and the buffer's total size."""
+    offs, total = [], 0
+    for t in tensors:
+        total = -(-total // align) * align
+        offs.append(total)
+        total += t.numel() * t.element_size()
+    return offs, total
+
+
+def packed_views(buf, offs, like):
+    """Typed views of the 1-D uint8 `buf` at `offs`, shaped like `like`."""
+    return [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape) for o, t in zip(offs, like)]
+
+
 # ---------------------------------------------------------------------------
 # workload state on the GPU
 # ---------------------------------------------------------------------------
@@ -395,19 +411,23 @@ def run_starkv(args, w, rank, world, local):
         raise RuntimeError(f"device status {status:#x} during the timed region")
     tokens_per_step = int(st.seq_lens.sum())
     value, ms_max = job_throughput(tokens_per_step * args.steps, ms, world, device)
-    # ---- end to end through the public API with host buffers
-    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
-    Xh = pin(gen.bf16_bits(st.X_np).view(np.int16)).view(torch.bfloat16)
-    qh = pin(gen.bf16_bits(st.q_np).view(np.int16)).view(torch.bfloat16)
-    slh, bth, lh = pin(st.slots_np), pin(st.bt_np), pin(st.seq_lens.astype(np.int32))
+    # ---- end to end through the public API with host buffers: the step's
+    # inputs sit packed in one pinned staging buffer and cross in one copy
+    t_ = lambda a: torch.from_numpy(np.ascontiguousarray(a))
+    srcs = [t_(gen.bf16_bits(st.X_np).view(np.int16)).view(torch.bfloat16),
+            t_(gen.bf16_bits(st.q_np).view(np.int16)).view(torch.bfloat16),
+            t_(st.slots_np), t_(st.bt_np), t_(st.seq_lens.astype(np.int32))]
+    offs, h2d = pack_layout(srcs)
+    hbuf = torch.zeros(h2d, dtype=torch.uint8).pin_memory()
+    for v, s in zip(packed_views(hbuf, offs, srcs), srcs):
+        v.copy_(s)
+    dbuf = torch.empty(h2d, dtype=torch.uint8, device=device)
+    Xd, qd, sld, btd, ld = packed_views(dbuf, offs, srcs)
     outh = torch.empty(st.q.shape, dtype=torch.bfloat16).pin_memory()
-    Xd, qd, sld, btd, ld = (torch.empty_like(t, device=device) for t in (Xh, qh, slh, bth, lh))
-    h2d = sum(t.numel() * t.element_size() for t in (Xh, qh, slh, bth, lh))
     d2h = outh.numel() * outh.element_size()
 
     def e2e_step(i):
-        for d, h in ((Xd, Xh), (qd, qh), (sld, slh), (btd, bth), (ld, lh)):
-            d.copy_(h, non_blocking=True)
+        dbuf.copy_(hbuf, non_blocking=True)
         c = st.caches[i % len(st.caches)]
         S.starkv_append(st.kv.ctx, c.struct, Xd, sld)
         S.starkv_decode_attn(st.kv.ctx, c.struct, qd, btd, ld, st.out, st.ws)

@@ -54,3 +54,24 @@ def test_prefill_flops_match_the_scope_table():
     assert fl["key_reexpansion"] / 4 == pytest.approx(8.6e9, rel=1e-2)
     assert fl["projection"] / 4 == pytest.approx(34e9, rel=2e-2)
     assert sum(fl.values()) == pytest.approx(5.53e12, rel=1e-3)
+
+
+def test_packed_staging_buffer_round_trips_every_input():
+    """The end-to-end leg stages a step's inputs in one byte buffer: every
+    view must start aligned, not overlap the next, and read back its input."""
+    import torch
+    srcs = [torch.arange(16 * 4096, dtype=torch.float32).to(torch.bfloat16).view(16, 4096),
+            torch.randn(16, 32, 128).to(torch.bfloat16),
+            torch.arange(16, dtype=torch.int64) * 7 + 3,
+            torch.arange(16 * 257, dtype=torch.int32).view(16, 257),
+            torch.arange(16, dtype=torch.int32) + 4000]
+    offs, total = bench.pack_layout(srcs)
+    assert all(o % 256 == 0 for o in offs)
+    ends = [o + s.numel() * s.element_size() for o, s in zip(offs, srcs)]
+    assert all(e <= n for e, n in zip(ends, offs[1:])) and ends[-1] == total
+    buf = torch.zeros(total, dtype=torch.uint8)
+    for v, s in zip(bench.packed_views(buf, offs, srcs), srcs):
+        v.copy_(s)
+    for v, s in zip(bench.packed_views(buf.clone(), offs, srcs), srcs):
+        assert v.dtype == s.dtype and v.shape == s.shape and v.is_contiguous()
+        assert torch.equal(v, s)

@@ -1076,6 +1076,7 @@ struct ProjArgs {
 
 constexpr int kProjM = 16;   // sequences per projection CTA (the MMA's M)
 constexpr int kProjC = 128;  // latent channels per projection CTA
+constexpr int kProjVecLoads = kProjC * (128 / 8) / 256;  // 16-byte B'_v loads per thread at d = 128
 
 // grid (H, R / kc, ceil(B / 16)), 256 threads, kc = 128 channels (64 when R is
 // not a multiple of 128).  Every load of the CTA (its
@@ -1110,43 +1111,71 @@ __global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, i
     nparts_s[tid] = np;
   }
   // B'_v rows of this slice straight into shared memory (they do not depend on
-  // the kernels before, so this overlaps the value kernel's tail)
-  for (int e = tid; e < kc * (d / 8); e += 256) {
-    const int r = e / (d / 8), q8 = e % (d / 8);
-    *reinterpret_cast<uint4*>(&Bs[r][q8 * 8]) =
-        __ldg(reinterpret_cast<const uint4*>(a.Bv16 + (int64_t)(ch0 + r) * ldg + kv * d + q8 * 8));
+  // the kernels before, so this overlaps the value kernel's tail).  All of a
+  // thread's loads are issued before the first store.
+  {
+    const int nvec = kc * (d / 8);
+    uint4 v[kProjVecLoads];
+#pragma unroll
+    for (int i = 0; i < kProjVecLoads; ++i) {
+      const int e = tid + i * 256, r = e / (d / 8), q8 = e % (d / 8);
+      if (e < nvec) v[i] = __ldg(reinterpret_cast<const uint4*>(a.Bv16 + (int64_t)(ch0 + r) * ldg + kv * d + q8 * 8));
+    }
+#pragma unroll
+    for (int i = 0; i < kProjVecLoads; ++i) {
+      const int e = tid + i * 256, r = e / (d / 8), q8 = e % (d / 8);
+      if (e < nvec) *reinterpret_cast<uint4*>(&Bs[r][q8 * 8]) = v[i];
+    }
   }
   pdl_wait();  // partial sums, l and the zeroed accumulators
   pdl_launch_dependents();
   __syncthreads();
   if (tid < kProjM) {
-    const int b = b0 + tid;
+    const int b = b0 + tid, np = nparts_s[tid];
     float l = 0.f;
-    for (int sp = 0; sp < nparts_s[tid]; ++sp) l += __ldcg(a.lpart + ((int64_t)b * a.nclust + sp) * a.H + h);
+    for (int sp0 = 0; sp0 < np; sp0 += 4) {
+      float v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        v[u] = sp0 + u < np ? __ldcg(a.lpart + ((int64_t)b * a.nclust + sp0 + u) * a.H + h) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) l += v[u];
+    }
     linv[tid] = l > 0.f ? 1.f / l : 0.f;
   }
-  // o_lat sums: 2 items of 4 channels per thread (16 sequences x 32 quads)
+  // o_lat sums: 2 items of 4 channels per thread (16 sequences x 32 quads),
+  // added in partial order; both items' loads of a round are in flight together
   float4 acc[2];
+  const float* base[2];
+  int np[2];
   const int items = kProjM * (kc / 4);
+  const int64_t stride = (int64_t)a.H * R;
 #pragma unroll
   for (int it = 0; it < 2; ++it) {
     const int e = tid + it * 256;
     const int r = e / (kc / 4), c4 = (e % (kc / 4)) * 4;
     const int b = b0 + r;
     acc[it] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (e < items && b < batch) {
-      const int np = nparts_s[r];
-      const float* base = a.part + ((int64_t)b * a.nclust * a.H + h) * R + ch0 + c4;
-      const int64_t stride = (int64_t)a.H * R;
-#pragma unroll 4
-      for (int sp = 0; sp < np; ++sp) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(base + sp * stride));
-        acc[it].x += v.x;
-        acc[it].y += v.y;
-        acc[it].z += v.z;
-        acc[it].w += v.w;
+    np[it] = (e < items && b < batch) ? nparts_s[r] : 0;
+    base[it] = a.part + ((int64_t)b * a.nclust * a.H + h) * R + ch0 + c4;
+  }
+  for (int sp0 = 0; sp0 < max(np[0], np[1]); sp0 += 4) {
+    float4 v[2][4];
+#pragma unroll
+    for (int it = 0; it < 2; ++it)
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        v[it][u] = sp0 + u < np[it] ? __ldcg(reinterpret_cast<const float4*>(base[it] + (sp0 + u) * stride))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int it = 0; it < 2; ++it)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc[it].x += v[it][u].x;
+        acc[it].y += v[it][u].y;
+        acc[it].z += v[it][u].z;
+        acc[it].w += v[it][u].w;
       }
-    }
   }
   __syncthreads();
 #pragma unroll
@@ -1190,11 +1219,23 @@ __global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, i
   __syncthreads();
   if (last) {
     __threadfence();
-    for (int e = tid; e < kProjM * d; e += 256) {
-      const int b = b0 + e / d, col = e % d;
-      if (b < batch) {
-        const int64_t o = ((int64_t)b * a.H + h) * d + col;
-        a.out[o] = __float2bfloat16_rn(__ldcg(a.oacc + o));
+    // 4 columns per item, both items' loads before the stores
+    float4 v[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int e = (tid + i * 256) * 4, b = b0 + e / d;
+      if (e < kProjM * d && b < batch)
+        v[i] = __ldcg(reinterpret_cast<const float4*>(a.oacc + ((int64_t)b * a.H + h) * d + e % d));
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int e = (tid + i * 256) * 4, b = b0 + e / d;
+      if (e < kProjM * d && b < batch) {
+        __nv_bfloat16* o = a.out + ((int64_t)b * a.H + h) * d + e % d;
+        o[0] = __float2bfloat16_rn(v[i].x);
+        o[1] = __float2bfloat16_rn(v[i].y);
+        o[2] = __float2bfloat16_rn(v[i].z);
+        o[3] = __float2bfloat16_rn(v[i].w);
       }
     }
   }

@@ -181,6 +181,17 @@ def packed_views(buf, offs, like):
     return [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape) for o, t in zip(offs, like)]
 
 
+def stream_schedule(seq_lens0, n_steps: int, block_table):
+    """Long-context stream: at step s every sequence appends the token at
+    position L0 + s and then decodes its context of L0 + s + 1 tokens.
+    Returns (slots [n_steps, B] int64, seq_lens [n_steps, B] int32)."""
+    L0 = np.asarray(seq_lens0, np.int64)
+    steps = np.arange(n_steps, dtype=np.int64)
+    slots = np.stack([gen.slots_for(block_table, b, L0[b] + steps) for b in range(L0.shape[0])], axis=1)
+    lens = (L0[None, :] + steps[:, None] + 1).astype(np.int32)
+    return slots.reshape(n_steps, L0.shape[0]), lens
+
+
 # ---------------------------------------------------------------------------
 # workload state on the GPU
 # ---------------------------------------------------------------------------
@@ -266,6 +277,86 @@ class DecodeState:
         if ev is not None:
             ev[0].record()
         if self.lib.starkv_decode_attn(*dec):
+            raise RuntimeError(self.lib.starkv_last_error().decode())
+        if ev is not None:
+            ev[1].record()
+
+
+class StreamState:
+    """Long-context stream (batch-1 style): run step i is stream step
+    s = i mod n, which appends one token per sequence at position L0 + s and
+    decodes the grown context of L0 + s + 1 tokens.
+
+    Every replica is filled through all n stream positions before timing, the
+    stream positions by the same single-token append a step issues, so a step's
+    append rewrites identical bytes, and a decode, which reads only positions
+    below its length, always sees exactly the stream's context."""
+
+    def __init__(self, w, seed, device, replicas):
+        import ctypes
+        import torch
+        from rank_mixed_precision_b200 import starkv as S
+        self.S, self.w, self.n = S, w, w.steps
+        bf = lambda a: torch.from_numpy(gen.bf16_bits(a).view(np.int16).copy()).view(torch.bfloat16).to(device)
+        f = gen.make_factors(w, seed)
+        B, n = w.batch, w.steps
+        self.L0 = gen.make_seq_lens(w, seed)
+        caps = self.L0.astype(np.int64) + n
+        cfg = S.make_config(w.H, w.h_kv, w.d_h, w.hidden, w.r_k, w.R, int(caps.max()) + 16, w.top_fraction,
+                            w.rope_base)
+        self.kv = S.StarKV(cfg, bf(f.A_k), bf(f.A_v), bf(f.B_k), bf(f.B_v))
+        bt, n_pages = gen.make_block_table(caps, seed)
+        self.bt_np, self.max_pages = bt, bt.shape[1]
+        self.slots_np, self.lens_np = stream_schedule(self.L0, n, bt)
+        self.X_np = np.stack([gen.make_hidden(B, w.hidden, seed, name="X_step", sub=s) for s in range(n)])
+        self.q_np = np.stack([gen.make_queries(B, w.H, w.d_h, seed, name="q_step", sub=s) for s in range(n)])
+        self.X, self.q = bf(self.X_np), bf(self.q_np)
+        self.slots = torch.from_numpy(self.slots_np).to(device)
+        self.lens = torch.from_numpy(self.lens_np).to(device)
+        self.bt = torch.from_numpy(bt).to(device)
+        self.caches = [self.kv.new_cache(n_pages) for _ in range(replicas)]
+        c0 = self.caches[0]
+        chunk = 4096
+        for b in range(B):
+            L = int(self.L0[b])
+            for s0 in range(0, L, chunk):
+                m = min(chunk, L - s0)
+                X = bf(gen.make_hidden(m, w.hidden, seed, name="X", sub=1000 * b + s0 // chunk))
+                sl = torch.from_numpy(gen.slots_for(bt, b, np.arange(s0, s0 + m))).to(device)
+                self.kv.append(c0, X, sl)
+        for s in range(n):
+            self.kv.append(c0, self.X[s], self.slots[s])
+        torch.cuda.synchronize()
+        for c in self.caches[1:]:
+            for name in ("k_codes", "v_codes", "k_meta", "v_meta"):
+                getattr(c, name).copy_(getattr(c0, name))
+        self.out = torch.empty_like(self.q[0])
+        self.ws = self.kv.workspace(S.OP_DECODE, B, self.max_pages)
+        st = self.kv.status()
+        if st:
+            raise RuntimeError(f"device status {st:#x} after cache fill")
+        # pre-marshalled C-ABI arguments (the timed loop calls the C entry points directly)
+        self.lib = S.lib()
+        vp = ctypes.c_void_p
+        strm = vp(torch.cuda.current_stream().cuda_stream)
+        self.refs = [ctypes.byref(c.struct) for c in self.caches]
+        self.app = [(vp(self.X[s].data_ptr()), vp(self.slots[s].data_ptr()), B, None, strm) for s in range(n)]
+        self.dec = [(vp(self.q[s].data_ptr()), vp(self.bt.data_ptr()), vp(self.lens[s].data_ptr()), B,
+                     self.max_pages, vp(self.out.data_ptr()), vp(self.ws.data_ptr()), self.ws.numel(), strm)
+                    for s in range(n)]
+
+    def tokens(self, i) -> int:
+        """Context tokens the decode of run step i attends to."""
+        return int(self.lens_np[i % self.n].sum())
+
+    def step(self, i, ev=None):
+        s, ref = i % self.n, self.refs[i % len(self.refs)]
+        x, sl, B, lat, strm = self.app[s]
+        if self.lib.starkv_append(self.kv.ctx, ref, x, sl, B, lat, strm):
+            raise RuntimeError(self.lib.starkv_last_error().decode())
+        if ev is not None:
+            ev[0].record()
+        if self.lib.starkv_decode_attn(self.kv.ctx, ref, *self.dec[s]):
             raise RuntimeError(self.lib.starkv_last_error().decode())
         if ev is not None:
             ev[1].record()
@@ -491,6 +582,122 @@ def run_starkv(args, w, rank, world, local):
     return line
 
 
+def run_stream(args, w, rank, world, local):
+    """Long-context stream: each timed step appends one token per sequence and
+    decodes the grown context; the run walks the stream's steps in order."""
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    replicas = max(2, int(np.ceil(3 * L2_BYTES / max(1, w.batch * w.ctx * bytes_per_token(w)))))
+    st = StreamState(w, args.seed, device, replicas)
+    S = st.S
+    launches_per_step = 6  # append (split-K projection, quantise), decode (query fold, scores, values, projection)
+    for i in range(args.warmup):
+        st.step(i)
+    torch.cuda.synchronize()
+    # ---- device-resident timed region: stream steps 0, 1, ... in order
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record()
+        for i in range(args.steps):
+            st.step(i, pairs[i])
+        t1.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = t0.elapsed_time(t1)
+    dec_ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+    status = st.kv.status()
+    if status:
+        raise RuntimeError(f"device status {status:#x} during the timed region")
+    tokens = sum(st.tokens(i) for i in range(args.steps))
+    value, ms_max = job_throughput(tokens, ms, world, device)
+    # ---- end to end through the public API with host buffers: each stream
+    # step's inputs sit packed in one row of a pinned staging buffer
+    t_ = lambda a: torch.from_numpy(np.ascontiguousarray(a))
+
+    def host_inputs(s):
+        return [t_(gen.bf16_bits(st.X_np[s]).view(np.int16)).view(torch.bfloat16),
+                t_(gen.bf16_bits(st.q_np[s]).view(np.int16)).view(torch.bfloat16),
+                t_(st.slots_np[s]), t_(st.bt_np), t_(st.lens_np[s])]
+
+    offs, h2d = pack_layout(host_inputs(0))
+    hbuf = torch.zeros((st.n, h2d), dtype=torch.uint8).pin_memory()
+    for s in range(st.n):
+        srcs = host_inputs(s)
+        for v, x in zip(packed_views(hbuf[s], offs, srcs), srcs):
+            v.copy_(x)
+    dbuf = torch.empty(h2d, dtype=torch.uint8, device=device)
+    Xd, qd, sld, btd, ld = packed_views(dbuf, offs, host_inputs(0))
+    outh = torch.empty(st.out.shape, dtype=torch.bfloat16).pin_memory()
+    d2h = outh.numel() * outh.element_size()
+
+    def e2e_step(i):
+        dbuf.copy_(hbuf[i % st.n], non_blocking=True)
+        c = st.caches[i % len(st.caches)]
+        S.starkv_append(st.kv.ctx, c.struct, Xd, sld)
+        S.starkv_decode_attn(st.kv.ctx, c.struct, qd, btd, ld, st.out, st.ws)
+        outh.copy_(st.out, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_value, _ = job_throughput(tokens, e0.elapsed_time(e1), world, device)
+
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peaks()
+    mean_tokens = tokens / args.steps
+    alg = decode_algorithmic_bytes(w, mean_tokens, w.batch, st.max_pages)
+    achieved = alg / (dec_ms / 1e3) / 1e9
+    L0, Ln = int(st.L0.max()), int(st.L0.max()) + st.n
+    line = {
+        "metric": "decode context-tokens/s",
+        "value": value,
+        "unit": "context-tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp16 tensor-core operands, fp32 accumulation",
+        "data": "synthetic (seeded; shapes of the named model, no weights)",
+        "config": {"workload": w.name, "batch": w.batch, "ctx": f"{L0} -> {Ln}",
+                   "heads": w.H, "kv_heads": w.h_kv, "head_dim": w.d_h, "rank_k": w.r_k, "rank_v": w.R,
+                   "bits": "4/3 (top 25% of channels 4-bit)", "page_tokens": 16,
+                   "step": f"append 1 token per sequence + decode of the grown context; "
+                           f"run step i is stream step i mod {st.n}",
+                   "parallelism": f"dp{world} (independent sequences per GPU)",
+                   "l2": f"{len(st.caches)} rotating cache replicas "
+                         f"({len(st.caches) * st.caches[0].nbytes() / 2**20:.0f} MiB > 126 MiB L2)"},
+        "roofline": {"bound": "hbm", "kernel": "starkv_decode_attn (scores + values + projection kernels)",
+                     "achieved": achieved, "peak": peak, "peak_kind": f"hbm copy GB/s ({peak_kind})",
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": DECODE_TRAFFIC_NCU.get(w.name),
+                     "algorithmic_bytes_per_launch": alg, "launch_ms": dec_ms,
+                     "achieved_context_tokens_per_s_decode_only": mean_tokens / (dec_ms / 1e3)},
+        "e2e": {"value": e2e_value, "unit": "context-tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.seed, args.cpu_seconds)
+    return line
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample)
 # ---------------------------------------------------------------------------
@@ -582,6 +789,8 @@ def main(argv=None):
         line = run_reference(args, w, rank, world)
     elif w.chunk > 0:
         line = run_prefill(args, w, rank, world, local)
+    elif w.steps > 0:
+        line = run_stream(args, w, rank, world, local)
     else:
         line = run_starkv(args, w, rank, world, local)
     if line is not None:

@@ -75,3 +75,29 @@ def test_packed_staging_buffer_round_trips_every_input():
     for v, s in zip(bench.packed_views(buf.clone(), offs, srcs), srcs):
         assert v.dtype == s.dtype and v.shape == s.shape and v.is_contiguous()
         assert torch.equal(v, s)
+
+
+def test_stream_schedule_appends_then_decodes_the_grown_context():
+    """Stream step s appends position L0 + s through the block table and then
+    decodes L0 + s + 1 tokens, so every decode includes the token just added."""
+    import numpy as np
+    L0 = np.array([37, 100], np.int32)
+    n = 20
+    bt, _ = gen.make_block_table(L0 + n, seed=3)
+    slots, lens = bench.stream_schedule(L0, n, bt)
+    assert slots.shape == (n, 2) and slots.dtype == np.int64
+    assert lens.shape == (n, 2) and lens.dtype == np.int32
+    for s in range(n):
+        for b in range(2):
+            pos = int(L0[b]) + s
+            assert slots[s, b] == bt[b, pos // 16] * 16 + pos % 16
+            assert lens[s, b] == pos + 1
+    # distinct physical slots, all inside the sequence's own pages
+    for b in range(2):
+        assert len(set(slots[:, b].tolist())) == n
+        assert set((slots[:, b] // 16).tolist()) <= set(bt[b][bt[b] >= 0].tolist())
+
+
+def test_stream_workload_dispatches_to_the_stream_leg():
+    w = gen.workload("longchat7b_stream_b1_t32768_s128")
+    assert w.steps == 128 and w.chunk == 0 and w.batch == 1 and w.ctx == 32768

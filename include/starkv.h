@@ -90,8 +90,11 @@ typedef struct CUstream_st* starkv_stream_t;
  *   group is g = gcd(16, n_top, r - n_top) channels, so no group straddles the
  *   two precision blocks; g must be 4, 8 or 16.
  * Supported: head_dim in {64, 128}; num_q_heads % num_kv_heads == 0;
- *   rank_k <= head_dim, rank_k % 16 == 0; rank_v <= num_kv_heads*head_dim,
- *   rank_v % 16 == 0; hidden % 64 == 0; rope_base > 1; max_position >= 1. */
+ *   num_q_heads, num_kv_heads <= 1024; rank_k <= head_dim, rank_k <= 64,
+ *   rank_k % 16 == 0; rank_v <= num_kv_heads*head_dim, rank_v <= 1024,
+ *   rank_v % 16 == 0; hidden % 64 == 0, hidden <= 65536; rope_base > 1;
+ *   1 <= max_position <= 2^24 (the context holds max_position * head_dim * 6
+ *   bytes of RoPE tables on the device and, while it is created, on the host). */
 typedef struct starkv_config {
   int32_t num_q_heads;  /* H                                            */
   int32_t num_kv_heads; /* h_kv                                         */

@@ -17,6 +17,10 @@ namespace {
 
 thread_local char g_err[512] = "";
 
+// Bounds that keep every size product of the checks and launches in range.
+constexpr int kMaxHeads = 1024;
+constexpr int kMaxHidden = 1 << 16;
+
 starkv_status fail(starkv_status code, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -67,6 +71,9 @@ starkv_status check_config(const starkv_config* c, LatentGeom* key, LatentGeom* 
       c->rank_k <= 0 || c->rank_v <= 0 || c->max_position <= 0)
     return fail(STARKV_ERR_INVALID_ARG, "config sizes must be positive");
   if (c->flags != 0) return fail(STARKV_ERR_INVALID_ARG, "config.flags must be 0");
+  if (c->num_q_heads > kMaxHeads || c->num_kv_heads > kMaxHeads || c->hidden > kMaxHidden)
+    return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "num_q_heads, num_kv_heads <= %d and hidden <= %d", kMaxHeads,
+                kMaxHidden);
   if (!(c->top_fraction >= 0.0 && c->top_fraction <= 1.0))
     return fail(STARKV_ERR_INVALID_ARG, "top_fraction must lie in [0, 1]");
   if (!(c->rope_base > 1.0)) return fail(STARKV_ERR_INVALID_ARG, "rope_base must exceed 1");
@@ -237,9 +244,18 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
   if (e == cudaSuccess) e = cudaMemsetAsync(c->status, 0, sizeof(unsigned int), s);
   // RoPE table: angle p * base^(-2i/d) in fp64, cos/sin in fp64, stored as fp32
   // and the same angles as an fp16 [cos.. | sin..] row per position (tensor-core operand)
-  std::vector<float2> rope((size_t)cfg->max_position * half);
-  std::vector<__half> trig((size_t)cfg->max_position * d);
-  std::vector<double> theta(half);
+  std::vector<float2> rope;
+  std::vector<__half> trig;
+  std::vector<double> theta;
+  try {
+    rope.resize((size_t)cfg->max_position * half);
+    trig.resize((size_t)cfg->max_position * d);
+    theta.resize(half);
+  } catch (const std::bad_alloc&) {
+    if (e == cudaSuccess) cudaStreamSynchronize(s);
+    cleanup();
+    return fail(STARKV_ERR_CUDA, "out of host memory for the RoPE tables of %d positions", cfg->max_position);
+  }
   for (int i = 0; i < half; ++i) theta[i] = pow(cfg->rope_base, -2.0 * i / d);
   for (int p = 0; p < cfg->max_position; ++p)
     for (int i = 0; i < half; ++i) {

@@ -625,7 +625,8 @@ def run_stream(args, w, rank, world, local):
                 t_(st.slots_np[s]), t_(st.bt_np), t_(st.lens_np[s])]
 
     offs, h2d = pack_layout(host_inputs(0))
-    hbuf = torch.zeros((st.n, h2d), dtype=torch.uint8).pin_memory()
+    pitch = -(-h2d // 256) * 256  # rows start aligned for every view's dtype
+    hbuf = torch.zeros((st.n, pitch), dtype=torch.uint8).pin_memory()
     for s in range(st.n):
         srcs = host_inputs(s)
         for v, x in zip(packed_views(hbuf[s], offs, srcs), srcs):
@@ -636,7 +637,7 @@ def run_stream(args, w, rank, world, local):
     d2h = outh.numel() * outh.element_size()
 
     def e2e_step(i):
-        dbuf.copy_(hbuf[i % st.n], non_blocking=True)
+        dbuf.copy_(hbuf[i % st.n, :h2d], non_blocking=True)
         c = st.caches[i % len(st.caches)]
         S.starkv_append(st.kv.ctx, c.struct, Xd, sld)
         S.starkv_decode_attn(st.kv.ctx, c.struct, qd, btd, ld, st.out, st.ws)

@@ -1,0 +1,176 @@
+"""bench.py's decode and stream legs run end to end on the CPU against
+stand-ins for CUDA (events, streams, pinned memory) and for the library's
+device entry points.
+
+The stand-ins check what reaches the C ABI: the argument count and the pointer
+types of every call, and, for the stream leg, that step i of a run appends and
+decodes stream step i mod n: its hidden states, slots, query and lengths.
+Layout queries go to the real library (host-only).  Nothing here measures
+anything; it guards the bench's plumbing.
+"""
+import contextlib
+import ctypes
+import io
+import json
+import time
+
+import pytest
+import torch
+
+import bench
+from harness import gen
+from rank_mixed_precision_b200 import starkv as S
+
+
+class _Event:
+    def __init__(self, enable_timing=False):
+        self.t = None
+
+    def record(self, *a):
+        self.t = time.perf_counter()
+
+    def elapsed_time(self, other):
+        return max(1e-6, (other.t - self.t) * 1e3)
+
+
+class _Stream:
+    cuda_stream = 0
+
+
+class _Lib:
+    """Device entry points recorded; everything else goes to the real library."""
+
+    def __init__(self, real, log):
+        self.real, self.log = real, log
+
+    def __getattr__(self, name):
+        return getattr(self.real, name)
+
+    def starkv_append(self, *a):
+        assert len(a) == 7
+        _, _, x, sl, n, lat, _ = a
+        assert isinstance(x, ctypes.c_void_p) and x.value and isinstance(sl, ctypes.c_void_p) and sl.value
+        assert int(n) >= 1 and lat is None
+        self.log.append(("append", x.value, sl.value))
+        return 0
+
+    def starkv_decode_attn(self, *a):
+        assert len(a) == 11
+        _, _, q, bt, ln, B, mp, out, ws, wsb, _ = a
+        assert all(isinstance(p, ctypes.c_void_p) and p.value for p in (q, bt, ln, out, ws))
+        assert int(B) >= 1 and int(mp) >= 1 and int(wsb) > 0
+        self.log.append(("decode", q.value, ln.value))
+        return 0
+
+    def starkv_last_error(self):
+        return b""
+
+
+class _KV:
+    """StarKV without a device: caches in host memory, fills recorded."""
+
+    def __init__(self, log):
+        self.log = log
+
+    def __call__(self, cfg, *factors, stream=None):
+        self.cfg, self.ctx = cfg, ctypes.c_void_p(1)
+        return self
+
+    def new_cache(self, n_pages):
+        return S.LatentCache(self.cfg, n_pages, device="cpu")
+
+    def append(self, cache, X, slots):
+        assert X.dtype == torch.bfloat16 and X.dim() == 2 and X.is_contiguous()
+        assert slots.dtype == torch.int64 and slots.shape == (X.shape[0],)
+        assert 0 <= int(slots.min()) and int(slots.max()) < cache.n_pages * 16
+        self.log.append(("fill", X.shape[0], slots.tolist()))
+
+    def workspace(self, op, batch, max_pages):
+        return torch.zeros(1 << 12, dtype=torch.uint8)
+
+    def status(self):
+        return 0
+
+
+def _need_host(t, dtype, name, ndim=None):
+    assert isinstance(t, torch.Tensor) and t.dtype == dtype and t.is_contiguous(), name
+    assert ndim is None or t.dim() == ndim, name
+
+
+@pytest.fixture
+def dry(monkeypatch):
+    log = []
+    real_device = torch.device
+    monkeypatch.setattr(torch.cuda, "Event", _Event)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "set_device", lambda *a: None)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a: _Stream())
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+    monkeypatch.setattr(torch, "device", lambda *a, **k: real_device("cpu"))
+    lib = _Lib(S.lib(), log)
+    monkeypatch.setattr(S, "lib", lambda: lib)
+    monkeypatch.setattr(S, "StarKV", _KV(log))
+    monkeypatch.setattr(S, "_need", _need_host)
+    small = {
+        "dry_stream": gen.shrink(gen.workload("longchat7b_stream_b1_t32768_s128"), name="dry_stream", H=4, h_kv=4,
+                                 d_h=64, hidden=256, r_k=16, R=64, batch=2, ctx=70, steps=9),
+        "dry_decode": gen.shrink(gen.workload("longchat7b_decode_b16_t4096"), name="dry_decode", H=4, h_kv=4,
+                                 d_h=64, hidden=256, r_k=16, R=64, batch=3, ctx=50),
+    }
+    monkeypatch.setattr(gen, "WORKLOADS", {**gen.WORKLOADS, **small})
+    states = []
+    init = bench.StreamState.__init__
+
+    def recording_init(self, *a, **k):
+        init(self, *a, **k)
+        states.append(self)
+
+    monkeypatch.setattr(bench.StreamState, "__init__", recording_init)
+    return log, states
+
+
+def _run(argv):
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.main(argv)
+    return json.loads(buf.getvalue().strip().splitlines()[-1])
+
+
+def test_stream_leg_walks_the_stream_in_order(dry):
+    log, states = dry
+    steps, warm = 25, 3
+    line = _run(["--workload", "dry_stream", "--steps", str(steps), "--warmup", str(warm), "--no-cpu-baseline"])
+    st = states[-1]
+    n, L0 = st.n, st.L0
+    # every replica source: context [0, L0) in chunks, then each stream token alone, in order
+    fills = [e for e in log if e[0] == "fill"]
+    assert sum(e[1] for e in fills) == int(L0.sum()) + n * len(L0)
+    assert [e[2] for e in fills[-n:]] == [st.slots_np[s].tolist() for s in range(n)]
+    apps = [e for e in log if e[0] == "append"]
+    decs = [e for e in log if e[0] == "decode"]
+    assert len(apps) == len(decs) == 2 * (warm + steps)   # device-resident leg, then end to end
+    for i in range(steps):
+        s = i % n
+        assert apps[warm + i][1:] == (st.X[s].data_ptr(), st.slots[s].data_ptr())
+        assert decs[warm + i][1:] == (st.q[s].data_ptr(), st.lens[s].data_ptr())
+    for s in range(n):
+        for b in range(len(L0)):
+            pos = int(L0[b]) + s
+            assert st.lens_np[s, b] == pos + 1
+            assert st.slots_np[s, b] == st.bt_np[b, pos // 16] * 16 + pos % 16
+    assert line["steps"] == steps and line["warmup"] == warm
+    assert line["config"]["ctx"] == f"{int(L0.max())} -> {int(L0.max()) + n}"
+    assert line["e2e"]["h2d_bytes_per_step"] > 0 and line["e2e"]["d2h_bytes_per_step"] == 2 * 4 * 64 * 2
+    assert line["gpu_launches"] == 6 * steps and line["roofline"]["traffic"] is None
+
+
+def test_decode_leg_line_has_the_contract_keys(dry):
+    log, _ = dry
+    line = _run(["--workload", "dry_decode", "--steps", "7", "--warmup", "3", "--no-cpu-baseline"])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert k in line, k
+    for k in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert k in line["roofline"], k
+    assert line["config"]["workload"] == "dry_decode" and line["n_gpus"] == 1
+    assert sum(1 for e in log if e[0] == "decode") == 2 * (3 + 7)

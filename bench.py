@@ -425,6 +425,41 @@ def prefill_flops(w) -> dict:
     return {k: v * w.batch for k, v in per.items()}
 
 
+def prefill_launches_per_step(max_pages: int, n_append: int) -> int:
+    """Kernels one prefill step launches: the append (the general kernel above
+    64 tokens, else the split-K projection and the quantiser) and the prefill
+    (init, then expand + attention per key chunk of up to 512 positions, finalize)."""
+    max_len = max_pages * 16
+    chunk = 512 if max_len >= 512 else max(32, -(-max_len // 32) * 32)
+    return (1 if n_append > 64 else 2) + 2 + 2 * (-(-max_len // chunk))
+
+
+def prefill_sample_flops(w, n_q: int, L: int) -> float:
+    """Algorithmic flops of n_q queries at positions L - n_q .. L - 1 of one
+    sequence: their causal attention pairs, plus their share (n_q of the chunk's
+    queries) of one sequence's key/value re-expansion and projection."""
+    fl = prefill_flops(w)
+    pairs = sum(L - n_q + i + 1 for i in range(n_q))
+    rest = (fl["value_reexpansion"] + fl["key_reexpansion"] + fl["projection"]) / w.batch
+    return pairs * w.H * 4 * w.d_h + rest * n_q / w.chunk
+
+
+def cpu_baseline_prefill(w, seed, seconds, n_q=4):
+    O, oc, bt, L, f, _ = _oracle_setup(w, seed, 0)
+    q = gen.make_queries(n_q, w.H, w.d_h, seed, name="q_chunk")
+    done, t0 = 0, time.perf_counter()
+    while True:
+        O.prefill(oc, q, [0, n_q], f.B_k, f.B_v, bt, [L])
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": done * prefill_sample_flops(w, n_q, L) / el / 1e12, "unit": "TFLOP/s",
+            "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{done} oracle prefill call(s) of {n_q} queries at the end of one {L}-token sequence, "
+                      f"all {w.H} heads, fp64 numpy, {el:.1f} s", "host_cpu_count": os.cpu_count()}
+
+
 def run_prefill(args, w, rank, world, local):
     import torch
     torch.cuda.set_device(local)
@@ -451,6 +486,37 @@ def run_prefill(args, w, rank, world, local):
     total = sum(fl.values())
     value, ms_max = job_throughput(total * args.steps / 1e12, t0.elapsed_time(t1), world, device)
     attn_ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+    # ---- end to end through the public API with host buffers: the step's
+    # inputs packed in one pinned staging buffer, one copy each way
+    srcs = [st.X.cpu(), st.slots.cpu(), st.q.cpu(), st.cu_q.cpu(), st.bt.cpu(), st.sl.cpu()]
+    offs, h2d = pack_layout(srcs)
+    hbuf = torch.zeros(h2d, dtype=torch.uint8).pin_memory()
+    for v, x in zip(packed_views(hbuf, offs, srcs), srcs):
+        v.copy_(x)
+    dbuf = torch.empty(h2d, dtype=torch.uint8, device=device)
+    Xd, sld, qd, cud, btd, lnd = packed_views(dbuf, offs, srcs)
+    outh = torch.empty(st.out.shape, dtype=torch.bfloat16).pin_memory()
+    d2h = outh.numel() * outh.element_size()
+    S = st.S
+
+    def e2e_step():
+        dbuf.copy_(hbuf, non_blocking=True)
+        S.starkv_append(st.kv.ctx, st.cache.struct, Xd, sld)
+        S.starkv_prefill_attn(st.kv.ctx, st.cache.struct, qd, cud, btd, lnd, w.chunk, st.out, st.ws)
+        outh.copy_(st.out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_value, _ = job_throughput(total * args.steps / 1e12, e0.elapsed_time(e1), world, device)
     if rank != 0:
         return None
     peaks = {}
@@ -460,18 +526,24 @@ def run_prefill(args, w, rank, world, local):
         pass
     peak = float(peaks.get("bf16_tflops", 1590.0))
     achieved = (total - fl["projection"]) / (attn_ms / 1e3) / 1e12
-    return {
+    line = {
         "metric": "prefill TFLOP/s (algorithmic)", "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32 (CUDA-core prefill)", "data": "synthetic (seeded)",
         "config": {"workload": w.name, "batch": w.batch, "ctx": w.ctx, "chunk": w.chunk,
-                   "step": "append the chunk + causal prefill attention of its queries"},
+                   "step": "append the chunk + causal prefill attention of its queries",
+                   "l2": f"cache {st.cache.nbytes() / 2**20:.0f} MiB read per step (vs 126 MiB L2)"},
         "flops_per_step": fl,
         "roofline": {"bound": "tensor", "kernel": "starkv_prefill_attn (expand + attention kernels)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "traffic": None, "launch_ms": attn_ms},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": prefill_launches_per_step(int(st.bt.shape[1]), w.batch * w.chunk) * args.steps,
         "clocks": clk.summary(),
     }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_prefill(w, args.seed, args.cpu_seconds)
+    return line
 
 
 def run_starkv(args, w, rank, world, local):
@@ -744,6 +816,8 @@ def run_reference(args, w, rank, world):
     stays within a few minutes."""
     if rank != 0:
         return None
+    if w.chunk > 0:
+        return _run_reference_prefill(args, w, world)
     O, oc, bt, L, f, q = _oracle_setup(w, args.seed, 0)
     t0 = time.perf_counter()
     O.decode(oc, q, f.B_k, f.B_v, bt, [L])
@@ -768,6 +842,37 @@ def run_reference(args, w, rank, world):
         "cpu_baseline": {"value": v, "unit": "context-tokens/s", "cores": _blas_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": v, "unit": "context-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def _run_reference_prefill(args, w, world, n_q=4):
+    """Prefill workloads: each step is n_q queries at the end of one sequence,
+    on a subset of the heads sized so the run stays within a few minutes;
+    flops are the sample's algorithmic share, scaled by the heads taken."""
+    O, oc, bt, L, f, _ = _oracle_setup(w, args.seed, 0)
+    q = gen.make_queries(n_q, w.H, w.d_h, args.seed, name="q_chunk")
+    t0 = time.perf_counter()
+    O.prefill(oc, q, [0, n_q], f.B_k, f.B_v, bt, [L])
+    t_full = time.perf_counter() - t0
+    heads = max(1, min(w.H, int(w.H * 150.0 / max(1e-9, args.steps * t_full))))
+    hs = list(range(heads))
+    for _ in range(min(args.warmup, 1)):
+        O.prefill(oc, q, [0, n_q], f.B_k, f.B_v, bt, [L], heads=hs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.prefill(oc, q, [0, n_q], f.B_k, f.B_v, bt, [L], heads=hs)
+    el = time.perf_counter() - t0
+    v = args.steps * prefill_sample_flops(w, n_q, L) * (heads / w.H) / el / 1e12
+    sample = (f"each step: {n_q} queries at the end of one {L}-token sequence, {heads} of {w.H} heads "
+              f"(counted as {heads}/{w.H} of their algorithmic flops)")
+    return {
+        "metric": "prefill TFLOP/s (algorithmic)", "value": v, "unit": "TFLOP/s", "impl": "reference",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "batch": w.batch, "ctx": w.ctx, "chunk": w.chunk, "sample": sample},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 

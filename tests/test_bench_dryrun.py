@@ -1,4 +1,4 @@
-"""bench.py's decode and stream legs run end to end on the CPU against
+"""bench.py's decode, stream and prefill legs run end to end on the CPU against
 stand-ins for CUDA (events, streams, pinned memory) and for the library's
 device entry points.
 
@@ -62,6 +62,14 @@ class _Lib:
         self.log.append(("decode", q.value, ln.value))
         return 0
 
+    def starkv_prefill_attn(self, *a):
+        assert len(a) == 14
+        _, _, q, cu, bt, ln, B, mp, tq, mq, out, ws, wsb, _ = a
+        assert all(isinstance(p, ctypes.c_void_p) and p.value for p in (q, cu, bt, ln, out, ws))
+        assert int(B) >= 1 and int(mp) >= 1 and int(tq) >= int(B) and 1 <= int(mq) <= int(mp) * 16 and int(wsb) > 0
+        self.log.append(("prefill", q.value, int(tq), int(mq)))
+        return 0
+
     def starkv_last_error(self):
         return b""
 
@@ -85,7 +93,7 @@ class _KV:
         assert 0 <= int(slots.min()) and int(slots.max()) < cache.n_pages * 16
         self.log.append(("fill", X.shape[0], slots.tolist()))
 
-    def workspace(self, op, batch, max_pages):
+    def workspace(self, op, batch, max_pages, total_q=0):
         return torch.zeros(1 << 12, dtype=torch.uint8)
 
     def status(self):
@@ -116,6 +124,8 @@ def dry(monkeypatch):
                                  d_h=64, hidden=256, r_k=16, R=64, batch=2, ctx=70, steps=9),
         "dry_decode": gen.shrink(gen.workload("longchat7b_decode_b16_t4096"), name="dry_decode", H=4, h_kv=4,
                                  d_h=64, hidden=256, r_k=16, R=64, batch=3, ctx=50),
+        "dry_prefill": gen.shrink(gen.workload("longchat7b_prefill_b4_t30720_c2048"), name="dry_prefill", H=4,
+                                  h_kv=4, d_h=64, hidden=256, r_k=16, R=64, batch=2, ctx=40, chunk=24),
     }
     monkeypatch.setattr(gen, "WORKLOADS", {**gen.WORKLOADS, **small})
     states = []
@@ -174,3 +184,29 @@ def test_decode_leg_line_has_the_contract_keys(dry):
         assert k in line["roofline"], k
     assert line["config"]["workload"] == "dry_decode" and line["n_gpus"] == 1
     assert sum(1 for e in log if e[0] == "decode") == 2 * (3 + 7)
+
+
+def test_prefill_leg_line_counts_its_launches_and_copies(dry):
+    log, _ = dry
+    steps, warm = 4, 3
+    line = _run(["--workload", "dry_prefill", "--steps", str(steps), "--warmup", str(warm), "--no-cpu-baseline"])
+    pre = [e for e in log if e[0] == "prefill"]
+    assert len(pre) == 2 * (warm + steps)                  # device-resident leg, then end to end
+    assert all(e[2] == 2 * 24 and e[3] == 24 for e in pre)
+    # 64 positions in 4 pages: one key chunk; 48 appended tokens take the split-K append (2 kernels)
+    assert line["gpu_launches"] == (2 + 2 + 2) * steps
+    assert line["e2e"]["unit"] == "TFLOP/s" and line["e2e"]["d2h_bytes_per_step"] == 48 * 4 * 64 * 2
+    assert line["e2e"]["h2d_bytes_per_step"] >= 48 * 256 * 2 + 48 * 8 + 48 * 4 * 64 * 2
+
+
+def test_prefill_reference_arm_reports_the_prefill_metric():
+    w = gen.shrink(gen.workload("longchat7b_prefill_b4_t30720_c2048"), H=4, h_kv=4, d_h=64, hidden=256, r_k=16,
+                   R=64, batch=2, ctx=40, chunk=24)
+
+    class A:
+        seed, steps, warmup = 0, 2, 1
+
+    line = bench._run_reference_prefill(A, w, 1)
+    assert line["metric"] == "prefill TFLOP/s (algorithmic)" and line["unit"] == "TFLOP/s"
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["value"] == line["value"] and line["e2e"]["h2d_bytes_per_step"] == 0

@@ -5,17 +5,23 @@ device entry points.
 The stand-ins check what reaches the C ABI: the argument count and the pointer
 types of every call, and, for the stream leg, that step i of a run appends and
 decodes stream step i mod n: its hidden states, slots, query and lengths.
-Layout queries go to the real library (host-only).  Nothing here measures
-anything; it guards the bench's plumbing.
+Layout queries go to the real library (host-only).  The same legs also run
+as two gloo ranks (the bench's N > 1 path with gloo in place of NCCL): each rank
+runs its own batch, rank 0 alone prints, and the job rate is the tokens of all
+ranks over the slowest rank's time.  Nothing here measures anything; it guards
+the bench's plumbing.
 """
 import contextlib
 import ctypes
 import io
 import json
+import os
+import socket
 import time
 
 import pytest
 import torch
+import torch.multiprocessing as mp
 
 import bench
 from harness import gen
@@ -105,8 +111,8 @@ def _need_host(t, dtype, name, ndim=None):
     assert ndim is None or t.dim() == ndim, name
 
 
-@pytest.fixture
-def dry(monkeypatch):
+def _install(monkeypatch):
+    """Stand-ins for CUDA and the device entry points, plus small workloads."""
     log = []
     real_device = torch.device
     monkeypatch.setattr(torch.cuda, "Event", _Event)
@@ -137,6 +143,11 @@ def dry(monkeypatch):
 
     monkeypatch.setattr(bench.StreamState, "__init__", recording_init)
     return log, states
+
+
+@pytest.fixture
+def dry(monkeypatch):
+    return _install(monkeypatch)
 
 
 def _run(argv):
@@ -210,3 +221,54 @@ def test_prefill_reference_arm_reports_the_prefill_metric():
     assert line["metric"] == "prefill TFLOP/s (algorithmic)" and line["unit"] == "TFLOP/s"
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["cpu_baseline"]["value"] == line["value"] and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _rank_worker(rank, world, port, workload, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    patch = pytest.MonkeyPatch()
+    try:
+        log, _ = _install(patch)
+        init = bench.init_dist
+        patch.setattr(bench, "init_dist", lambda world, backend: init(world, "gloo"))
+        buf = io.StringIO()
+        with contextlib.redirect_stdout(buf):
+            bench.main(["--workload", workload, "--steps", "6", "--warmup", "3", "--no-cpu-baseline",
+                        "--gpus", str(world)])
+        q.put((rank, buf.getvalue(), sum(1 for e in log if e[0] == "decode")))
+    except Exception as e:  # reported to the parent, which fails the test
+        q.put((rank, "error", repr(e)))
+    finally:
+        patch.undo()
+
+
+@pytest.mark.parametrize("workload", ["dry_decode", "dry_stream"])
+def test_two_gloo_ranks_run_the_bench_and_rank0_prints_the_job_line(workload):
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    procs = [ctx.Process(target=_rank_worker, args=(r, world, port, workload, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(world):
+        item = q.get(timeout=180)
+        res[item[0]] = item
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in range(world):
+        assert res[r][1] != "error", res[r]
+        assert res[r][2] == 2 * (3 + 6)             # every rank runs its own batch: no work is skipped
+    assert res[1][1].strip() == ""                   # only rank 0 prints
+    line = json.loads(res[0][1].strip().splitlines()[-1])
+    assert line["n_gpus"] == 2 and line["scaling"] == "weak" and line["steps"] == 6
+    w = gen.shrink(gen.workload("longchat7b_decode_b16_t4096"), H=4, h_kv=4, d_h=64, hidden=256, r_k=16, R=64,
+                   batch=3, ctx=50) if workload == "dry_decode" else None
+    if w is not None:
+        # whole-job rate: tokens of both ranks over the slowest rank's time
+        tokens = 2 * 6 * int(gen.make_seq_lens(w).sum())
+        assert line["value"] == pytest.approx(tokens / (line["ms_per_step"] * 6 / 1e3), rel=1e-9)

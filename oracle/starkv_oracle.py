@@ -8,7 +8,7 @@ Notation: fl32 / fl16 = IEEE round-to-nearest-even to binary32 / binary16.
 numpy float32 arithmetic rounds every +, -, *, / once, so a float32 numpy
 expression *is* the fl32 of each step.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * channel split: the first ``round(top_fraction * r)`` channels of a latent
   (singular-value order) are the 4-bit outlier block, the rest the 3-bit

@@ -822,8 +822,8 @@ def run_reference(args, w, rank, world):
     t0 = time.perf_counter()
     O.decode(oc, q, f.B_k, f.B_v, bt, [L])
     t_full = time.perf_counter() - t0
-    budget = 150.0
-    heads = max(1, min(w.H, int(w.H * budget / max(1e-9, args.steps * t_full))))
+    cap_s = 150.0  # host seconds the timed oracle steps may take
+    heads = max(1, min(w.H, int(w.H * cap_s / max(1e-9, args.steps * t_full))))
     hs = list(range(heads))
     for _ in range(min(args.warmup, 1)):
         O.decode(oc, q, f.B_k, f.B_v, bt, [L], heads=hs)

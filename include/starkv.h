@@ -58,7 +58,7 @@ typedef int32_t starkv_status;
 enum {
   STARKV_OK = 0,
   STARKV_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad enum   */
-  STARKV_ERR_UNSUPPORTED_SHAPE = 2,  /* a configuration this build cannot run   */
+  STARKV_ERR_UNSUPPORTED_SHAPE = 2,  /* a configuration the library cannot run */
   STARKV_ERR_WORKSPACE_TOO_SMALL = 3,/* workspace_bytes below the required size */
   STARKV_ERR_CUDA = 4,               /* a CUDA runtime call failed               */
   STARKV_ERR_DEVICE_STATUS = 5       /* the device status word is non-zero       */

@@ -208,6 +208,41 @@ def merge_k(weight_l=True):
     return lse_merge
 
 
+def project_k(fp32_accumulate=False, keep_fp64=False):
+    def project(X, A):
+        if fp32_accumulate:
+            X32, A32 = np.asarray(X, np.float32), np.asarray(A, np.float32)
+            out = np.zeros((X32.shape[0], A32.shape[1]), np.float32)
+            for k in range(X32.shape[1]):
+                out += X32[:, k:k + 1] * A32[k:k + 1, :]
+            return out
+        prod = np.asarray(X, np.float64) @ np.asarray(A, np.float64)
+        return prod if keep_fp64 else prod.astype(np.float32)
+    return project
+
+
+def prefill_k(shift=0):
+    def prefill(cache, q, cu_q, B_k, B_v, block_table, seq_lens, select=None, heads=None):
+        cfg = cache.cfg
+        q = np.asarray(q)
+        out = np.full((q.shape[0], cfg.H, cfg.d_h), np.nan)
+        heads = list(range(cfg.H)) if heads is None else list(heads)
+        for b in range(len(cu_q) - 1):
+            nb = int(cu_q[b + 1] - cu_q[b])
+            if nb == 0 or (select is not None and b not in select):
+                continue
+            idx = np.arange(nb) if select is None else np.asarray(select[b], np.int64)
+            if idx.size == 0:
+                continue
+            n = int(seq_lens[b])
+            zk, zv = OM.gather_sequence(cache, block_table[b], n)
+            zk, zv = OM.unrotate_fp64(zk, cfg.key.g), OM.unrotate_fp64(zv, cfg.val.g)
+            rows = int(cu_q[b]) + idx
+            out[np.ix_(rows, heads)] = OM.attend_latents(cfg, zk, zv, q[rows], n - nb + idx + shift, B_k, B_v, heads)
+        return out
+    return prefill
+
+
 def eq14_k(swap=False):
     def eq14_mean_bits(top_fraction, top_bits=4, bottom_bits=3):
         if swap:
@@ -245,6 +280,8 @@ PINS = {
                        lambda: TA.test_decode_through_paged_cache_equals_direct()],
     "partial_softmax": [lambda: TA.test_partition_identity_merge()],
     "lse_merge": [lambda: TA.test_partition_identity_merge()],
+    "project": [lambda: TQ.test_projection_is_the_correctly_rounded_product()],
+    "prefill": [lambda: TA.test_prefill_is_causal_decode_per_query()],
     "eq14_mean_bits": [lambda: TB.test_eq14_printed_values()],
     "eq16_retained_fraction": [lambda: TB.test_eq16_printed_values()],
 }
@@ -254,7 +291,7 @@ FAITHFUL = {
     "unrotate_fp64": unrotate_k(), "quantize_groups": quantize_k(), "dequantize_codes": dequantize_k(),
     "pack_region": pack_k(), "write_latents": write_k(), "gather_sequence": gather_k(),
     "attend_latents": attend_k(), "partial_softmax": partial_k(), "lse_merge": merge_k(),
-    "eq14_mean_bits": eq14_k(), "eq16_retained_fraction": eq16_k(),
+    "eq14_mean_bits": eq14_k(), "eq16_retained_fraction": eq16_k(), "project": project_k(), "prefill": prefill_k(),
 }
 
 PLANTS = {
@@ -283,6 +320,9 @@ PLANTS = {
     "query position one past seq_len - 1": ("attend_latents", attend_k(qshift=1)),
     "split partial sums values without weights": ("partial_softmax", partial_k(unweighted_acc=True)),
     "split merge leaves l unweighted": ("lse_merge", merge_k(weight_l=False)),
+    "projection accumulated in fp32": ("project", project_k(fp32_accumulate=True)),
+    "projection left in fp64": ("project", project_k(keep_fp64=True)),
+    "prefill queries one position late": ("prefill", prefill_k(shift=1)),
     "eq. 14 bit widths swapped": ("eq14_mean_bits", eq14_k(swap=True)),
     "eq. 16 drops the exempt layers": ("eq16_retained_fraction", eq16_k(drop_exempt=True)),
 }

@@ -186,3 +186,21 @@ def test_write_latents_partial_pages_keep_other_rows():
 def test_quant_error_raises_on_fp16_overflow():
     with pytest.raises(O.QuantError):
         O.quantize_groups(np.array([[0.0, 1e6, 0.0, 0.0]], np.float32), 4)
+
+
+def test_projection_is_the_correctly_rounded_product():
+    # pre-quantisation latent = fl32 of the exact product X A ([Review] section 2.2, eq. 2;
+    # the rounding is a reading of the pages).  Cases whose fp64 sums are exact:
+    # integers (exact in fp32 as well), a cancellation that fp32 accumulation loses,
+    # and a sum just above a rounding tie that fp32 accumulation rounds down.
+    rng = np.random.default_rng(9)
+    X = rng.integers(-8, 9, (5, 64)).astype(np.float64)
+    A = rng.integers(-8, 9, (64, 7)).astype(np.float64)
+    exact = [[sum(int(X[i, k]) * int(A[k, j]) for k in range(64)) for j in range(7)] for i in range(5)]
+    got = O.project(X, A)
+    assert got.dtype == np.float32
+    np.testing.assert_array_equal(got, np.array(exact, np.float32))
+    X2 = np.array([[1.0, 2.0 ** -30, -1.0], [1.0, 2.0 ** -24, 2.0 ** -26]])
+    got2 = O.project(X2, np.ones((3, 1)))
+    assert got2[0, 0] == np.float32(2.0 ** -30)
+    assert got2[1, 0] == np.float32(1.0 + 2.0 ** -23)

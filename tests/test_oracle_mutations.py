@@ -94,13 +94,34 @@ def quantize_k(levels_pow2=False, rounding="rint", zero="min"):
     return quantize_groups
 
 
-def dequantize_k(zp_sign=1.0):
+def dequantize_k(zp_sign=1.0, half_step=False):
     def dequantize_codes(codes, s, zp, lat):
         n = codes.shape[0]
         c = codes.reshape(n, lat.n_groups, lat.g).astype(np.float32)
+        if half_step:
+            c = c + np.float32(0.5)
         zh = c * s.astype(np.float32)[..., None] + np.float32(zp_sign) * zp.astype(np.float32)[..., None]
         return zh.reshape(n, lat.r)
     return dequantize_codes
+
+
+def quantize_latent_k(all_bits=None, top_shift=0):
+    def quantize_latent(z, lat):
+        z = np.asarray(z, np.float32)
+        n = z.shape[0]
+        zr = OM.rotate_fl32(z, lat.g).reshape(n, lat.n_groups, lat.g)
+        codes = np.empty((n, lat.n_groups, lat.g), np.uint8)
+        s = np.empty((n, lat.n_groups), np.float16)
+        zp = np.empty((n, lat.n_groups), np.float16)
+        t = min(max(lat.n_top_groups + top_shift, 0), lat.n_groups)
+        if all_bits is not None:
+            t = lat.n_groups if all_bits == 4 else 0
+        if t:
+            codes[:, :t], s[:, :t], zp[:, :t] = OM.quantize_groups(zr[:, :t], 4)
+        if t < lat.n_groups:
+            codes[:, t:], s[:, t:], zp[:, t:] = OM.quantize_groups(zr[:, t:], 3)
+        return codes.reshape(n, lat.r), s, zp
+    return quantize_latent
 
 
 def pack_k(hi_first=False, planes_swapped=False, meta_swapped=False):
@@ -271,7 +292,12 @@ PINS = {
     "quantize_groups": [lambda: TQ.test_grid_values_round_trip(4),
                         lambda: TQ.test_codes_are_nearest_grid_point_bruteforce(3),
                         lambda: TQ.test_quantisation_error_bound(4)],
-    "dequantize_codes": [lambda: TA.test_quantised_attention_close_to_unquantised()],
+    "dequantize_codes": [lambda: TA.test_quantised_attention_close_to_unquantised(),
+                         lambda: TQ.test_grid_values_round_trip(4),
+                         lambda: TQ.test_constant_group_has_zero_scale()],
+    "quantize_latent": [lambda: TQ.test_quantize_latent_bit_width_per_group(64),
+                        lambda: TQ.test_quantize_latent_bit_width_per_group(32),
+                        lambda: TQ.test_quantize_latent_scale_per_group_on_hand_built_input()],
     "pack_region": [lambda: TQ.test_pack_matches_hand_derived_bytes(),
                     lambda: TQ.test_pack_unpack_exhaustive(32, 0.25)],
     "write_latents": [lambda: TQ.test_write_latents_partial_pages_keep_other_rows()],
@@ -289,6 +315,7 @@ PINS = {
 FAITHFUL = {
     "rope": rope_k(), "hadamard_fp64": hadamard_k(), "rotate_fl32": rotate_k(),
     "unrotate_fp64": unrotate_k(), "quantize_groups": quantize_k(), "dequantize_codes": dequantize_k(),
+    "quantize_latent": quantize_latent_k(),
     "pack_region": pack_k(), "write_latents": write_k(), "gather_sequence": gather_k(),
     "attend_latents": attend_k(), "partial_softmax": partial_k(), "lse_merge": merge_k(),
     "eq14_mean_bits": eq14_k(), "eq16_retained_fraction": eq16_k(), "project": project_k(), "prefill": prefill_k(),
@@ -308,6 +335,11 @@ PLANTS = {
     "codes truncated, not rounded": ("quantize_groups", quantize_k(rounding="floor")),
     "zero point at the group maximum": ("quantize_groups", quantize_k(zero="max")),
     "dequant subtracts the zero point": ("dequantize_codes", dequantize_k(zp_sign=-1.0)),
+    "dequant adds half a step": ("dequantize_codes", dequantize_k(half_step=True)),
+    "every group quantised at 3 bits": ("quantize_latent", quantize_latent_k(all_bits=3)),
+    "every group quantised at 4 bits": ("quantize_latent", quantize_latent_k(all_bits=4)),
+    "4-bit block one group too wide": ("quantize_latent", quantize_latent_k(top_shift=1)),
+    "4-bit block one group too narrow": ("quantize_latent", quantize_latent_k(top_shift=-1)),
     "4-bit tile: high nibble first": ("pack_region", pack_k(hi_first=True)),
     "3-bit tile: 1-bit plane before 2-bit plane": ("pack_region", pack_k(planes_swapped=True)),
     "metadata: zero in the low half": ("pack_region", pack_k(meta_swapped=True)),

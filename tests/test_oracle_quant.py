@@ -53,11 +53,16 @@ def test_fwht_within_fp32_bound_of_matrix_product(g):
     assert np.all(np.abs(back - z) <= 2 * bound)
 
 
+def _one_group(bits, g=16):
+    """Geometry of a latent that is a single group of g channels at `bits` bits."""
+    return O.Latent(g, g if bits == 4 else 0, 0 if bits == 4 else g, g)
+
+
 def test_constant_group_has_zero_scale():
     z = np.full((3, 8), 1.2345678, np.float32)
     codes, s, zp = O.quantize_groups(z, 3)
     assert np.all(s == 0) and np.all(codes == 0)
-    zh = codes.astype(np.float32) * s.astype(np.float32)[:, None] + zp.astype(np.float32)[:, None]
+    zh = O.dequantize_codes(codes, s[:, None], zp[:, None], _one_group(3, 8))
     np.testing.assert_array_equal(zh, np.float16(np.float32(1.2345678)).astype(np.float32))
 
 
@@ -76,6 +81,9 @@ def test_grid_values_round_trip(bits):
             continue                             # range not exact in fp32 (rare); skip
         assert s2[0] == s and zp2[0] == zp
         np.testing.assert_array_equal(codes[0], k)
+        # values on the grid come back exactly through the dequantiser: k s + zp
+        back = O.dequantize_codes(codes, s2[:, None], zp2[:, None], _one_group(bits))
+        np.testing.assert_array_equal(back[0], z)
 
 
 @pytest.mark.parametrize("bits", [3, 4])
@@ -204,3 +212,50 @@ def test_projection_is_the_correctly_rounded_product():
     got2 = O.project(X2, np.ones((3, 1)))
     assert got2[0, 0] == np.float32(2.0 ** -30)
     assert got2[1, 0] == np.float32(1.0 + 2.0 ** -23)
+
+
+@pytest.mark.parametrize("r", [16, 32, 64, 512, 1024])
+def test_quantize_latent_bit_width_per_group(r):
+    # [Review] eq. 14 with the card's calibration recipe (top_fraction 0.25,
+    # top_bits 4, bottom_bits 3): the leading 25% of a latent's channels, in
+    # singular-value order, are the 4-bit block and the rest the 3-bit block.
+    # Every group's largest element lands on the top code of its grid, so the
+    # largest code of a group tells its width: 15 for a 4-bit group, 7 for a
+    # 3-bit group.  The mean width over the channels is then eq. 14's 3.25.
+    rng = np.random.default_rng(r)
+    lat = O.latent_split(r, 0.25)
+    z = (rng.standard_normal((64, r)) * rng.uniform(0.5, 4.0, (64, 1))).astype(np.float32)
+    codes, s, zp = O.quantize_latent(z, lat)
+    assert codes.shape == (64, r) and s.shape == (64, r // lat.g)
+    top_channels = r // 4                                  # 25% of the channels, counted by hand
+    width = np.empty(r)
+    for c0 in range(0, r, lat.g):
+        top = codes[:, c0:c0 + lat.g].max(axis=1)
+        want = 15 if c0 < top_channels else 7
+        assert np.all(top == want), (c0, np.unique(top))
+        assert codes[:, c0:c0 + lat.g].min(axis=1).max() == 0
+        width[c0:c0 + lat.g] = 4 if want == 15 else 3
+    assert width.mean() == pytest.approx(O.eq14_mean_bits(0.25))
+    assert width.mean() == pytest.approx(0.25 * 4 + 0.75 * 3)
+
+
+def test_quantize_latent_scale_per_group_on_hand_built_input():
+    # One token, r = 64 (g = 16): after the rotation, group gi spans a known range.
+    # Feed the inverse rotation of a ramp so the rotated values are the ramp
+    # itself (up to fp32 rounding of the butterflies, checked below), then the
+    # scale of a group is fl16(range / 15) for the first 16 channels (4-bit) and
+    # fl16(range / 7) for the other 48 (3-bit).
+    lat = O.latent_split(64, 0.25)
+    assert (lat.g, lat.n_top) == (16, 16)
+    ramp = np.concatenate([np.arange(16, dtype=np.float64) * (gi + 1) * 0.25 - gi for gi in range(4)])
+    z = O.unrotate_fp64(ramp[None], 16).astype(np.float32)      # H_g is its own inverse
+    zr = O.rotate_fl32(z, 16).astype(np.float64)[0]
+    _, s, zp = O.quantize_latent(z, lat)
+    for gi in range(4):
+        seg = zr[16 * gi:16 * gi + 16]
+        qmax = 15 if gi == 0 else 7
+        want = np.float16(np.float32(np.float32(seg.max()) - np.float32(seg.min())) / np.float32(qmax))
+        assert s[0, gi] == want, gi
+        assert zp[0, gi] == np.float16(np.float32(seg.min()))
+        # the range is the ramp's (gi + 1) * 0.25 * 15 to within the rotation's rounding
+        assert abs((seg.max() - seg.min()) - (gi + 1) * 0.25 * 15) < 1e-4

@@ -224,12 +224,17 @@ STARKV_API starkv_status starkv_decode_attn(starkv_ctx* ctx, const starkv_cache*
  * enter the allocator.  The split partials live in a built-in 16 MiB scratch
  * array that every GPU loading this library holds until the process exits;
  * the call itself allocates nothing.  The first call on a device looks up that
- * array's device address (once per device, with the device current); make this
- * first call before any stream capture.  All calls on a device share the
- * scratch, so calls that overlap on the GPU (other streams, other contexts on
- * the same device) race; serialise them.  A shape whose partials exceed the
- * scratch (batch * num_q_heads * splits * (rank_v + 2) * 4 bytes > 16 MiB) is
- * rejected with STARKV_ERR_UNSUPPORTED_SHAPE before anything is launched.
+ * array's device address (once per device, with the device current) and keeps
+ * it for the life of the process; make this first call before any stream
+ * capture, and do not use the library across a cudaDeviceReset of that device.
+ * All calls on a device share the scratch, so calls that overlap on the GPU
+ * (other streams, other contexts on the same device) race; serialise them.
+ * Size limit: the call needs exactly the workspace starkv_decode_attn would
+ * take, so a shape is accepted when
+ *   starkv_workspace_bytes(ctx, STARKV_OP_DECODE, batch, max_pages, 0) <= 16 MiB
+ * (query that call to check a shape; the workspace grows with batch and with
+ * max_pages).  A larger shape is rejected with STARKV_ERR_UNSUPPORTED_SHAPE
+ * before anything is launched.
  * Errors: as starkv_decode_attn, plus UNSUPPORTED_SHAPE for oversize shapes. */
 STARKV_API starkv_status starkv_decode_attn_noalloc(starkv_ctx* ctx, const starkv_cache* cache,
                                                     const void* q, const int32_t* block_table,

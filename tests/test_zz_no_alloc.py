@@ -12,7 +12,8 @@ import torch
 
 from harness import gen
 
-from _cases import ATOL_MAX, REL_L2, bf16_tensor, make_ctx, oracle_cache, skv, upload
+import oracle as O
+from _cases import ATOL_MAX, REL_L2, bf16_tensor, check_attention, make_ctx, oracle_cache, skv, upload
 
 pytestmark = pytest.mark.gpu
 
@@ -31,6 +32,7 @@ def test_noalloc_matches_workspace_decode_twice(wi, lens):
         btd = torch.from_numpy(bt).cuda()
         sl = torch.tensor(np.asarray(lens, np.int32)).cuda()
         ref = kv.decode(lc, q, btd, sl).float()
+        want = O.decode(oc, gen.make_queries(len(lens), w.H, w.d_h), f.B_k, f.B_v, bt, lens)
         for call in range(2):           # the scratch keeps the previous call's contents
             out = torch.full_like(q, float("nan"))
             S.starkv_decode_attn_noalloc(kv.ctx, lc.struct, q, btd, sl, out)
@@ -39,6 +41,7 @@ def test_noalloc_matches_workspace_decode_twice(wi, lens):
             err = (got - ref).abs().max().item()
             rel = (torch.linalg.norm(got - ref) / torch.linalg.norm(ref).clamp_min(1e-30)).item()
             assert err <= ATOL_MAX and rel <= REL_L2, f"call {call}: max-abs {err:.3e} rel-L2 {rel:.3e}"
+            check_attention(got.cpu().numpy(), want, f"call {call} against the oracle")
         assert kv.status() == 0
     finally:
         kv.close()
@@ -58,5 +61,85 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
             S.starkv_decode_attn_noalloc(kv.ctx, lc.struct, q, bt, sl, torch.empty_like(q))
         assert e.value.code == S.ERR_UNSUPPORTED_SHAPE
         assert "scratch" in S.starkv_last_error()
+    finally:
+        kv.close()
+
+
+SCRATCH = 16 << 20
+
+
+def _simt_workspace(batch, H, R, max_pages):
+    """Partials of the CUDA-core decode plan: batch * H * splits * (R + 2) * 4 bytes."""
+    splits = min(-(-4 * 148 // (batch * H)), -(-max_pages // 16))
+    splits = max(splits, 1)
+    pps = max(-(-max_pages // splits), 1)
+    return batch * H * (-(-max_pages // pps)) * (R + 2) * 4
+
+
+def test_noalloc_at_the_largest_accepted_workspace():
+    """A shape whose tensor-core workspace sits just under the 16 MiB scratch:
+    the last bytes of the array are in use, so an offset past its end would show."""
+    S = skv()
+    w = gen.workload(0)                    # 4 heads, d_h 64, r_k 16, R 64: the tensor-core path
+    B = 2
+    kv0, _ = make_ctx(w, max_position=64)
+    try:
+        best = None
+        for mp in range(1024, 40000, 256):
+            ws = S.starkv_workspace_bytes(kv0.ctx, S.OP_DECODE, B, mp)
+            if ws <= SCRATCH:
+                best = (mp, ws)
+            else:
+                break
+        assert best is not None
+        mp, ws = best
+        assert ws > SCRATCH - (1 << 20), f"largest accepted workspace {ws} is not near the scratch size"
+        assert ws != _simt_workspace(B, w.H, w.R, mp)     # the tensor-core plan, not the CUDA-core one
+    finally:
+        kv0.close()
+    lens = [mp * 16, mp * 16 - 37]
+    kv, f = make_ctx(w, max_position=mp * 16 + 16)
+    try:
+        cfg, oc, bt, n_pages = oracle_cache(w, lens, extra_pages=1)
+        bt = np.pad(bt, ((0, 0), (0, mp - bt.shape[1])))
+        lc = kv.new_cache(n_pages)
+        upload(lc, oc)
+        qn = gen.make_queries(B, w.H, w.d_h, seed=7)
+        q = bf16_tensor(qn)
+        btd = torch.from_numpy(np.ascontiguousarray(bt)).cuda()
+        sl = torch.tensor(np.asarray(lens, np.int32)).cuda()
+        assert S.starkv_workspace_bytes(kv.ctx, S.OP_DECODE, B, mp) == ws
+        ref = kv.decode(lc, q, btd, sl).float().cpu().numpy()
+        want = O.decode(oc, qn, f.B_k, f.B_v, bt, lens)
+        check_attention(ref, want, "workspace decode")
+        for call in range(2):
+            out = torch.full_like(q, float("nan"))
+            S.starkv_decode_attn_noalloc(kv.ctx, lc.struct, q, btd, sl, out)
+            got = out.float().cpu().numpy()
+            check_attention(got, want, f"no-allocation decode, call {call}")
+            assert np.abs(got - ref).max() <= ATOL_MAX
+        assert kv.status() == 0
+    finally:
+        kv.close()
+
+
+def test_noalloc_limit_is_the_tensor_core_workspace():
+    """A shape whose CUDA-core partials would fit in 16 MiB but whose
+    tensor-core workspace (score rows, query images, partials) does not is
+    rejected: the documented limit is starkv_workspace_bytes, not the partials."""
+    S = skv()
+    w = gen.workload(1)
+    kv, _ = make_ctx(w, max_position=64)
+    try:
+        B, mp = 64, 2048
+        assert _simt_workspace(B, w.H, w.R, mp) <= SCRATCH
+        assert S.starkv_workspace_bytes(kv.ctx, S.OP_DECODE, B, mp) > SCRATCH
+        lc = kv.new_cache(1)
+        q = torch.zeros((B, w.H, w.d_h), dtype=torch.bfloat16, device="cuda")
+        bt = torch.zeros((B, mp), dtype=torch.int32, device="cuda")
+        sl = torch.ones(B, dtype=torch.int32, device="cuda")
+        with pytest.raises(S.StarKVError) as e:
+            S.starkv_decode_attn_noalloc(kv.ctx, lc.struct, q, bt, sl, torch.empty_like(q))
+        assert e.value.code == S.ERR_UNSUPPORTED_SHAPE
     finally:
         kv.close()

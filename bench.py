@@ -2,26 +2,38 @@
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl starkv|reference] [--workload NAME]
 
-One step = one pass of the decode hot path over one batch: append one new token
-per sequence (project, rotate, quantise, pack) and then batched single-query
-attention over the packed cache (dequantise, re-expand and RoPE keys, online
-softmax, P Z_v in the latent, split merge, B_v projection).  Default workload:
-LongChat-7B-shaped layer, 32 heads, d_h 128, r_k 32, R 1024, batch 16, context
-4096, 16-token pages.  Inputs are seeded and synthetic (no weights or datasets).
+One step = one pass of the hot path over one batch.  Decode workloads: append
+one new token per sequence (project, rotate, quantise, pack), then batched
+single-query attention over the packed cache (dequantise, re-expand and RoPE
+keys, online softmax, P Z_v in the latent, split merge, B_v projection).
+Prefill workload: append a chunk of tokens, then causal attention of the
+chunk's queries over the whole cache.
 
-For N > 1 (torchrun), every rank runs its own batch of independent sequences
-(weak scaling, no collective on the data path); the timing is the maximum over
-ranks.  The reference arm times the fp64 CPU oracle on a bounded sample of the
-same workload.
+Default (headline) workload: Llama-3-8B-shaped GQA decode layer, 32 query
+heads over 8 KV heads, d_h 128, r_k 64, R 512, batch 32, ragged contexts
+U[4096, 8192], 16-token pages.  At N = 1 the line also carries one record per
+other workload (LongChat-7B-shaped decode at batch 16 x 4096, the 128-step
+single-stream run from 32768 tokens, and the chunked prefill), each with its
+own roofline, end-to-end figure, clocks and CPU oracle baseline.  Inputs are
+seeded and synthetic (no weights or datasets).
+
+With --gpus N > 1 outside torchrun, the bench starts N ranks itself through
+torch.distributed.run (one process per GPU).  Every rank runs its own batch of
+independent sequences (weak scaling, no collective on the data path); the
+timing is the maximum over ranks.  The reference arm times the fp64 CPU oracle
+on a bounded sample of the same workload.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 import numpy as np
@@ -33,16 +45,16 @@ if ROOT not in sys.path:
 from harness import gen  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
-FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0          # B200 HBM3e bandwidth as specified (DGX figure)
+FALLBACK_HBM_GBS = 6650.0      # copy bandwidth measured earlier on this kind of GPU
+FALLBACK_BF16_TFLOPS = 1590.0  # cuBLAS bf16 burst measured earlier on this kind of GPU
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 
-# DRAM bytes (read + write) of one decode call, summed over its four kernels,
-# from one ncu capture of the current kernels (profiles/decode_kernels_*.md);
-# None for a workload without a capture.  Reset whenever a decode kernel changes.
-DECODE_TRAFFIC_NCU: dict = {}
-# The last capture, taken before the projection kernel's loads were reordered
-# (same loads and bytes, issued earlier); reported under its own key, never as
-# `traffic`.
-DECODE_TRAFFIC_LAST_CAPTURE = {"longchat7b_decode_b16_t4096": 134_520_000}
+HEADLINE = "llama3_8b_gqa_decode_b32_t4096to8192"
+SUBRECORDS = ["longchat7b_decode_b16_t4096", "longchat7b_stream_b1_t32768_s128",
+              "longchat7b_prefill_b4_t30720_c2048"]
+CSRC = os.path.join(ROOT, "rank_mixed_precision_b200", "csrc")
+TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 
 
 # ---------------------------------------------------------------------------
@@ -104,57 +116,151 @@ def shard_sequences(batch: int, rank: int, world: int, scaling: str = "weak"):
     return list(range(rank * per, min(batch, (rank + 1) * per))), 0
 
 
-# ---------------------------------------------------------------------------
-# clocks
-# ---------------------------------------------------------------------------
-class ClockSampler:
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+def free_port() -> int:
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
 
-    def __init__(self, gpu_index: int):
-        self.idx = gpu_index
-        self.proc = None
+
+def launch_ranks(n: int, argv) -> int:
+    """Run this script as n ranks (one process per GPU) under torch.distributed.run."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__)] + list(argv)
+    return subprocess.call(cmd)
+
+
+# ---------------------------------------------------------------------------
+# clocks: sampled by a host thread from warm-up to the end of the repeat pass
+# ---------------------------------------------------------------------------
+# NVML clock event reason bits
+_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+_IDLE = 0x1
+
+
+class ClockSampler:
+    """Samples SM clock, its maximum, power and throttle reasons every ~10 ms
+    (NVML, read-only queries; nvidia-smi when NVML is unavailable).  mark()
+    records the start of a named phase so a summary covers chosen phases."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active")
+
+    def __init__(self, gpu_index: int, period_s: float = 0.01):
+        self.idx, self.period = gpu_index, period_s
+        self.samples = []           # (t, sm_mhz, max_mhz, reasons_mask, power_w)
+        self.marks = {}
+        self._stop = threading.Event()
+        self._thread = None
+        self.source = None
+
+    def _nvml_loop(self, nv, h):
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                rs = get(h)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1e3
+                self.samples.append((time.perf_counter(), float(sm), float(mx), int(rs), float(pw)))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def _smi_loop(self, proc):
+        for line in proc.stdout:
+            if self._stop.is_set():
+                break
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 5:
+                continue
+            try:
+                self.samples.append((time.perf_counter(), float(p[1]), float(p[2]), int(p[4], 16),
+                                     float(p[3])))
+            except ValueError:
+                continue
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "50"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self._physical_index())
+            self.source = "nvml"
+            self._thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
         except Exception:
             self.proc = None
+            try:
+                self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self._physical_index()), f"--query-gpu={self.Q}",
+                                              "--format=csv,noheader,nounits", "-lms", "50"],
+                                             stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi"
+                self._thread = threading.Thread(target=self._smi_loop, args=(self.proc,), daemon=True)
+            except Exception:
+                self._thread = None
+        if self._thread is not None:
+            self._thread.start()
+            t0 = time.perf_counter()
+            while not self.samples and time.perf_counter() - t0 < 5.0:  # the sampler sees the run from its start
+                time.sleep(0.005)
+        self.mark("start")
         return self
 
-    def __exit__(self, *a):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except Exception:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+    def _physical_index(self) -> int:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            ids = [v.strip() for v in vis.split(",") if v.strip()]
+            if self.idx < len(ids) and ids[self.idx].isdigit():
+                return int(ids[self.idx])
+        return self.idx
 
-    def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
-            p = [x.strip() for x in l.split(",")]
-            if len(p) < 9:
-                continue
-            try:
-                sm.append(float(p[1]))
-                mx.append(float(p[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, p[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+    def mark(self, name):
+        self.marks[name] = time.perf_counter()
+
+    def __exit__(self, *a):
+        self.mark("end")
+        self._stop.set()
+        if getattr(self, "proc", None) is not None:
+            self.proc.terminate()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+
+    def summary(self, since: str = "start", until: str = "end"):
+        t0, t1 = self.marks.get(since, 0.0), self.marks.get(until, float("inf"))
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        busy = [s for s in win if not s[3] & _IDLE] or win
+        if not busy:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        reasons = sorted({n for s in busy for bit, n in _REASONS.items() if s[3] & bit})
+        return {"sm_mhz": statistics.median(s[1] for s in busy), "sm_max_mhz": max(s[2] for s in busy),
+                "power_w_max": max(s[4] for s in busy), "reasons": reasons, "samples": len(busy),
+                "source": self.source, "window_s": round(t1 - t0, 3) if t1 != float("inf") else None}
+
+
+def sustained_pass(step, first: int, seconds: float):
+    """Steps back to back for at least `seconds` of device time (CUDA events on
+    the launching stream); returns steps run and ms per step."""
+    import torch
+    n, ms, chunk = 0, 0.0, 32
+    while ms < seconds * 1e3:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for k in range(chunk):
+            step(first + n + k)
+        b.record()
+        b.synchronize()
+        ms += a.elapsed_time(b)
+        n += chunk
+        chunk = min(chunk * 2, 4096)
+    return n, ms / n
+
+
+def sustained_record(n, ms_per_step, units_per_step, clocks, unit):
+    rec = {"steps": n, "seconds": n * ms_per_step / 1e3, "ms_per_step": ms_per_step,
+           "value": units_per_step / (ms_per_step / 1e3), "unit": unit}
+    if clocks.get("sm_mhz"):
+        rec["sm_mhz_median"] = clocks["sm_mhz"]
+        rec["ms_x_mhz"] = ms_per_step * clocks["sm_mhz"]
+    return rec
 
 
 def measured_peaks():
@@ -163,6 +269,47 @@ def measured_peaks():
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """(sustained bf16 TFLOP/s, kind): the denominator for a kernel timed inside a long step."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        if "bf16_tflops_sustained" in d:
+            return float(d["bf16_tflops_sustained"]), "measured, sustained"
+        return float(d["bf16_tflops"]), "measured, burst"
+    return FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback, sustained"
+
+
+def kernel_source_digest() -> str:
+    """Digest of the library's CUDA sources: DRAM traffic counted on one version
+    of the kernels is reported only while the sources are unchanged."""
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            h.update(open(os.path.join(CSRC, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(workload: str, what: str):
+    """DRAM bytes (read + write) per call from the committed ncu summary table:
+    lines `<workload> <what> <bytes> <source digest>`; None when the kernels
+    changed after the capture or nothing was captured."""
+    try:
+        lines = open(TRAFFIC_TABLE).read().splitlines()
+    except OSError:
+        return None, "no capture"
+    digest = kernel_source_digest()
+    stale = False
+    for ln in lines:
+        p = ln.split()
+        if len(p) >= 4 and not ln.startswith("#") and p[0] == workload and p[1] == what:
+            if p[3] == digest:
+                return int(p[2]), "ncu capture of the current kernels"
+            stale = True
+    return None, "kernels changed since the last capture" if stale else "no capture"
 
 
 def pack_layout(tensors, align: int = 256):
@@ -401,7 +548,7 @@ class PrefillState:
         if st:
             raise RuntimeError(f"device status {st:#x} after cache fill")
 
-    def step(self, ev=None):
+    def step(self, i=0, ev=None):
         S = self.S
         S.starkv_append(self.kv.ctx, self.cache.struct, self.X, self.slots)
         if ev is not None:
@@ -425,6 +572,10 @@ def prefill_flops(w) -> dict:
     return {k: v * w.batch for k, v in per.items()}
 
 
+PREFILL_DTYPE = "f32 (CUDA-core prefill)"
+PREFILL_KERNELS = "expand + attention kernels"
+
+
 def prefill_launches_per_step(max_pages: int, n_append: int) -> int:
     """Kernels one prefill step launches: the append (the general kernel above
     64 tokens, else the split-K projection and the quantiser) and the prefill
@@ -432,6 +583,99 @@ def prefill_launches_per_step(max_pages: int, n_append: int) -> int:
     max_len = max_pages * 16
     chunk = 512 if max_len >= 512 else max(32, -(-max_len // 32) * 32)
     return (1 if n_append > 64 else 2) + 2 + 2 * (-(-max_len // chunk))
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baselines (bounded samples, host cores; a baseline, not a target)
+# ---------------------------------------------------------------------------
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def _timed(fn, seconds, at_least=1):
+    done, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds and done >= at_least:
+            return done, el
+
+
+def _one_thread(fn, seconds):
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:
+        return None
+    with threadpool_limits(limits=1):
+        return _timed(fn, seconds)
+
+
+def _oracle_setup(w, seed, b, extra=0):
+    import oracle as O
+    cfg = O.config_of(w)
+    L = int(gen.make_seq_lens(w, seed)[b])
+    bt, n_pages = gen.make_block_table([L + extra], seed)
+    oc = O.new_cache(cfg, n_pages)
+    zk, zv = gen.make_latents(w, L, seed, sub=b)
+    O.write_latents(oc, gen.slots_for(bt, 0, np.arange(L)), zk, zv)
+    f = gen.make_factors(w, seed)
+    q = gen.make_queries(1, w.H, w.d_h, seed, name="q_step", sub=b)
+    return O, oc, bt, L, f, q
+
+
+def cpu_baseline(w, seed, seconds):
+    """One oracle decode call of one whole sequence (all heads), repeated for
+    about `seconds`; then the same call on one BLAS thread."""
+    O, oc, bt, L, f, q = _oracle_setup(w, seed, 0)
+    call = lambda: O.decode(oc, q, f.B_k, f.B_v, bt, [L])
+    done, el = _timed(call, seconds)
+    rec = {"value": done * L / el, "unit": "context-tokens/s", "cores": _blas_threads(), "kind": "oracle",
+           "sample": f"{done} oracle decode call(s) of one {L}-token sequence, all {w.H} heads, "
+                     f"fp64 numpy, {el:.1f} s", "host_cpu_count": os.cpu_count()}
+    one = _one_thread(call, seconds / 4)
+    if one:
+        rec["one_thread"] = {"value": one[0] * L / one[1], "cores": 1,
+                             "sample": f"{one[0]} call(s) of the same sequence on one BLAS thread, {one[1]:.1f} s"}
+    return rec
+
+
+def cpu_baseline_stream(w, seed, n_steps=8):
+    """The first n_steps stream steps on the oracle: append one token (projection,
+    rotation, quantiser, packing) then decode the grown context, per step."""
+    O, oc, bt, L0, f, _ = _oracle_setup(w, seed, 0, extra=n_steps)
+    X = [gen.make_hidden(1, w.hidden, seed, name="X_step", sub=s) for s in range(n_steps)]
+    q = [gen.make_queries(1, w.H, w.d_h, seed, name="q_step", sub=s) for s in range(n_steps)]
+    state = {"s": 0}
+
+    def step():
+        s = state["s"]
+        O.append(oc, X[s % n_steps], f.A_k, f.A_v, gen.slots_for(bt, 0, [L0 + s % n_steps]))
+        O.decode(oc, q[s % n_steps], f.B_k, f.B_v, bt, [L0 + s % n_steps + 1])
+        state["s"] += 1
+
+    t0 = time.perf_counter()
+    for _ in range(n_steps):
+        step()
+    el = time.perf_counter() - t0
+    tokens = sum(L0 + s + 1 for s in range(n_steps))
+    rec = {"value": tokens / el, "unit": "context-tokens/s", "cores": _blas_threads(), "kind": "oracle",
+           "sample": f"the first {n_steps} stream steps (append 1 token + decode of {L0 + 1}..{L0 + n_steps} "
+                     f"tokens, all {w.H} heads), fp64 numpy, {el:.1f} s, {el / n_steps:.2f} s per step",
+           "seconds_per_step": el / n_steps, "host_cpu_count": os.cpu_count()}
+    hs = list(range(max(1, w.H // 8)))
+    one = _one_thread(lambda: O.decode(oc, q[0], f.B_k, f.B_v, bt, [L0 + 1], heads=hs), 0.0)
+    if one:
+        rec["one_thread"] = {"value": (L0 + 1) * (len(hs) / w.H) * one[0] / one[1], "cores": 1,
+                             "sample": f"{one[0]} decode(s) of the first stream step's {L0 + 1} tokens on one "
+                                       f"BLAS thread, {len(hs)} of {w.H} heads (counted as {len(hs)}/{w.H} of "
+                                       f"its tokens), {one[1]:.1f} s"}
+    return rec
 
 
 def prefill_sample_flops(w, n_q: int, L: int) -> float:
@@ -447,45 +691,65 @@ def prefill_sample_flops(w, n_q: int, L: int) -> float:
 def cpu_baseline_prefill(w, seed, seconds, n_q=4):
     O, oc, bt, L, f, _ = _oracle_setup(w, seed, 0)
     q = gen.make_queries(n_q, w.H, w.d_h, seed, name="q_chunk")
-    done, t0 = 0, time.perf_counter()
-    while True:
-        O.prefill(oc, q, [0, n_q], f.B_k, f.B_v, bt, [L])
-        done += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    return {"value": done * prefill_sample_flops(w, n_q, L) / el / 1e12, "unit": "TFLOP/s",
-            "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{done} oracle prefill call(s) of {n_q} queries at the end of one {L}-token sequence, "
-                      f"all {w.H} heads, fp64 numpy, {el:.1f} s", "host_cpu_count": os.cpu_count()}
+    call = lambda: O.prefill(oc, q, [0, n_q], f.B_k, f.B_v, bt, [L])
+    done, el = _timed(call, seconds)
+    fl = prefill_sample_flops(w, n_q, L)
+    rec = {"value": done * fl / el / 1e12, "unit": "TFLOP/s",
+           "cores": _blas_threads(), "kind": "oracle",
+           "sample": f"{done} oracle prefill call(s) of {n_q} queries at the end of one {L}-token sequence, "
+                     f"all {w.H} heads, fp64 numpy, {el:.1f} s", "host_cpu_count": os.cpu_count()}
+    one = _one_thread(call, seconds / 4)
+    if one:
+        rec["one_thread"] = {"value": one[0] * fl / one[1] / 1e12, "cores": 1,
+                             "sample": f"{one[0]} call(s) of the same sample on one BLAS thread, {one[1]:.1f} s"}
+    return rec
 
 
-def run_prefill(args, w, rank, world, local):
+# ---------------------------------------------------------------------------
+# legs
+# ---------------------------------------------------------------------------
+def _timed_region(st, args, world, local, n_steps, timed_steps=None):
+    """Warm-up, the timed steps (CUDA events on the launching stream, barriers
+    on both sides) and a repeat pass of at least --sustain-seconds, all inside
+    one clock sampler.  Returns (step ms total, per-step call events, sustained
+    (n, ms/step), clocks of the timed region + repeat pass)."""
+    import torch
+    with ClockSampler(local) as clk:
+        for i in range(args.warmup):
+            st.step(i)
+        torch.cuda.synchronize()
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(n_steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        clk.mark("timed")
+        t0.record()
+        for i in range(n_steps):
+            st.step(i, pairs[i])
+        t1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        sus = sustained_pass(st.step, n_steps, args.sustain_seconds) if args.sustain_seconds > 0 else None
+        torch.cuda.synchronize()
+        clk.mark("after")
+    return t0.elapsed_time(t1), pairs, sus, clk.summary("timed", "after")
+
+
+def run_prefill(args, w, rank, world, local, with_cpu=True, n_steps=None):
     import torch
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     init_dist(world, "nccl")
+    n_steps = n_steps or args.steps
     st = PrefillState(w, args.seed, device)
-    for _ in range(args.warmup):
-        st.step()
-    torch.cuda.synchronize()
-    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t0.record()
-        for i in range(args.steps):
-            st.step(pairs[i])
-        t1.record()
-        torch.cuda.synchronize()
-    barrier(world)
+    ms, pairs, sus, clocks = _timed_region(st, args, world, local, n_steps)
     if st.kv.status():
         raise RuntimeError("device status set during the timed region")
     fl = prefill_flops(w)
     total = sum(fl.values())
-    value, ms_max = job_throughput(total * args.steps / 1e12, t0.elapsed_time(t1), world, device)
-    attn_ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+    value, ms_max = job_throughput(total * n_steps / 1e12, ms, world, device)
+    attn_ms = sum(a.elapsed_time(b) for a, b in pairs) / n_steps
     # ---- end to end through the public API with host buffers: the step's
     # inputs packed in one pinned staging buffer, one copy each way
     srcs = [st.X.cpu(), st.slots.cpu(), st.q.cpu(), st.cu_q.cpu(), st.bt.cpu(), st.sl.cpu()]
@@ -511,73 +775,103 @@ def run_prefill(args, w, rank, world, local):
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(args.steps):
+    for _ in range(n_steps):
         e2e_step()
     e1.record()
     torch.cuda.synchronize()
     barrier(world)
-    e2e_value, _ = job_throughput(total * args.steps / 1e12, e0.elapsed_time(e1), world, device)
+    e2e_value, _ = job_throughput(total * n_steps / 1e12, e0.elapsed_time(e1), world, device)
     if rank != 0:
         return None
-    peaks = {}
-    try:
-        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
-    except (OSError, ValueError):
-        pass
-    peak = float(peaks.get("bf16_tflops", 1590.0))
+    peak, peak_kind = measured_tensor_peak()
     achieved = (total - fl["projection"]) / (attn_ms / 1e3) / 1e12
+    traffic, tnote = dram_traffic(w.name, "prefill_call")
     line = {
         "metric": "prefill TFLOP/s (algorithmic)", "value": value, "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32 (CUDA-core prefill)", "data": "synthetic (seeded)",
+        "steps": n_steps, "warmup": args.warmup, "ms_per_step": ms_max / n_steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": PREFILL_DTYPE, "data": "synthetic (seeded)",
         "config": {"workload": w.name, "batch": w.batch, "ctx": w.ctx, "chunk": w.chunk,
                    "step": "append the chunk + causal prefill attention of its queries",
                    "l2": f"cache {st.cache.nbytes() / 2**20:.0f} MiB read per step (vs 126 MiB L2)"},
         "flops_per_step": fl,
-        "roofline": {"bound": "tensor", "kernel": "starkv_prefill_attn (expand + attention kernels)",
-                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "traffic": None, "launch_ms": attn_ms},
+        "roofline": {"bound": "tensor", "kernel": "starkv_prefill_attn (" + PREFILL_KERNELS + ")",
+                     "achieved": achieved, "peak": peak, "peak_kind": f"bf16 dense TFLOP/s ({peak_kind}); "
+                     "fp16 operands share the nominal dense rate", "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": traffic, "traffic_source": tnote, "launch_ms": attn_ms},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": prefill_launches_per_step(int(st.bt.shape[1]), w.batch * w.chunk) * args.steps,
-        "clocks": clk.summary(),
+        "gpu_launches": prefill_launches_per_step(int(st.bt.shape[1]), w.batch * w.chunk) * n_steps,
+        "clocks": clocks,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if sus:
+        line["sustained"] = sustained_record(sus[0], sus[1], total / 1e12, clocks, "TFLOP/s")
+    if world == 1 and with_cpu:
         line["cpu_baseline"] = cpu_baseline_prefill(w, args.seed, args.cpu_seconds)
     return line
 
 
-def run_starkv(args, w, rank, world, local):
+def decode_launches_per_step(n_append: int) -> int:
+    """Kernels of one decode step: the append (split-K projection + quantiser for
+    up to 64 tokens, one fused kernel above) and the decode (query fold, scores,
+    values, projection)."""
+    return (2 if n_append <= 64 else 1) + 4
+
+
+def _decode_line(w, args, world, st, n_steps, ms_max, dec_ms, value, tokens_per_step, e2e, clocks, sus, cfg_extra):
+    peak, peak_kind = measured_peaks()
+    alg = decode_algorithmic_bytes(w, tokens_per_step, w.batch, st.max_pages)
+    achieved = alg / (dec_ms / 1e3) / 1e9
+    traffic, tnote = dram_traffic(w.name, "decode_call")
+    line = {
+        "metric": "decode context-tokens/s",
+        "value": value,
+        "unit": "context-tokens/s",
+        "n_gpus": world,
+        "steps": n_steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max / n_steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp16 tensor-core operands, fp32 accumulation",
+        "data": "synthetic (seeded; shapes of the named model, no weights)",
+        "config": {"workload": w.name, "batch": w.batch,
+                   "heads": w.H, "kv_heads": w.h_kv, "head_dim": w.d_h, "rank_k": w.r_k, "rank_v": w.R,
+                   "bits": "4/3 (top 25% of channels 4-bit)", "page_tokens": 16,
+                   "parallelism": f"dp{world} (independent sequences per GPU)",
+                   "l2": f"{len(st.caches)} rotating cache replicas "
+                         f"({len(st.caches) * st.caches[0].nbytes() / 2**20:.0f} MiB > 126 MiB L2)", **cfg_extra},
+        "roofline": {"bound": "hbm", "kernel": "starkv_decode_attn (query fold + scores + values + projection)",
+                     "achieved": achieved, "peak": peak, "peak_kind": f"hbm copy GB/s ({peak_kind})",
+                     "unit": "GB/s", "frac": achieved / peak, "spec_gbs": SPEC_HBM_GBS,
+                     "frac_of_spec": achieved / SPEC_HBM_GBS, "traffic": traffic, "traffic_source": tnote,
+                     "algorithmic_bytes_per_launch": alg, "launch_ms": dec_ms,
+                     "achieved_context_tokens_per_s_decode_only": tokens_per_step / (dec_ms / 1e3)},
+        "e2e": e2e,
+        "gpu_launches": decode_launches_per_step(w.batch) * n_steps,
+        "clocks": clocks,
+    }
+    if sus:
+        line["sustained"] = sustained_record(sus[0], sus[1], tokens_per_step, clocks, "context-tokens/s")
+    return line
+
+
+def run_starkv(args, w, rank, world, local, with_cpu=True, n_steps=None):
     import torch
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     init_dist(world, "nccl")
+    n_steps = n_steps or args.steps
     replicas = max(1, int(np.ceil(3 * L2_BYTES / max(1, w.batch * w.ctx * bytes_per_token(w)))))
     replicas = max(replicas, 2)
     st = DecodeState(w, args.seed, device, replicas)
     S = st.S
-    launches_per_step = 6  # append (split-K projection, quantise), decode (query fold, scores, values, projection)
-    for i in range(args.warmup):
-        st.step(i)
-    torch.cuda.synchronize()
-    # ---- device-resident timed region
-    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t0.record()
-        for i in range(args.steps):
-            st.step(i, pairs[i])
-        t1.record()
-        torch.cuda.synchronize()
-    barrier(world)
-    ms = t0.elapsed_time(t1)
-    dec_ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+    ms, pairs, sus, clocks = _timed_region(st, args, world, local, n_steps)
+    dec_ms = sum(a.elapsed_time(b) for a, b in pairs) / n_steps
     status = st.kv.status()
     if status:
         raise RuntimeError(f"device status {status:#x} during the timed region")
     tokens_per_step = int(st.seq_lens.sum())
-    value, ms_max = job_throughput(tokens_per_step * args.steps, ms, world, device)
+    value, ms_max = job_throughput(tokens_per_step * n_steps, ms, world, device)
     # ---- end to end through the public API with host buffers: the step's
     # inputs sit packed in one pinned staging buffer and cross in one copy
     t_ = lambda a: torch.from_numpy(np.ascontiguousarray(a))
@@ -606,86 +900,41 @@ def run_starkv(args, w, rank, world, local):
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for i in range(args.steps):
+    for i in range(n_steps):
         e2e_step(i)
     e1.record()
     torch.cuda.synchronize()
     barrier(world)
-    e2e_value, _ = job_throughput(tokens_per_step * args.steps, e0.elapsed_time(e1), world, device)
+    e2e_value, _ = job_throughput(tokens_per_step * n_steps, e0.elapsed_time(e1), world, device)
 
     if rank != 0:
         return None
-    peak, peak_kind = measured_peaks()
-    alg = decode_algorithmic_bytes(w, tokens_per_step, w.batch, st.max_pages)
-    achieved = alg / (dec_ms / 1e3) / 1e9
-    line = {
-        "metric": "decode context-tokens/s",
-        "value": value,
-        "unit": "context-tokens/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": ms_max / args.steps,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "fp16 tensor-core operands, fp32 accumulation",
-        "data": "synthetic (seeded; shapes of the named model, no weights)",
-        "config": {"workload": w.name, "batch": w.batch, "ctx": int(st.seq_lens.max()),
-                   "heads": w.H, "kv_heads": w.h_kv, "head_dim": w.d_h, "rank_k": w.r_k, "rank_v": w.R,
-                   "bits": "4/3 (top 25% of channels 4-bit)", "page_tokens": 16,
-                   "step": "append 1 token per sequence + decode attention",
-                   "parallelism": f"dp{world} (independent sequences per GPU)",
-                   "l2": f"{len(st.caches)} rotating cache replicas "
-                         f"({len(st.caches) * st.caches[0].nbytes() / 2**20:.0f} MiB > 126 MiB L2)"},
-        "roofline": {"bound": "hbm", "kernel": "starkv_decode_attn (scores + values + projection kernels)",
-                     "achieved": achieved, "peak": peak, "peak_kind": f"hbm copy GB/s ({peak_kind})",
-                     "unit": "GB/s", "frac": achieved / peak, "traffic": DECODE_TRAFFIC_NCU.get(w.name),
-                     "traffic_last_capture": DECODE_TRAFFIC_LAST_CAPTURE.get(w.name),
-                     "algorithmic_bytes_per_launch": alg, "launch_ms": dec_ms,
-                     "achieved_context_tokens_per_s_decode_only": tokens_per_step / (dec_ms / 1e3)},
-        "e2e": {"value": e2e_value, "unit": "context-tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
-    }
-    if world == 1 and not args.no_cpu_baseline:
+    e2e = {"value": e2e_value, "unit": "context-tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    extra = {"ctx": int(st.seq_lens.max()), "ctx_min": int(st.seq_lens.min()),
+             "step": "append 1 token per sequence + decode attention"}
+    line = _decode_line(w, args, world, st, n_steps, ms_max, dec_ms, value, tokens_per_step, e2e, clocks, sus, extra)
+    if world == 1 and with_cpu:
         line["cpu_baseline"] = cpu_baseline(w, args.seed, args.cpu_seconds)
     return line
 
 
-def run_stream(args, w, rank, world, local):
+def run_stream(args, w, rank, world, local, with_cpu=True, n_steps=None):
     """Long-context stream: each timed step appends one token per sequence and
     decodes the grown context; the run walks the stream's steps in order."""
     import torch
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     init_dist(world, "nccl")
+    n_steps = n_steps or args.steps
     replicas = max(2, int(np.ceil(3 * L2_BYTES / max(1, w.batch * w.ctx * bytes_per_token(w)))))
     st = StreamState(w, args.seed, device, replicas)
     S = st.S
-    launches_per_step = 6  # append (split-K projection, quantise), decode (query fold, scores, values, projection)
-    for i in range(args.warmup):
-        st.step(i)
-    torch.cuda.synchronize()
-    # ---- device-resident timed region: stream steps 0, 1, ... in order
-    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t0.record()
-        for i in range(args.steps):
-            st.step(i, pairs[i])
-        t1.record()
-        torch.cuda.synchronize()
-    barrier(world)
-    ms = t0.elapsed_time(t1)
-    dec_ms = sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+    ms, pairs, sus, clocks = _timed_region(st, args, world, local, n_steps)
+    dec_ms = sum(a.elapsed_time(b) for a, b in pairs) / n_steps
     status = st.kv.status()
     if status:
         raise RuntimeError(f"device status {status:#x} during the timed region")
-    tokens = sum(st.tokens(i) for i in range(args.steps))
+    tokens = sum(st.tokens(i) for i in range(n_steps))
     value, ms_max = job_throughput(tokens, ms, world, device)
     # ---- end to end through the public API with host buffers: each stream
     # step's inputs sit packed in one row of a pinned staging buffer
@@ -721,7 +970,7 @@ def run_stream(args, w, rank, world, local):
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for i in range(args.steps):
+    for i in range(n_steps):
         e2e_step(i)
     e1.record()
     torch.cuda.synchronize()
@@ -730,84 +979,16 @@ def run_stream(args, w, rank, world, local):
 
     if rank != 0:
         return None
-    peak, peak_kind = measured_peaks()
-    mean_tokens = tokens / args.steps
-    alg = decode_algorithmic_bytes(w, mean_tokens, w.batch, st.max_pages)
-    achieved = alg / (dec_ms / 1e3) / 1e9
+    mean_tokens = tokens / n_steps
     L0, Ln = int(st.L0.max()), int(st.L0.max()) + st.n
-    line = {
-        "metric": "decode context-tokens/s",
-        "value": value,
-        "unit": "context-tokens/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": ms_max / args.steps,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "fp16 tensor-core operands, fp32 accumulation",
-        "data": "synthetic (seeded; shapes of the named model, no weights)",
-        "config": {"workload": w.name, "batch": w.batch, "ctx": f"{L0} -> {Ln}",
-                   "heads": w.H, "kv_heads": w.h_kv, "head_dim": w.d_h, "rank_k": w.r_k, "rank_v": w.R,
-                   "bits": "4/3 (top 25% of channels 4-bit)", "page_tokens": 16,
-                   "step": f"append 1 token per sequence + decode of the grown context; "
-                           f"run step i is stream step i mod {st.n}",
-                   "parallelism": f"dp{world} (independent sequences per GPU)",
-                   "l2": f"{len(st.caches)} rotating cache replicas "
-                         f"({len(st.caches) * st.caches[0].nbytes() / 2**20:.0f} MiB > 126 MiB L2)"},
-        "roofline": {"bound": "hbm", "kernel": "starkv_decode_attn (scores + values + projection kernels)",
-                     "achieved": achieved, "peak": peak, "peak_kind": f"hbm copy GB/s ({peak_kind})",
-                     "unit": "GB/s", "frac": achieved / peak, "traffic": DECODE_TRAFFIC_NCU.get(w.name),
-                     "algorithmic_bytes_per_launch": alg, "launch_ms": dec_ms,
-                     "achieved_context_tokens_per_s_decode_only": mean_tokens / (dec_ms / 1e3)},
-        "e2e": {"value": e2e_value, "unit": "context-tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
-    }
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, args.seed, args.cpu_seconds)
+    e2e = {"value": e2e_value, "unit": "context-tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    extra = {"ctx": f"{L0} -> {Ln}",
+             "step": f"append 1 token per sequence + decode of the grown context; "
+                     f"run step i is stream step i mod {st.n}"}
+    line = _decode_line(w, args, world, st, n_steps, ms_max, dec_ms, value, mean_tokens, e2e, clocks, sus, extra)
+    if world == 1 and with_cpu:
+        line["cpu_baseline"] = cpu_baseline_stream(w, args.seed)
     return line
-
-
-# ---------------------------------------------------------------------------
-# CPU oracle baseline (bounded sample)
-# ---------------------------------------------------------------------------
-def _oracle_setup(w, seed, b):
-    import oracle as O
-    cfg = O.config_of(w)
-    L = int(gen.make_seq_lens(w, seed)[b])
-    bt, n_pages = gen.make_block_table([L], seed)
-    oc = O.new_cache(cfg, n_pages)
-    zk, zv = gen.make_latents(w, L, seed, sub=b)
-    O.write_latents(oc, gen.slots_for(bt, 0, np.arange(L)), zk, zv)
-    f = gen.make_factors(w, seed)
-    q = gen.make_queries(1, w.H, w.d_h, seed, name="q_step", sub=b)
-    return O, oc, bt, L, f, q
-
-
-def _blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
-        return int(max(n)) if n else 1
-    except Exception:
-        return 1
-
-
-def cpu_baseline(w, seed, seconds):
-    O, oc, bt, L, f, q = _oracle_setup(w, seed, 0)
-    done, t0 = 0, time.perf_counter()
-    while True:
-        O.decode(oc, q, f.B_k, f.B_v, bt, [L])
-        done += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    return {"value": done * L / el, "unit": "context-tokens/s", "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{done} oracle decode call(s) of one {L}-token sequence, all {w.H} heads, "
-                      f"fp64 numpy, {el:.1f} s", "host_cpu_count": os.cpu_count()}
 
 
 def run_reference(args, w, rank, world):
@@ -876,29 +1057,65 @@ def _run_reference_prefill(args, w, world, n_q=4):
     }
 
 
+def run_leg(args, w, rank, world, local, with_cpu, n_steps=None):
+    if w.chunk > 0:
+        return run_prefill(args, w, rank, world, local, with_cpu, n_steps)
+    if w.steps > 0:
+        return run_stream(args, w, rank, world, local, with_cpu, n_steps)
+    return run_starkv(args, w, rank, world, local, with_cpu, n_steps)
+
+
+def subrecord_steps(w, steps: int) -> int:
+    """Timed steps of a workload's record: the stream walks all its steps at least once;
+    a prefill step is a long call, so at most 10 are timed."""
+    if w.steps > 0:
+        return max(steps, w.steps)
+    if w.chunk > 0:
+        return max(1, min(steps, 10))
+    return steps
+
+
 def main(argv=None):
+    argv = list(sys.argv[1:] if argv is None else argv)
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="starkv", choices=["starkv", "reference"])
-    ap.add_argument("--workload", default="longchat7b_decode_b16_t4096")
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--only", action="store_true", help="the named workload alone, without the other records")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--sustain-seconds", type=float, default=1.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "starkv":
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        rc = launch_ranks(args.gpus, argv)
+        if rc:
+            raise SystemExit(rc)
+        return
     rank, world, local = dist_env()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but {world} ranks were launched")
     w = gen.workload(args.workload)
     if args.impl == "reference":
         line = run_reference(args, w, rank, world)
-    elif w.chunk > 0:
-        line = run_prefill(args, w, rank, world, local)
-    elif w.steps > 0:
-        line = run_stream(args, w, rank, world, local)
     else:
-        line = run_starkv(args, w, rank, world, local)
+        line = run_leg(args, w, rank, world, local, not args.no_cpu_baseline)
+        if world == 1 and not args.only and line is not None:
+            recs = {}
+            for name in SUBRECORDS:
+                if name == w.name:
+                    continue
+                ws = gen.workload(name)
+                recs[name] = run_leg(args, ws, rank, world, local, not args.no_cpu_baseline,
+                                     subrecord_steps(ws, args.steps))
+            if recs:
+                line["workloads"] = recs
     if line is not None:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -171,6 +171,7 @@ __global__ void __launch_bounds__(128) decode_wprep_kernel(const __nv_bfloat16* 
 // TMEM columns of the score accumulators: two buffers of up to 256 columns.
 constexpr uint32_t kScoreTmemCols = 512;
 constexpr int kMaxKeyStages = 6;  // deepest key-stage ring
+constexpr int kMaxScoreItemsPerCta = 256;  // 128-token tiles per score CTA at most (8 KiB of page ids)
 
 // Issue the TMEM loads of one RK-column row into raw registers (no wait).
 template <int RK>
@@ -1415,8 +1416,12 @@ TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
     const double work = (double)bt * t.tpad * tok_bytes;
     const double part_unit = 2.0 * f.num_q_heads * f.rank_v * 4.0;
     const int threads = (kVRoleWarps + t.nW) * 32;
-    VSmem probe;
-    t.ok = value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, 1, probe);  // largest page table
+    VSmem probe;  // shared memory at the largest split count considered (for the residency query)
+    t.ok = value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, s0, probe);
+    while (!t.ok && s0 < t.stages_total) {  // very long contexts: more splits, smaller page tables
+      s0 = s0 * 2 < t.stages_total ? s0 * 2 : t.stages_total;
+      t.ok = value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, s0, probe);
+    }
     double best = -1.0;
     t.splits = 1;
     t.CS = 1;
@@ -1436,8 +1441,16 @@ TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
         t.CS = cs;
       }
     }
+    // a split's block-table entries live in shared memory: long contexts need
+    // enough splits (in whole clusters) for that table to fit
+    if (t.ok) {
+      t.ok = value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, t.splits, t.vs);
+      while (!t.ok && t.splits < t.stages_total) {
+        t.splits += t.CS;
+        t.ok = value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, t.splits, t.vs);
+      }
+    }
     t.nclust = t.splits / t.CS;
-    if (t.ok) t.ok = value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, t.splits, t.vs);
   }
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
   size_t o = 0;
@@ -1559,6 +1572,9 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   int ctas = sm_count();
   if (ctas > A.total_items) ctas = A.total_items;
   A.items_per_cta = (A.total_items + ctas - 1) / ctas;
+  // a CTA's block-table entries sit in shared memory: beyond this many tiles
+  // per CTA the grid grows past one wave instead
+  if (A.items_per_cta > kMaxScoreItemsPerCta) A.items_per_cta = kMaxScoreItemsPerCta;
   ctas = (A.total_items + A.items_per_cta - 1) / A.items_per_cta;
   A.n_pages = cache.n_pages;
   A.q = q;

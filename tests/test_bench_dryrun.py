@@ -38,6 +38,9 @@ class _Event:
     def elapsed_time(self, other):
         return max(1e-6, (other.t - self.t) * 1e3)
 
+    def synchronize(self):
+        pass
+
 
 class _Stream:
     cuda_stream = 0
@@ -160,7 +163,8 @@ def _run(argv):
 def test_stream_leg_walks_the_stream_in_order(dry):
     log, states = dry
     steps, warm = 25, 3
-    line = _run(["--workload", "dry_stream", "--steps", str(steps), "--warmup", str(warm), "--no-cpu-baseline"])
+    line = _run(["--workload", "dry_stream", "--steps", str(steps), "--warmup", str(warm), "--no-cpu-baseline",
+                 "--only", "--sustain-seconds", "0"])
     st = states[-1]
     n, L0 = st.n, st.L0
     # every replica source: context [0, L0) in chunks, then each stream token alone, in order
@@ -187,20 +191,25 @@ def test_stream_leg_walks_the_stream_in_order(dry):
 
 def test_decode_leg_line_has_the_contract_keys(dry):
     log, _ = dry
-    line = _run(["--workload", "dry_decode", "--steps", "7", "--warmup", "3", "--no-cpu-baseline"])
+    line = _run(["--workload", "dry_decode", "--steps", "7", "--warmup", "3", "--no-cpu-baseline", "--only",
+                 "--sustain-seconds", "0.01"])
     for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
-              "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+              "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks", "sustained"):
         assert k in line, k
-    for k in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+    for k in ("bound", "achieved", "peak", "unit", "frac", "traffic", "spec_gbs", "frac_of_spec"):
         assert k in line["roofline"], k
+    assert line["roofline"]["frac_of_spec"] == pytest.approx(line["roofline"]["achieved"] / 8000.0)
     assert line["config"]["workload"] == "dry_decode" and line["n_gpus"] == 1
-    assert sum(1 for e in log if e[0] == "decode") == 2 * (3 + 7)
+    # timed steps and the repeat pass: every one through the C ABI, then the end-to-end leg
+    sus = line["sustained"]["steps"]
+    assert sus >= 32 and sum(1 for e in log if e[0] == "decode") == 2 * (3 + 7) + sus
 
 
 def test_prefill_leg_line_counts_its_launches_and_copies(dry):
     log, _ = dry
     steps, warm = 4, 3
-    line = _run(["--workload", "dry_prefill", "--steps", str(steps), "--warmup", str(warm), "--no-cpu-baseline"])
+    line = _run(["--workload", "dry_prefill", "--steps", str(steps), "--warmup", str(warm), "--no-cpu-baseline",
+                 "--only", "--sustain-seconds", "0"])
     pre = [e for e in log if e[0] == "prefill"]
     assert len(pre) == 2 * (warm + steps)                  # device-resident leg, then end to end
     assert all(e[2] == 2 * 24 and e[3] == 24 for e in pre)
@@ -234,7 +243,7 @@ def _rank_worker(rank, world, port, workload, q):
         buf = io.StringIO()
         with contextlib.redirect_stdout(buf):
             bench.main(["--workload", workload, "--steps", "6", "--warmup", "3", "--no-cpu-baseline",
-                        "--gpus", str(world)])
+                        "--gpus", str(world), "--sustain-seconds", "0"])
         q.put((rank, buf.getvalue(), sum(1 for e in log if e[0] == "decode")))
     except Exception as e:  # reported to the parent, which fails the test
         q.put((rank, "error", repr(e)))
@@ -272,3 +281,47 @@ def test_two_gloo_ranks_run_the_bench_and_rank0_prints_the_job_line(workload):
         # whole-job rate: tokens of both ranks over the slowest rank's time
         tokens = 2 * 6 * int(gen.make_seq_lens(w).sum())
         assert line["value"] == pytest.approx(tokens / (line["ms_per_step"] * 6 / 1e3), rel=1e-9)
+
+
+def test_headline_line_carries_a_record_per_workload(dry, monkeypatch):
+    log, _ = dry
+    monkeypatch.setattr(bench, "SUBRECORDS", ["dry_decode", "dry_stream", "dry_prefill"])
+    line = _run(["--workload", "dry_decode", "--steps", "4", "--warmup", "3", "--no-cpu-baseline",
+                 "--sustain-seconds", "0"])
+    recs = line["workloads"]
+    assert set(recs) == {"dry_stream", "dry_prefill"}          # the headline is not repeated
+    for name, r in recs.items():
+        for k in ("metric", "value", "unit", "roofline", "e2e", "clocks", "gpu_launches", "config"):
+            assert k in r, (name, k)
+        assert r["config"]["workload"] == name
+    assert recs["dry_stream"]["steps"] == 9                    # the stream walks all its steps
+    assert recs["dry_prefill"]["roofline"]["bound"] == "tensor"
+
+
+def test_gpus_flag_starts_the_ranks_itself(monkeypatch):
+    calls = []
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(bench.subprocess, "call", lambda cmd: calls.append(cmd) or 0)
+    bench.main(["--gpus", "2", "--steps", "5", "--warmup", "3"])
+    (cmd,) = calls
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=2" in cmd and "--master-addr=127.0.0.1" in cmd and "--nnodes=1" in cmd
+    assert cmd[-6:] == ["--gpus", "2", "--steps", "5", "--warmup", "3"]
+    assert cmd[-7].endswith("bench.py")
+
+
+def test_gpus_flag_must_match_the_launched_ranks(monkeypatch):
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    with pytest.raises(SystemExit):
+        bench.main(["--gpus", "4", "--steps", "5", "--warmup", "3"])
+
+
+def test_traffic_is_reported_only_for_the_captured_kernels(tmp_path, monkeypatch):
+    table = tmp_path / "t.txt"
+    d = bench.kernel_source_digest()
+    table.write_text(f"# workload what bytes digest\nwl decode_call 123456 {d}\nwl2 decode_call 7 0000000000000000\n")
+    monkeypatch.setattr(bench, "TRAFFIC_TABLE", str(table))
+    assert bench.dram_traffic("wl", "decode_call") == (123456, "ncu capture of the current kernels")
+    assert bench.dram_traffic("wl2", "decode_call")[0] is None
+    assert "changed" in bench.dram_traffic("wl2", "decode_call")[1]
+    assert bench.dram_traffic("other", "decode_call")[0] is None

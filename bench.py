@@ -236,11 +236,13 @@ class ClockSampler:
                 "source": self.source, "window_s": round(t1 - t0, 3) if t1 != float("inf") else None}
 
 
-def sustained_pass(step, first: int, seconds: float):
+def sustained_pass(step, first: int, seconds: float, ms_hint: float = 0.0):
     """Steps back to back for at least `seconds` of device time (CUDA events on
-    the launching stream); returns steps run and ms per step."""
+    the launching stream); returns steps run and ms per step.  ms_hint (a step's
+    time from the timed region) sizes the first batch of steps."""
     import torch
-    n, ms, chunk = 0, 0.0, 32
+    chunk = 32 if ms_hint <= 0 else max(1, min(32, int(0.05 * seconds * 1e3 / ms_hint)))
+    n, ms = 0, 0.0
     while ms < seconds * 1e3:
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
@@ -572,17 +574,15 @@ def prefill_flops(w) -> dict:
     return {k: v * w.batch for k, v in per.items()}
 
 
-PREFILL_DTYPE = "f32 (CUDA-core prefill)"
-PREFILL_KERNELS = "expand + attention kernels"
+PREFILL_DTYPE = "fp16 tensor-core operands, fp32 accumulation"
+PREFILL_KERNELS = "tcgen05 key/value re-expansion + tcgen05 flash attention"
 
 
 def prefill_launches_per_step(max_pages: int, n_append: int) -> int:
     """Kernels one prefill step launches: the append (the general kernel above
     64 tokens, else the split-K projection and the quantiser) and the prefill
-    (init, then expand + attention per key chunk of up to 512 positions, finalize)."""
-    max_len = max_pages * 16
-    chunk = 512 if max_len >= 512 else max(32, -(-max_len // 32) * 32)
-    return (1 if n_append > 64 else 2) + 2 + 2 * (-(-max_len // chunk))
+    (re-expansion, then attention)."""
+    return (1 if n_append > 64 else 2) + 2
 
 
 # ---------------------------------------------------------------------------
@@ -730,7 +730,8 @@ def _timed_region(st, args, world, local, n_steps, timed_steps=None):
         t1.record()
         torch.cuda.synchronize()
         barrier(world)
-        sus = sustained_pass(st.step, n_steps, args.sustain_seconds) if args.sustain_seconds > 0 else None
+        ms_step = t0.elapsed_time(t1) / max(1, n_steps)
+        sus = sustained_pass(st.step, n_steps, args.sustain_seconds, ms_step) if args.sustain_seconds > 0 else None
         torch.cuda.synchronize()
         clk.mark("after")
     return t0.elapsed_time(t1), pairs, sus, clk.summary("timed", "after")

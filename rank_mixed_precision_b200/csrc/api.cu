@@ -206,6 +206,8 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
     cudaFree(c->Bv16);
     cudaFree(c->zpart);
     cudaFree(c->status);
+    cudaFree(c->Bk16);
+    cudaFree(c->Bv16p);
     delete c;
   };
   // small appends: K splits of the projection so that about every SM streams a
@@ -229,7 +231,8 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
       (e = cudaMalloc(&c->trig, trig_bytes)) != cudaSuccess || (e = cudaMalloc(&c->Bv16, bv_bytes / 2)) != cudaSuccess ||
       (e = cudaMalloc(&c->zpart, (size_t)(c->app_splits > 0 ? c->app_splits : 1) * kSmallAppend * c->lat_cols * 4)) !=
           cudaSuccess ||
-      (e = cudaMalloc(&c->status, sizeof(unsigned int))) != cudaSuccess) {
+      (e = cudaMalloc(&c->status, sizeof(unsigned int))) != cudaSuccess ||
+      (e = cudaMalloc(&c->Bk16, bk_bytes / 2)) != cudaSuccess || (e = cudaMalloc(&c->Bv16p, bv_bytes / 2)) != cudaSuccess) {
     cleanup();
     return cuda_fail(e, "cudaMalloc (context factors)");
   }
@@ -241,6 +244,7 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
                           (size_t)cfg->rank_v * 2, cfg->hidden, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = launch_prepare_factors(*c, (const __nv_bfloat16*)B_k, (const __nv_bfloat16*)B_v, s);
   if (e == cudaSuccess) e = launch_prepare_tc_factors(*c, s);
+  if (e == cudaSuccess) e = launch_prepare_prefill_factors(*c, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->status, 0, sizeof(unsigned int), s);
   // RoPE table: angle p * base^(-2i/d) in fp64, cos/sin in fp64, stored as fp32
   // and the same angles as an fp16 [cos.. | sin..] row per position (tensor-core operand)
@@ -275,6 +279,9 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
   const char* path = getenv("STARKV_DECODE_PATH");
   const bool want_simt = path && strcmp(path, "simt") == 0;
   c->tc = !want_simt && tc_decode_supported(c->cfg) && c->val.g == 16 && make_trig_map(c);
+  const char* ppath = getenv("STARKV_PREFILL_PATH");
+  const bool want_simt_prefill = ppath && strcmp(ppath, "simt") == 0;
+  c->tc_prefill = !want_simt_prefill && tc_prefill_supported(*c) && make_prefill_maps(c);
   if (c->app_splits > 0) {
     const int kl = cfg->hidden / c->app_splits;
     if (!starkv::encode_map_2d(&c->a_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->A, (uint64_t)c->lat_cols,
@@ -298,6 +305,8 @@ starkv_status starkv_destroy(starkv_ctx* ctx) {
   cudaFree(c->Bv16);
   cudaFree(c->zpart);
   cudaFree(c->status);
+  cudaFree(c->Bk16);
+  cudaFree(c->Bv16p);
   delete c;
   return ok();
 }

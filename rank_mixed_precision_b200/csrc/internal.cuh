@@ -48,6 +48,13 @@ struct Ctx {
   unsigned int* status;   // device status word
   CUtensorMap trig_map;   // TMA map of `trig`: box 64 x 128, 128-byte swizzle
   bool tc;                // tensor-core decode available for this shape
+  // tensor-core prefill operands
+  __half* Bk16;           // [h_kv][r_k][d_h] fp16 B'_k
+  __half* Bv16p;          // [R][h_kv*d_h] fp16 B'_v, rows of each 16-channel group in the order the
+                          // value dequantiser emits them (value_channel_of_position)
+  CUtensorMap bk_map;     // TMA map of Bk16 as [h_kv*r_k][d_h]: box 64 x r_k, 128-byte swizzle
+  CUtensorMap bvp_map;    // TMA map of Bv16p: box 64 x 64, 128-byte swizzle
+  bool tc_prefill;        // tensor-core prefill available for this shape
 };
 
 // 2-D TMA map over a row-major [rows][inner] array (no interleave, zero fill).
@@ -279,6 +286,20 @@ struct PrefillPlan {
   size_t ws_bytes;
 };
 PrefillPlan plan_prefill(const Ctx& c, int batch, int max_pages, int64_t total_q);
+PrefillPlan plan_prefill_simt(const Ctx& c, int batch, int max_pages, int64_t total_q);
+cudaError_t launch_prefill_simt(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
+                                const int32_t* cu_q, const int32_t* block_table, const int32_t* seq_lens,
+                                int batch, int max_pages, int64_t total_q, int max_q_len,
+                                __nv_bfloat16* out, void* ws, const PrefillPlan& plan, cudaStream_t s);
+// tensor-core prefill (prefill_tc.cu)
+bool tc_prefill_supported(const Ctx& c);
+PrefillPlan plan_prefill_tc(const Ctx& c, int batch, int max_pages, int64_t total_q);
+cudaError_t launch_prefill_tc(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
+                              const int32_t* cu_q, const int32_t* block_table, const int32_t* seq_lens,
+                              int batch, int max_pages, int64_t total_q, int max_q_len,
+                              __nv_bfloat16* out, void* ws, const PrefillPlan& plan, cudaStream_t s);
+cudaError_t launch_prepare_prefill_factors(const Ctx& c, cudaStream_t s);
+bool make_prefill_maps(Ctx* c);
 cudaError_t launch_prefill(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
                            const int32_t* cu_q, const int32_t* block_table, const int32_t* seq_lens,
                            int batch, int max_pages, int64_t total_q, int max_q_len,

@@ -48,7 +48,7 @@ __device__ inline bool seq_len_ok(const PrefillArgs& a, int L) {
 }
 
 // grid (chunk/32, h_kv, B), 256 threads: keys and values of 32 positions of one KV head.
-__global__ void __launch_bounds__(256) prefill_expand_kernel(PrefillArgs a, int c0) {
+__global__ void __launch_bounds__(256) prefill_simt_expand_kernel(PrefillArgs a, int c0) {
   __shared__ float Zk[32][65];
   __shared__ float Zv[32][33];
   __shared__ float Bs[32][128];
@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(256) prefill_expand_kernel(PrefillArgs a, int 
 }
 
 // grid (ceil(max_q_len/32), H, B), 256 threads = 32 queries x 8 lanes.
-__global__ void __launch_bounds__(256) prefill_attn_kernel(PrefillArgs a, int c0) {
+__global__ void __launch_bounds__(256) prefill_simt_attn_kernel(PrefillArgs a, int c0) {
   constexpr int KT = 16;  // keys per tile
   __shared__ float Qs[32][129];
   __shared__ float Ks[KT][129];
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(256) prefill_attn_kernel(PrefillArgs a, int c0
   }
 }
 
-__global__ void prefill_init_kernel(PrefillArgs a) {
+__global__ void prefill_simt_init_kernel(PrefillArgs a) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t n = a.total_q * a.H;
   if (idx >= n) return;
@@ -268,7 +268,7 @@ __global__ void prefill_init_kernel(PrefillArgs a) {
 }
 
 // one thread per (query row, head, dim); also validates the query spans
-__global__ void prefill_finalize_kernel(PrefillArgs a) {
+__global__ void prefill_simt_finalize_kernel(PrefillArgs a) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx == 0) {
     bool bad = a.cu_q[0] != 0 || a.cu_q[a.batch] != a.total_q;
@@ -287,7 +287,7 @@ __global__ void prefill_finalize_kernel(PrefillArgs a) {
   a.out[idx] = __float2bfloat16_rn(l > 0.f ? a.O[idx] / l : 0.f);
 }
 
-PrefillPlan plan_prefill(const Ctx& c, int batch, int max_pages, int64_t total_q) {
+PrefillPlan plan_prefill_simt(const Ctx& c, int batch, int max_pages, int64_t total_q) {
   PrefillPlan p;
   const int max_len = max_pages * kPage;
   p.chunk = 512;
@@ -301,10 +301,10 @@ PrefillPlan plan_prefill(const Ctx& c, int batch, int max_pages, int64_t total_q
   return p;
 }
 
-cudaError_t launch_prefill(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
-                           const int32_t* cu_q, const int32_t* block_table, const int32_t* seq_lens,
-                           int batch, int max_pages, int64_t total_q, int max_q_len,
-                           __nv_bfloat16* out, void* ws, const PrefillPlan& plan, cudaStream_t s) {
+cudaError_t launch_prefill_simt(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
+                                const int32_t* cu_q, const int32_t* block_table, const int32_t* seq_lens,
+                                int batch, int max_pages, int64_t total_q, int max_q_len,
+                                __nv_bfloat16* out, void* ws, const PrefillPlan& plan, cudaStream_t s) {
   if (batch == 0 || total_q == 0) return cudaSuccess;
   PrefillArgs a;
   a.key = c.key;
@@ -344,15 +344,34 @@ cudaError_t launch_prefill(const Ctx& c, const starkv_cache& cache, const __nv_b
   a.out = out;
   a.status = c.status;
   const int64_t nqh = total_q * a.H;
-  prefill_init_kernel<<<(unsigned)((nqh + 255) / 256), 256, 0, s>>>(a);
+  prefill_simt_init_kernel<<<(unsigned)((nqh + 255) / 256), 256, 0, s>>>(a);
   const int max_len = max_pages * kPage;
   for (int c0 = 0; c0 < max_len; c0 += plan.chunk) {
-    prefill_expand_kernel<<<dim3(plan.chunk / 32, a.h_kv, batch), 256, 0, s>>>(a, c0);
-    prefill_attn_kernel<<<dim3((max_q_len + 31) / 32, a.H, batch), 256, 0, s>>>(a, c0);
+    prefill_simt_expand_kernel<<<dim3(plan.chunk / 32, a.h_kv, batch), 256, 0, s>>>(a, c0);
+    prefill_simt_attn_kernel<<<dim3((max_q_len + 31) / 32, a.H, batch), 256, 0, s>>>(a, c0);
   }
   const int64_t tot = nqh * a.d;
-  prefill_finalize_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(a);
+  prefill_simt_finalize_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(a);
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Path selection: the tensor-core kernels (prefill_tc.cu) for every shape they
+// cover, the CUDA-core kernels above otherwise.
+// ---------------------------------------------------------------------------
+PrefillPlan plan_prefill(const Ctx& c, int batch, int max_pages, int64_t total_q) {
+  return c.tc_prefill ? plan_prefill_tc(c, batch, max_pages, total_q) : plan_prefill_simt(c, batch, max_pages, total_q);
+}
+
+cudaError_t launch_prefill(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
+                           const int32_t* cu_q, const int32_t* block_table, const int32_t* seq_lens,
+                           int batch, int max_pages, int64_t total_q, int max_q_len,
+                           __nv_bfloat16* out, void* ws, const PrefillPlan& plan, cudaStream_t s) {
+  if (c.tc_prefill)
+    return launch_prefill_tc(c, cache, q, cu_q, block_table, seq_lens, batch, max_pages, total_q, max_q_len, out, ws,
+                             plan, s);
+  return launch_prefill_simt(c, cache, q, cu_q, block_table, seq_lens, batch, max_pages, total_q, max_q_len, out, ws,
+                             plan, s);
 }
 
 }  // namespace starkv

@@ -213,8 +213,8 @@ def test_prefill_leg_line_counts_its_launches_and_copies(dry):
     pre = [e for e in log if e[0] == "prefill"]
     assert len(pre) == 2 * (warm + steps)                  # device-resident leg, then end to end
     assert all(e[2] == 2 * 24 and e[3] == 24 for e in pre)
-    # 64 positions in 4 pages: one key chunk; 48 appended tokens take the split-K append (2 kernels)
-    assert line["gpu_launches"] == (2 + 2 + 2) * steps
+    # 48 appended tokens take the split-K append (2 kernels); the prefill is re-expansion + attention
+    assert line["gpu_launches"] == (2 + 2) * steps
     assert line["e2e"]["unit"] == "TFLOP/s" and line["e2e"]["d2h_bytes_per_step"] == 48 * 4 * 64 * 2
     assert line["e2e"]["h2d_bytes_per_step"] >= 48 * 256 * 2 + 48 * 8 + 48 * 4 * 64 * 2
 

@@ -49,6 +49,59 @@ def test_tiny_prefill():
     check_attention(got, ref, "tiny prefill")
 
 
+def test_tiny_prefill_cuda_core_path(monkeypatch):
+    monkeypatch.setenv("STARKV_PREFILL_PATH", "simt")
+    w = gen.workload(0)
+    got, ref, st = run_prefill(w, [40, 0, 100], [9, 20, 37])
+    assert st == 0
+    check_attention(got, ref, "tiny prefill, CUDA-core path")
+
+
+def test_prefill_several_query_and_key_tiles():
+    # query tiles of 128 with a ragged last one, key tiles that straddle the
+    # chunk boundary, a sequence that is all chunk (no earlier context)
+    w = gen.workload(0)
+    got, ref, st = run_prefill(w, [700, 0, 129], [300, 257, 128])
+    assert st == 0
+    check_attention(got, ref, "tiny prefill, several tiles")
+
+
+def test_longchat_shapes_prefill_more_tiles():
+    w = gen.workload(4)
+    sel = {0: list(range(0, 260, 7)), 1: list(range(0, 131, 5))}
+    got, ref, st = run_prefill(w, [1000, 0], [260, 131], select=sel)
+    assert st == 0
+    check_attention(got, ref, "longchat prefill, several tiles (sampled)")
+
+
+def test_gqa_prefill_more_tiles():
+    w = gen.workload(3)
+    sel = {0: list(range(0, 200, 3))}
+    got, ref, st = run_prefill(w, [383], [200], select=sel)
+    assert st == 0
+    check_attention(got, ref, "gqa prefill, several tiles (sampled)")
+
+
+def test_prefill_bad_query_span_sets_status_and_zero_rows():
+    S = skv()
+    w = gen.workload(0)
+    kv, f = make_ctx(w, max_position=256)
+    try:
+        cfg, oc, bt, n_pages = oracle_cache(w, [50], extra_pages=1)
+        lc = kv.new_cache(n_pages)
+        upload(lc, oc)
+        q = bf16_tensor(gen.make_queries(8, w.H, w.d_h))
+        cu = torch.tensor([0, 8], dtype=torch.int32, device="cuda")
+        sl = torch.tensor([5], dtype=torch.int32, device="cuda")         # 8 queries but only 5 positions
+        out = torch.full_like(q, float("nan"))
+        S.starkv_prefill_attn(kv.ctx, lc.struct, q, cu, torch.from_numpy(bt).cuda(), sl, 8, out,
+                              kv.workspace(S.OP_PREFILL, 1, bt.shape[1], 8))
+        assert kv.status() & S.DEV_BAD_QUERY_SPAN
+        assert torch.all(out.float() == 0)
+    finally:
+        kv.close()
+
+
 def test_longchat_shapes_prefill_small():
     w = gen.workload(4)
     got, ref, st = run_prefill(w, [300, 17], [64, 33])

@@ -289,6 +289,12 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
                                CU_TENSOR_MAP_SWIZZLE_128B))
       c->app_splits = 0;  // the general append kernel serves every size
   }
+  const char* apath = getenv("STARKV_APPEND_PATH");
+  const bool want_simt_append = apath && strcmp(apath, "simt") == 0;
+  c->tc_append = !want_simt_append && tc_append_supported(*c) &&
+                 starkv::encode_map_2d(&c->a_map64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->A, (uint64_t)c->lat_cols,
+                                       (uint64_t)cfg->hidden, (uint64_t)c->lat_cols * 2, 64, 64,
+                                       CU_TENSOR_MAP_SWIZZLE_128B);
   *out = reinterpret_cast<starkv_ctx*>(c);
   return ok();
 }

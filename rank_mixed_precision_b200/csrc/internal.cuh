@@ -55,6 +55,8 @@ struct Ctx {
   CUtensorMap bk_map;     // TMA map of Bk16 as [h_kv*r_k][d_h]: box 64 x r_k, 128-byte swizzle
   CUtensorMap bvp_map;    // TMA map of Bv16p: box 64 x 64, 128-byte swizzle
   bool tc_prefill;        // tensor-core prefill available for this shape
+  CUtensorMap a_map64;    // TMA map of `A`: box 64 columns x 64 rows, 128-byte swizzle (tensor-core append)
+  bool tc_append;         // tensor-core append (more than 64 tokens) available
 };
 
 // 2-D TMA map over a row-major [rows][inner] array (no interleave, zero fill).
@@ -244,6 +246,37 @@ __device__ inline float2 unpack_meta(uint32_t m) {
 }
 
 // ---------------------------------------------------------------------------
+// Rotate + quantise + store one group of one token (shared by append and the
+// quantise entry).  x: the group's g pre-rotation latents.
+// ---------------------------------------------------------------------------
+template <int G>
+__device__ inline void rotate_quantize_store(const float* x_in, const LatentGeom& L, int gi,
+                                             uint8_t* region, uint32_t* meta_page, int t,
+                                             unsigned int* status) {
+  float x[G];
+#pragma unroll
+  for (int i = 0; i < G; ++i) x[i] = x_in[i];
+  fwht_fl32<G>(x);
+  uint8_t code[G];
+  __half s16, zp16;
+  const int bits = gi < L.top_groups ? 4 : 3;
+  if (!quantize_group<G>(x, bits, code, s16, zp16)) set_status(status, STARKV_DEV_QUANT_OVERFLOW);
+  store_group_codes<G>(region, L, gi, t, code);
+  const uint32_t m = (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(zp16) << 16);
+  meta_page[gi * kPage + t] = m;
+}
+
+__device__ inline void rotate_quantize_store_any(const float* x, const LatentGeom& L, int gi,
+                                                 uint8_t* region, uint32_t* meta_page, int t,
+                                                 unsigned int* status) {
+  switch (L.g) {
+    case 4: rotate_quantize_store<4>(x, L, gi, region, meta_page, t, status); break;
+    case 8: rotate_quantize_store<8>(x, L, gi, region, meta_page, t, status); break;
+    default: rotate_quantize_store<16>(x, L, gi, region, meta_page, t, status); break;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Launchers (defined in the .cu files)
 // ---------------------------------------------------------------------------
 cudaError_t launch_prepare_factors(const Ctx& c, const __nv_bfloat16* Bk, const __nv_bfloat16* Bv,
@@ -299,6 +332,10 @@ cudaError_t launch_prefill_tc(const Ctx& c, const starkv_cache& cache, const __n
                               int batch, int max_pages, int64_t total_q, int max_q_len,
                               __nv_bfloat16* out, void* ws, const PrefillPlan& plan, cudaStream_t s);
 cudaError_t launch_prepare_prefill_factors(const Ctx& c, cudaStream_t s);
+// tensor-core append of more than kSmallAppend tokens (append_tc.cu)
+bool tc_append_supported(const Ctx& c);
+cudaError_t launch_append_tc(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* X, const int64_t* slots,
+                             int64_t n, float* latents_out, cudaStream_t s);
 bool make_prefill_maps(Ctx* c);
 cudaError_t launch_prefill(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
                            const int32_t* cu_q, const int32_t* block_table, const int32_t* seq_lens,

@@ -51,37 +51,6 @@ cudaError_t launch_prepare_factors(const Ctx& c, const __nv_bfloat16* Bk, const 
 }
 
 // ---------------------------------------------------------------------------
-// Rotate + quantise + store one group of one token (shared by append and the
-// quantise entry).  x: the group's g pre-rotation latents.
-// ---------------------------------------------------------------------------
-template <int G>
-__device__ inline void rotate_quantize_store(const float* x_in, const LatentGeom& L, int gi,
-                                             uint8_t* region, uint32_t* meta_page, int t,
-                                             unsigned int* status) {
-  float x[G];
-#pragma unroll
-  for (int i = 0; i < G; ++i) x[i] = x_in[i];
-  fwht_fl32<G>(x);
-  uint8_t code[G];
-  __half s16, zp16;
-  const int bits = gi < L.top_groups ? 4 : 3;
-  if (!quantize_group<G>(x, bits, code, s16, zp16)) set_status(status, STARKV_DEV_QUANT_OVERFLOW);
-  store_group_codes<G>(region, L, gi, t, code);
-  const uint32_t m = (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(zp16) << 16);
-  meta_page[gi * kPage + t] = m;
-}
-
-__device__ inline void rotate_quantize_store_any(const float* x, const LatentGeom& L, int gi,
-                                                 uint8_t* region, uint32_t* meta_page, int t,
-                                                 unsigned int* status) {
-  switch (L.g) {
-    case 4: rotate_quantize_store<4>(x, L, gi, region, meta_page, t, status); break;
-    case 8: rotate_quantize_store<8>(x, L, gi, region, meta_page, t, status); break;
-    default: rotate_quantize_store<16>(x, L, gi, region, meta_page, t, status); break;
-  }
-}
-
-// ---------------------------------------------------------------------------
 // Quantise/pack entry: one thread per (token, group).  The pages are zeroed
 // by the launcher first.
 // ---------------------------------------------------------------------------
@@ -424,6 +393,8 @@ cudaError_t launch_append(const Ctx& c, const starkv_cache& cache, const __nv_bf
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
+  if (c.tc_append && (reinterpret_cast<uintptr_t>(X) & 15) == 0)
+    return launch_append_tc(c, cache, X, slots, n, latents_out, s);
   dim3 grid((unsigned)((n + kAppBM - 1) / kAppBM), (unsigned)((c.lat_cols + kAppBN - 1) / kAppBN));
   append_kernel<<<grid, 256, 0, s>>>(a);
   return cudaGetLastError();

@@ -39,7 +39,6 @@ using namespace sm100;
 
 namespace {
 constexpr int kTile = 128;                 // positions per tile (keys and queries)
-constexpr int kXThreads = 256;             // expand kernel
 constexpr int kQThreads = 192;             // attention kernel: producer, MMA, 4 softmax warps
 constexpr float kLog2eQ = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;        // move the running maximum when it grows by more than 2^8
@@ -72,29 +71,55 @@ struct ExpandArgs {
   __half* Kx;          // [B][h_kv][tpad][d] RoPE'd keys
   __half* Vx;          // [B][h_kv][tpad][d] values
   unsigned int* status;
-  uint32_t off_ak, off_bk, off_av, off_bv, off_bar, bk_head, bv_stage;
+  // shared-memory layout (bytes from the 1024-aligned base)
+  uint32_t off_ak, off_bk, off_kc, off_av, off_bv, off_vc, off_bar;
+  uint32_t bk_head, bv_stage;
+  uint32_t kc_codes, kc_page;      // key codes of one page of one head (bytes); a page's codes + meta pitch
+  uint32_t vc_codes_max, vc_page;  // value codes of one chunk of one page (at most); codes + meta pitch
 };
 
-// grid (tpad / 128, ceil(h_kv / HP), B), 256 threads.
+constexpr int kXWarps = 10;        // 8 dequant/epilogue warps, a copy warp, an MMA warp
+constexpr int kXStages = 4;        // value code stages
+constexpr int kXThreadsW = kXWarps * 32;
+
+// Bytes of value group tiles [4c, 4c + 4) of a page region and their offset.
+__device__ __forceinline__ void value_chunk_span(const LatentGeom& V, int c, uint32_t& off, uint32_t& bytes) {
+  const int g0 = 4 * c;
+  off = (uint32_t)tile_offset(V, g0);
+  bytes = (uint32_t)tile_offset(V, g0 + 4) - off;
+}
+
+// grid (tpad / 128, ceil(h_kv / HP), B), 320 threads:
+//   warps 0..7  dequantise latents from the staged pages into the MMA's A tiles,
+//               then the epilogue (two warps per TMEM lane quarter)
+//   warp 8      copies: the tile's key pages, then per 64-channel value chunk the
+//               8 pages' code tiles and metadata (one lane per bulk copy), and the
+//               B'_k / B'_v tiles by TMA
+//   warp 9      one thread issues every tcgen05 MMA
 //   TMEM columns [0, HP d): V accumulators; [256, 256 + HP d): K accumulators.
-__global__ void __launch_bounds__(kXThreads, 1)
+__global__ void __launch_bounds__(kXThreadsW, 1)
     prefill_expand_kernel(const __grid_constant__ CUtensorMap bk_map, const __grid_constant__ CUtensorMap bv_map,
                           const ExpandArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024p(smem_raw);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + a.off_bar);
-  uint64_t* bkfull = bar;       // B'_k tiles landed
-  uint64_t* bvfull = bar + 1;   // [2] B'_v chunk landed
-  uint64_t* mdone = bar + 3;    // [2] MMAs of a value chunk done (its operand slots are free)
-  uint64_t* alldone = bar + 5;  // every MMA of the CTA done
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 6);
-  int* pg = reinterpret_cast<int*>(bar + 7);  // [8] page ids of the tile (-1: none)
-  int* failed = pg + 8;
+  uint64_t* kfull = bar;                    // key pages + B'_k landed
+  uint64_t* kready = bar + 1;               // key A tiles written (8 warps)
+  uint64_t* cfull = bar + 2;                // [kXStages] value code stage landed
+  uint64_t* cempty = cfull + kXStages;      // [kXStages] value code stage read (8 warps)
+  uint64_t* bfull = cempty + kXStages;      // [2] B'_v chunk landed
+  uint64_t* afull = bfull + 2;              // [2] value A tile written (8 warps)
+  uint64_t* aempty = afull + 2;             // [2] MMAs of a chunk done (A tile and B'_v slot free)
+  uint64_t* alldone = aempty + 2;           // every MMA done
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(alldone + 1);
+  int* pg = reinterpret_cast<int*>(alldone + 2);  // [8] page ids of the tile (-1: none)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x, kv0 = blockIdx.y * a.HP, b = blockIdx.z;
   const int nh = min(a.HP, a.h_kv - kv0);
   const int d = a.d, nsub = d / 64;
   const int rk = a.key.r;
+  const LatentGeom& V = a.val;
+  const int nchunk = V.r / 64;
   // first kernel of the call: its inputs may come from any earlier kernel
   pdl_wait();
   pdl_launch_dependents();
@@ -104,15 +129,20 @@ __global__ void __launch_bounds__(kXThreads, 1)
     return;
   }
   if (tile * kTile >= L) return;
-  if (warp == 0) tmem_alloc(tslot, 512);
+  if (warp == 9) tmem_alloc(tslot, 512);
   if (tid == 0) {
-    mbar_init(bkfull, 1);
+    mbar_init(kfull, 1);
+    mbar_init(kready, 8);
+    for (int s = 0; s < kXStages; ++s) {
+      mbar_init(&cfull[s], 1);
+      mbar_init(&cempty[s], 8);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bvfull[s], 1);
-      mbar_init(&mdone[s], 1);
+      mbar_init(&bfull[s], 1);
+      mbar_init(&afull[s], 8);
+      mbar_init(&aempty[s], 1);
     }
     mbar_init(alldone, 1);
-    *failed = 0;
     fence_mbar_init();
   }
   if (tid < kTile / kPage) {
@@ -131,113 +161,176 @@ __global__ void __launch_bounds__(kXThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const int nchunk = a.val.r / 64;
   uint8_t* Ak = sm + a.off_ak;
   uint8_t* Bk = sm + a.off_bk;
+  uint8_t* Kc = sm + a.off_kc;
   uint8_t* Av = sm + a.off_av;
   uint8_t* Bv = sm + a.off_bv;
-  auto issue_bv = [&](int c) {
-    const int slot = c & 1;
-    mbar_arrive_expect_tx(&bvfull[slot], (uint32_t)(nh * nsub) * 8192u);
-    for (int i = 0; i < nh * nsub; ++i)
-      tma_load_2d(Bv + slot * a.bv_stage + i * 8192, &bv_map, kv0 * d + i * 64, c * 64, &bvfull[slot]);
-  };
-  if (tid == 0) {
-    mbar_arrive_expect_tx(bkfull, (uint32_t)(nh * nsub * rk * 128));
-    for (int hh = 0; hh < nh; ++hh)
-      for (int i = 0; i < nsub; ++i)
-        tma_load_2d(Bk + hh * a.bk_head + i * rk * 128, &bk_map, i * 64, (kv0 + hh) * rk, bkfull);
-    for (int c = 0; c < 2 && c < nchunk; ++c) issue_bv(c);
-  }
-  // ---- key latents of the tile, dequantised into K-major (row = position) fp16 tiles
-  for (int hh = 0; hh < nh; ++hh) {
-    uint8_t* tileA = Ak + hh * (kTile * 128);
-    for (int e = tid; e < kTile * rk; e += kXThreads) {
-      const int t = e / rk, c = e % rk;
-      const int pid = pg[t / kPage];
-      float z = 0.f;
-      if (pid >= 0 && tile * kTile + t < L) {
-        const int t16 = t % kPage, gi = c / a.key.g;
-        const int64_t reg = (int64_t)pid * a.h_kv + kv0 + hh;
-        const float2 sz = unpack_meta(a.k_meta[(reg * a.key.groups + gi) * kPage + t16]);
-        z = __fmaf_rn((float)load_code(a.k_codes + reg * a.key.region_bytes, a.key, gi, t16, c % a.key.g), sz.x, sz.y);
-      }
-      *reinterpret_cast<__half*>(tileA + sw128_kmajor_offset(t, c, kTile)) = __float2half_rn(z);
-    }
-  }
-  fence_async_smem();
-  __syncthreads();
-  const uint32_t idesc_k = make_idesc_f16(128, d, false, true);
-  const uint32_t idesc_v = make_idesc_f16(128, nh * d, false, true);
-  if (tid == 0) {
-    if (mbar_wait(bkfull, 0)) {
-      tc_fence_after();
+  uint8_t* Vc = sm + a.off_vc;
+  const uint32_t vstage = 8 * a.vc_page;
+  bool ok = true;
+
+  if (warp == 8) {
+    // ---------------- copies ----------------
+    const int npg = __popc(__ballot_sync(0xffffffffu, lane < 8 && pg[lane < 8 ? lane : 0] >= 0));
+    // key pages of the CTA's heads: codes (padded region) and metadata, one lane per copy
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kfull, (uint32_t)(npg * nh) * (a.kc_codes + (uint32_t)a.key.groups * kPage * 4) +
+                                       (uint32_t)(nh * nsub * rk * 128));
       for (int hh = 0; hh < nh; ++hh)
-        for (int ks = 0; ks < rk / 16; ++ks)
-          mma_f16(tmem + 256 + hh * d, make_sdesc(smem_u32(Ak + hh * kTile * 128) + ks * 32, 16, 1024, 2),
-                  make_sdesc(smem_u32(Bk + hh * a.bk_head) + ks * 2048, rk * 128, 1024, 2), idesc_k, ks > 0);
-    } else {
-      *failed = 1;
+        for (int i = 0; i < nsub; ++i)
+          tma_load_2d(Bk + hh * a.bk_head + i * rk * 128, &bk_map, i * 64, (kv0 + hh) * rk, kfull);
     }
-  }
-  // ---- value chunks of 64 latent channels (4 groups of 16)
-  for (int c = 0; c < nchunk; ++c) {
-    const int slot = c & 1;
-    if (c >= 2) {
-      // the MMAs of chunk c - 2 read this slot's operands
-      if (!__all_sync(0xffffffffu, mbar_wait(&mdone[slot], ((c - 2) >> 1) & 1))) {
-        if (lane == 0) *failed = 1;
-      }
-      __syncthreads();
-      if (*failed) break;
-      if (tid == 0) issue_bv(c);
+    __syncwarp();
+    for (int e = lane; e < 2 * 8 * nh; e += 32) {
+      const int p = (e >> 1) % 8, hh = (e >> 1) / 8;
+      const int pid = pg[p];
+      if (pid < 0) continue;
+      const int64_t reg = (int64_t)pid * a.h_kv + kv0 + hh;
+      uint8_t* dst = Kc + (hh * 8 + p) * a.kc_page;
+      if ((e & 1) == 0)
+        bulk_g2s(dst, a.k_codes + reg * a.key.region_bytes, a.kc_codes, kfull);
+      else
+        bulk_g2s(dst + a.kc_codes, a.k_meta + reg * a.key.groups * kPage, (uint32_t)a.key.groups * kPage * 4, kfull);
     }
-    uint8_t* tileA = Av + slot * (kTile * 128);
-    for (int e = tid; e < kTile * 4; e += kXThreads) {
-      const int t = e >> 2, gq = e & 3;
-      const int gi = c * 4 + gq;
-      const int pid = pg[t / kPage];
-      uint4 c0 = make_uint4(0, 0, 0, 0), c1 = make_uint4(0, 0, 0, 0);
-      if (pid >= 0 && tile * kTile + t < L) {
-        const int t16 = t % kPage;
-        const uint8_t* region = a.v_codes + (int64_t)pid * a.val.region_bytes;
-        const uint32_t mw = a.v_meta[((int64_t)pid * a.val.groups + gi) * kPage + t16];
-        if (gi < a.val.top_groups)
-          dequant16_4bit(region + gi * 128 + 8 * t16, mw, c0, c1);
-        else
-          dequant16_3bit(region + a.val.top_groups * 128 + (gi - a.val.top_groups) * 96, t16, mw, c0, c1);
+    // value chunks
+    for (int c = 0; c < nchunk; ++c) {
+      const int s = c % kXStages;
+      const uint32_t ph = (c / kXStages) & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&cempty[s], ph ^ 1))) {
+        ok = false;
+        break;
       }
-      *reinterpret_cast<uint4*>(tileA + sw128_kmajor_offset(t, gq * 16, kTile)) = c0;
-      *reinterpret_cast<uint4*>(tileA + sw128_kmajor_offset(t, gq * 16 + 8, kTile)) = c1;
+      uint32_t coff, cbytes;
+      value_chunk_span(V, c, coff, cbytes);
+      if (lane == 0) mbar_arrive_expect_tx(&cfull[s], (uint32_t)npg * (cbytes + 4 * kPage * 4));
+      __syncwarp();
+      if (lane < 16) {
+        const int p = lane >> 1;
+        const int pid = pg[p];
+        if (pid >= 0) {
+          uint8_t* dst = Vc + s * vstage + p * a.vc_page;
+          if ((lane & 1) == 0)
+            bulk_g2s(dst, a.v_codes + (int64_t)pid * V.region_bytes + coff, cbytes, &cfull[s]);
+          else
+            bulk_g2s(dst + a.vc_codes_max, a.v_meta + ((int64_t)pid * V.groups + 4 * c) * kPage, 4 * kPage * 4,
+                     &cfull[s]);
+        }
+      }
+      const int bs = c & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&aempty[bs], ((c >> 1) & 1) ^ 1))) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bfull[bs], (uint32_t)(nh * nsub) * 8192u);
+        for (int i = 0; i < nh * nsub; ++i)
+          tma_load_2d(Bv + bs * a.bv_stage + i * 8192, &bv_map, kv0 * d + i * 64, c * 64, &bfull[bs]);
+      }
+      __syncwarp();
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc_k = make_idesc_f16(128, d, false, true);
+      const uint32_t idesc_v = make_idesc_f16(128, nh * d, false, true);
+      if (mbar_wait(kfull, 0) && mbar_wait(kready, 0)) {
+        tc_fence_after();
+        for (int hh = 0; hh < nh; ++hh)
+          for (int ks = 0; ks < rk / 16; ++ks)
+            mma_f16(tmem + 256 + hh * d, make_sdesc(smem_u32(Ak + hh * kTile * 128) + ks * 32, 16, 1024, 2),
+                    make_sdesc(smem_u32(Bk + hh * a.bk_head) + ks * 2048, rk * 128, 1024, 2), idesc_k, ks > 0);
+      } else {
+        ok = false;
+      }
+      for (int c = 0; ok && c < nchunk; ++c) {
+        const int bs = c & 1;
+        const uint32_t ph = (c >> 1) & 1;
+        if (!mbar_wait(&afull[bs], ph) || !mbar_wait(&bfull[bs], ph)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t aa = smem_u32(Av + bs * (kTile * 128));
+        const uint32_t ba = smem_u32(Bv + bs * a.bv_stage);
+        for (int ks = 0; ks < 4; ++ks)
+          mma_f16(tmem, make_sdesc(aa + ks * 32, 16, 1024, 2), make_sdesc(ba + ks * 2048, 8192, 1024, 2), idesc_v,
+                  (c > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&aempty[bs]);
+      }
+      mma_commit(alldone);  // arrives once every MMA issued above has completed
+    }
+  } else {
+    // ---------------- dequantisation (warps 0..7) ----------------
+    // key latents: thread item = (position, channel), from the staged pages
+    if (!__all_sync(0xffffffffu, mbar_wait(kfull, 0))) ok = false;
+    if (ok) {
+      for (int hh = 0; hh < nh; ++hh) {
+        uint8_t* tileA = Ak + hh * (kTile * 128);
+        for (int e = tid; e < kTile * rk; e += 256) {
+          const int t = e / rk, c = e % rk;
+          const int p = t / kPage;
+          float z = 0.f;
+          if (pg[p] >= 0 && tile * kTile + t < L) {
+            const int t16 = t % kPage, gi = c / a.key.g;
+            const uint8_t* page = Kc + (hh * 8 + p) * a.kc_page;
+            const float2 sz = unpack_meta(reinterpret_cast<const uint32_t*>(page + a.kc_codes)[gi * kPage + t16]);
+            z = __fmaf_rn((float)load_code(page, a.key, gi, t16, c % a.key.g), sz.x, sz.y);
+          }
+          *reinterpret_cast<__half*>(tileA + sw128_kmajor_offset(t, c, kTile)) = __float2half_rn(z);
+        }
+      }
     }
     fence_async_smem();
-    __syncthreads();
-    if (tid == 0 && !*failed) {
-      if (mbar_wait(&bvfull[slot], (c >> 1) & 1)) {
-        tc_fence_after();
-        for (int ks = 0; ks < 4; ++ks)
-          mma_f16(tmem, make_sdesc(smem_u32(tileA) + ks * 32, 16, 1024, 2),
-                  make_sdesc(smem_u32(Bv + slot * a.bv_stage) + ks * 2048, 8192, 1024, 2), idesc_v,
-                  (c > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&mdone[slot]);
-      } else {
-        *failed = 1;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(kready);
+    // value chunks: thread item = (position, 16-channel group)
+    for (int c = 0; ok && c < nchunk; ++c) {
+      const int s = c % kXStages;
+      const int bs = c & 1;
+      const bool got = mbar_wait(&cfull[s], (c / kXStages) & 1) && mbar_wait(&aempty[bs], ((c >> 1) & 1) ^ 1);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      uint8_t* tileA = Av + bs * (kTile * 128);
+      const uint8_t* st = Vc + s * vstage;
+#pragma unroll
+      for (int it = 0; it < 2; ++it) {
+        const int e = tid + it * 256;
+        const int t = e >> 2, gq = e & 3;
+        const int gi = c * 4 + gq;
+        const int p = t / kPage, t16 = t % kPage;
+        uint4 c0 = make_uint4(0, 0, 0, 0), c1 = make_uint4(0, 0, 0, 0);
+        if (pg[p] >= 0 && tile * kTile + t < L) {
+          const uint8_t* page = st + p * a.vc_page;
+          const uint32_t mw = reinterpret_cast<const uint32_t*>(page + a.vc_codes_max)[gq * kPage + t16];
+          const uint32_t toff = (uint32_t)(tile_offset(V, gi) - tile_offset(V, c * 4));
+          if (gi < V.top_groups)
+            dequant16_4bit(page + toff + 8 * t16, mw, c0, c1);
+          else
+            dequant16_3bit(page + toff, t16, mw, c0, c1);
+        }
+        *reinterpret_cast<uint4*>(tileA + sw128_kmajor_offset(t, gq * 16, kTile)) = c0;
+        *reinterpret_cast<uint4*>(tileA + sw128_kmajor_offset(t, gq * 16 + 8, kTile)) = c1;
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&cempty[s]);
+        mbar_arrive(&afull[bs]);
       }
     }
   }
-  if (tid == 0) mma_commit(alldone);  // arrives once every MMA issued above has completed
+  // ---------------- epilogue (warps 0..7) ----------------
   const bool done = __all_sync(0xffffffffu, mbar_wait(alldone, 0));
-  __syncthreads();
-  const bool ok = done && !*failed;
-  if (!ok && tid == 0) set_status(a.status, kDevWaitTimeout);
+  if (!(done && ok) && lane == 0) set_status(a.status, kDevWaitTimeout);
   tc_fence_after();
-  // ---- epilogue: thread = position (TMEM lane), the two warps of a lane
-  // quarter split the frequency pairs (i, i + d/2)
-  {
+  if (warp < 8) {
     const int q4 = warp & 3, half = warp >> 2;
     const int t = q4 * 32 + lane;
     const int p = tile * kTile + t;
-    const bool valid = ok && p < L && pg[t / kPage] >= 0;
+    const bool valid = done && ok && p < L && pg[t / kPage] >= 0;
     const uint32_t lrow = (uint32_t)(q4 * 32) << 16;
     const int hd = d / 2;
     for (int hh = 0; hh < nh; ++hh) {
@@ -254,9 +347,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
         tmem_ld_wait();
         uint32_t vo0[8], vo1[8], ko0[8], ko1[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          vo0[u] = vo1[u] = ko0[u] = ko1[u] = 0u;
-        }
+        for (int u = 0; u < 8; ++u) vo0[u] = vo1[u] = ko0[u] = ko1[u] = 0u;
         if (valid) {
           const float2* cs = a.rope + (int64_t)p * hd + i0;
 #pragma unroll
@@ -270,26 +361,24 @@ __global__ void __launch_bounds__(kXThreads, 1)
             ko1[u / 2] = pack_half2(b0 * c2.x + a0 * c2.y, b1 * c2.z + a1 * c2.w);
           }
         }
-        if (p < a.tpad) {
-          uint4* kd0 = reinterpret_cast<uint4*>(krow + i0);
-          uint4* kd1 = reinterpret_cast<uint4*>(krow + hd + i0);
-          uint4* vd0 = reinterpret_cast<uint4*>(vrow + i0);
-          uint4* vd1 = reinterpret_cast<uint4*>(vrow + hd + i0);
-          kd0[0] = make_uint4(ko0[0], ko0[1], ko0[2], ko0[3]);
-          kd0[1] = make_uint4(ko0[4], ko0[5], ko0[6], ko0[7]);
-          kd1[0] = make_uint4(ko1[0], ko1[1], ko1[2], ko1[3]);
-          kd1[1] = make_uint4(ko1[4], ko1[5], ko1[6], ko1[7]);
-          vd0[0] = make_uint4(vo0[0], vo0[1], vo0[2], vo0[3]);
-          vd0[1] = make_uint4(vo0[4], vo0[5], vo0[6], vo0[7]);
-          vd1[0] = make_uint4(vo1[0], vo1[1], vo1[2], vo1[3]);
-          vd1[1] = make_uint4(vo1[4], vo1[5], vo1[6], vo1[7]);
-        }
+        uint4* kd0 = reinterpret_cast<uint4*>(krow + i0);
+        uint4* kd1 = reinterpret_cast<uint4*>(krow + hd + i0);
+        uint4* vd0 = reinterpret_cast<uint4*>(vrow + i0);
+        uint4* vd1 = reinterpret_cast<uint4*>(vrow + hd + i0);
+        kd0[0] = make_uint4(ko0[0], ko0[1], ko0[2], ko0[3]);
+        kd0[1] = make_uint4(ko0[4], ko0[5], ko0[6], ko0[7]);
+        kd1[0] = make_uint4(ko1[0], ko1[1], ko1[2], ko1[3]);
+        kd1[1] = make_uint4(ko1[4], ko1[5], ko1[6], ko1[7]);
+        vd0[0] = make_uint4(vo0[0], vo0[1], vo0[2], vo0[3]);
+        vd0[1] = make_uint4(vo0[4], vo0[5], vo0[6], vo0[7]);
+        vd1[0] = make_uint4(vo1[0], vo1[1], vo1[2], vo1[3]);
+        vd1[1] = make_uint4(vo1[4], vo1[5], vo1[6], vo1[7]);
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -634,7 +723,8 @@ bool tc_prefill_supported(const Ctx& c) {
 namespace {
 struct XLayout {
   int HP;
-  uint32_t off_ak, off_bk, off_av, off_bv, off_bar, bk_head, bv_stage;
+  uint32_t off_ak, off_bk, off_kc, off_av, off_bv, off_vc, off_bar, bk_head, bv_stage;
+  uint32_t kc_codes, kc_page, vc_codes_max, vc_page;
   size_t smem;
 };
 
@@ -644,6 +734,11 @@ XLayout expand_layout(const Ctx& c) {
   x.HP = c.cfg.num_kv_heads % 2 == 0 ? 2 : 1;
   x.bk_head = (uint32_t)(d / 64) * rk * 128;
   x.bv_stage = (uint32_t)(x.HP * d / 64) * 8192;
+  x.kc_codes = (uint32_t)c.key.region_bytes;                        // a multiple of 16
+  x.kc_page = x.kc_codes + (uint32_t)c.key.groups * kPage * 4;
+  // the largest 4-group span of the value region (all 4-bit groups)
+  x.vc_codes_max = 4 * 8 * (uint32_t)c.val.g;
+  x.vc_page = x.vc_codes_max + 4 * kPage * 4;
   uint32_t o = 0;
   x.off_ak = o;
   o += x.HP * kTile * 128;
@@ -653,8 +748,12 @@ XLayout expand_layout(const Ctx& c) {
   o += 2 * kTile * 128;
   x.off_bv = o;
   o += 2 * x.bv_stage;
-  x.off_bar = o;
-  o += 128;
+  x.off_kc = o;
+  o += (uint32_t)x.HP * 8 * x.kc_page;
+  x.off_vc = (o + 127) / 128 * 128;
+  o = x.off_vc + kXStages * 8 * x.vc_page;
+  x.off_bar = (o + 15) / 16 * 16;
+  o = x.off_bar + 256;
   x.smem = o + 1024;
   return x;
 }
@@ -761,15 +860,21 @@ cudaError_t launch_prefill_tc(const Ctx& c, const starkv_cache& cache, const __n
     a.status = c.status;
     a.off_ak = x.off_ak;
     a.off_bk = x.off_bk;
+    a.off_kc = x.off_kc;
     a.off_av = x.off_av;
     a.off_bv = x.off_bv;
+    a.off_vc = x.off_vc;
     a.off_bar = x.off_bar;
     a.bk_head = x.bk_head;
     a.bv_stage = x.bv_stage;
+    a.kc_codes = x.kc_codes;
+    a.kc_page = x.kc_page;
+    a.vc_codes_max = x.vc_codes_max;
+    a.vc_page = x.vc_page;
     e = cudaFuncSetAttribute(prefill_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)x.smem);
     if (e != cudaSuccess) return e;
     e = launch_chained(prefill_expand_kernel, dim3(tpad / kTile, (f.num_kv_heads + x.HP - 1) / x.HP, batch),
-                       dim3(kXThreads), x.smem, s, 1u, c.bk_map, c.bvp_map, a);
+                       dim3(kXThreadsW), x.smem, s, 1u, c.bk_map, c.bvp_map, a);
     if (e != cudaSuccess) return e;
   }
   // ---- B: attention

@@ -463,6 +463,63 @@ def decode(cache: Cache, q, B_k, B_v, block_table, seq_lens, seqs=None, heads=No
     return out
 
 
+def decode_slice(cache: Cache, q, B_k, B_v, block_table, seq_lens, key_pos0, q_pos, heads=None):
+    """starkv_decode_attn_slice: sequence b's cache holds one slice of its context,
+    seq_lens[b] tokens at positions key_pos0[b] .. key_pos0[b] + seq_lens[b] - 1
+    (block-table row from local index 0), and its query sits at q_pos[b].  The
+    query attends to the slice alone ([CaliDrop] attention decomposition theorem,
+    eq. 1: partials of disjoint key subsets merge exactly).
+
+    Returns (o [B, H, d_h] normalised within the slice, m [B, H], l [B, H]) in
+    natural-log units: m = max_j s_j, l = sum_j e^(s_j - m); an empty slice gives
+    (0, -inf, 0).  NaN where not requested by ``heads``.
+    """
+    cfg = cache.cfg
+    q = np.asarray(q)
+    Bn = q.shape[0]
+    d = cfg.d_h
+    heads = list(range(cfg.H)) if heads is None else list(heads)
+    o = np.full((Bn, cfg.H, d), np.nan)
+    m = np.full((Bn, cfg.H), np.nan)
+    l = np.full((Bn, cfg.H), np.nan)
+    B_k = np.asarray(B_k, np.float64)
+    B_v = np.asarray(B_v, np.float64)
+    for b in range(Bn):
+        n = int(seq_lens[b])
+        if n == 0:
+            o[b, heads], m[b, heads], l[b, heads] = 0.0, -np.inf, 0.0
+            continue
+        zk, zv = gather_sequence(cache, block_table[b], n)
+        zk = unrotate_fp64(zk, cfg.key.g)
+        zv = unrotate_fp64(zv, cfg.val.g)
+        pos = int(key_pos0[b]) + np.arange(n)
+        for h in heads:
+            kv = h // cfg.group
+            k = rope(zk[:, kv] @ B_k[kv], pos, cfg.rope_base)
+            qr = rope(np.asarray(q[b, h], np.float64), int(q_pos[b]), cfg.rope_base)
+            s = (k @ qr) / np.sqrt(d)
+            mb, lb, acc = partial_softmax(s, zv)
+            o[b, h] = (acc / lb) @ B_v[:, kv * d:(kv + 1) * d]
+            m[b, h], l[b, h] = mb, lb
+    return o, m, l
+
+
+def merge_slices(o_parts, m_parts, l_parts):
+    """Combine slice results of the same queries (the partition identity):
+    o = sum_r e^(m_r - M) l_r o_r / sum_r e^(m_r - M) l_r, M = max_r m_r over the
+    non-empty slices.  Inputs stacked on a leading slice axis: o [n, ..., d],
+    m and l [n, ...].  All slices empty: zeros."""
+    o_parts = np.asarray(o_parts, np.float64)
+    m_parts = np.asarray(m_parts, np.float64)
+    l_parts = np.asarray(l_parts, np.float64)
+    live = l_parts > 0
+    M = np.where(live, m_parts, -np.inf).max(axis=0)
+    w = np.where(live, np.exp(np.where(live, m_parts, 0.0) - np.where(np.isfinite(M), M, 0.0)) * l_parts, 0.0)
+    den = w.sum(axis=0)
+    num = (w[..., None] * o_parts).sum(axis=0)
+    return np.where(den[..., None] > 0, num / np.where(den > 0, den, 1.0)[..., None], 0.0)
+
+
 def prefill(cache: Cache, q, cu_q, B_k, B_v, block_table, seq_lens, select=None, heads=None):
     """starkv_prefill_attn: query i of sequence b (cu_q[b] <= row < cu_q[b+1]) sits at
     position seq_len_b - n_b + i and attends causally to positions <= its own.

@@ -200,3 +200,76 @@ def test_empty_sequence_decodes_to_zero_row():
     cache = O.new_cache(cfg, 1)
     q = gen.make_queries(1, w.H, w.d_h)
     assert np.all(O.decode(cache, q, f.B_k, f.B_v, np.zeros((1, 1), np.int32), [0]) == 0)
+
+
+def _slice_case(w, n, cuts, seed=0):
+    """One sequence of n tokens written whole into one cache and, slice by slice,
+    into one cache per slice (each slice's pages from local index 0)."""
+    cfg = O.config_of(w)
+    zk, zv = gen.make_latents(w, n, seed)
+    bt, n_pages = gen.make_block_table([n], seed)
+    whole = O.new_cache(cfg, n_pages)
+    O.write_latents(whole, gen.slots_for(bt, 0, np.arange(n)), zk, zv)
+    slices = []
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        sbt, sp = gen.make_block_table([max(hi - lo, 1)], seed + lo + 1)
+        c = O.new_cache(cfg, sp)
+        if hi > lo:
+            O.write_latents(c, gen.slots_for(sbt, 0, np.arange(hi - lo)), zk[lo:hi], zv[lo:hi])
+        slices.append((c, sbt, lo, hi))
+    return cfg, whole, bt, slices
+
+
+@pytest.mark.parametrize("wi", [0, 3])
+def test_slices_merge_to_the_whole_decode(wi):
+    # [CaliDrop] eq. 1 (partition identity): the query attends to disjoint key
+    # slices at their own positions and the merged result is the whole decode
+    w = gen.workload(wi)
+    n = 300
+    cuts = [0, 100, 100, 251, 300]                  # includes an empty slice
+    cfg, whole, bt, slices = _slice_case(w, n, cuts)
+    f = gen.make_factors(w)
+    q = gen.make_queries(1, w.H, w.d_h, seed=3)
+    ref = O.decode(whole, q, f.B_k, f.B_v, bt, [n])
+    parts = [O.decode_slice(c, q, f.B_k, f.B_v, sbt, [hi - lo], [lo], [n - 1]) for c, sbt, lo, hi in slices]
+    o = O.merge_slices([p[0] for p in parts], [p[1] for p in parts], [p[2] for p in parts])
+    np.testing.assert_allclose(o, ref, atol=1e-12, rtol=0)
+    # the empty slice has (o, m, l) = (0, -inf, 0)
+    assert np.all(parts[1][0] == 0) and np.all(parts[1][1] == -np.inf) and np.all(parts[1][2] == 0)
+
+
+def test_slice_statistics_against_materialised_scores():
+    # (m, l) of a slice from scores formed on fully materialised keys RoPE'd by the
+    # transformers helper at the slice's global positions
+    w = gen.workload(0)
+    n, lo, hi = 200, 60, 170
+    cfg, whole, bt, slices = _slice_case(w, n, [0, lo, hi, n])
+    f = gen.make_factors(w)
+    q = gen.make_queries(1, w.H, w.d_h, seed=5)
+    c, sbt, _, _ = slices[1]
+    o, m, l = O.decode_slice(c, q, f.B_k, f.B_v, sbt, [hi - lo], [lo], [n - 1])
+    zk, zv = O.gather_sequence(c, sbt[0], hi - lo)
+    zk = O.unrotate_fp64(zk, cfg.key.g)
+    zv = O.unrotate_fp64(zv, cfg.val.g)
+    for h in range(w.H):
+        kv = h // cfg.group
+        K = hf_rope(zk[:, kv] @ np.asarray(f.B_k[kv], np.float64), np.arange(lo, hi), cfg.rope_base)
+        qr = hf_rope(np.asarray(q[:, h], np.float64), [n - 1], cfg.rope_base)[0]
+        s = K @ qr / np.sqrt(w.d_h)
+        assert m[0, h] == pytest.approx(s.max(), abs=1e-12)
+        assert l[0, h] == pytest.approx(np.exp(s - s.max()).sum(), rel=1e-12)
+        p = np.exp(s - s.max()) / np.exp(s - s.max()).sum()
+        V = zv @ np.asarray(f.B_v, np.float64)[:, kv * w.d_h:(kv + 1) * w.d_h]
+        np.testing.assert_allclose(o[0, h], p @ V, atol=1e-12, rtol=0)
+
+
+def test_one_slice_is_the_whole_decode():
+    w = gen.workload(1)
+    w = gen.shrink(w, ctx=64)
+    n = 70
+    cfg, whole, bt, slices = _slice_case(w, n, [0, n])
+    f = gen.make_factors(w)
+    q = gen.make_queries(1, w.H, w.d_h, seed=7)
+    c, sbt, _, _ = slices[0]
+    o, m, l = O.decode_slice(c, q, f.B_k, f.B_v, sbt, [n], [0], [n - 1])
+    np.testing.assert_allclose(o, O.decode(whole, q, f.B_k, f.B_v, bt, [n]), atol=1e-12, rtol=0)

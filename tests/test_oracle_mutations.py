@@ -242,6 +242,49 @@ def project_k(fp32_accumulate=False, keep_fp64=False):
     return project
 
 
+def decode_slice_k(ignore_pos0=False, q_at_end_of_slice=False):
+    def decode_slice(cache, q, B_k, B_v, block_table, seq_lens, key_pos0, q_pos, heads=None):
+        cfg = cache.cfg
+        q = np.asarray(q)
+        Bn, d = q.shape[0], cfg.d_h
+        heads = list(range(cfg.H)) if heads is None else list(heads)
+        o = np.full((Bn, cfg.H, d), np.nan)
+        m = np.full((Bn, cfg.H), np.nan)
+        l = np.full((Bn, cfg.H), np.nan)
+        B_k, B_v = np.asarray(B_k, np.float64), np.asarray(B_v, np.float64)
+        for b in range(Bn):
+            n = int(seq_lens[b])
+            if n == 0:
+                o[b, heads], m[b, heads], l[b, heads] = 0.0, -np.inf, 0.0
+                continue
+            zk, zv = OM.gather_sequence(cache, block_table[b], n)
+            zk, zv = OM.unrotate_fp64(zk, cfg.key.g), OM.unrotate_fp64(zv, cfg.val.g)
+            pos = (0 if ignore_pos0 else int(key_pos0[b])) + np.arange(n)
+            qp = (int(key_pos0[b]) + n - 1) if q_at_end_of_slice else int(q_pos[b])
+            for h in heads:
+                kv = h // cfg.group
+                k = OM.rope(zk[:, kv] @ B_k[kv], pos, cfg.rope_base)
+                qr = OM.rope(np.asarray(q[b, h], np.float64), qp, cfg.rope_base)
+                mb, lb, acc = OM.partial_softmax((k @ qr) / np.sqrt(d), zv)
+                o[b, h] = (acc / lb) @ B_v[:, kv * d:(kv + 1) * d]
+                m[b, h], l[b, h] = mb, lb
+        return o, m, l
+    return decode_slice
+
+
+def merge_slices_k(drop_l=False, flip=False):
+    def merge_slices(o_parts, m_parts, l_parts):
+        o_parts, m_parts, l_parts = (np.asarray(a, np.float64) for a in (o_parts, m_parts, l_parts))
+        live = l_parts > 0
+        M = np.where(live, m_parts, -np.inf).max(axis=0)
+        e = np.where(live, m_parts, 0.0) - np.where(np.isfinite(M), M, 0.0)
+        w = np.where(live, np.exp(-e if flip else e) * (1.0 if drop_l else l_parts), 0.0)
+        den = w.sum(axis=0)
+        num = (w[..., None] * o_parts).sum(axis=0)
+        return np.where(den[..., None] > 0, num / np.where(den > 0, den, 1.0)[..., None], 0.0)
+    return merge_slices
+
+
 def prefill_k(shift=0):
     def prefill(cache, q, cu_q, B_k, B_v, block_table, seq_lens, select=None, heads=None):
         cfg = cache.cfg
@@ -308,6 +351,9 @@ PINS = {
     "lse_merge": [lambda: TA.test_partition_identity_merge()],
     "project": [lambda: TQ.test_projection_is_the_correctly_rounded_product()],
     "prefill": [lambda: TA.test_prefill_is_causal_decode_per_query()],
+    "decode_slice": [lambda: TA.test_slices_merge_to_the_whole_decode(0),
+                     lambda: TA.test_slice_statistics_against_materialised_scores()],
+    "merge_slices": [lambda: TA.test_slices_merge_to_the_whole_decode(0)],
     "eq14_mean_bits": [lambda: TB.test_eq14_printed_values()],
     "eq16_retained_fraction": [lambda: TB.test_eq16_printed_values()],
 }
@@ -319,6 +365,7 @@ FAITHFUL = {
     "pack_region": pack_k(), "write_latents": write_k(), "gather_sequence": gather_k(),
     "attend_latents": attend_k(), "partial_softmax": partial_k(), "lse_merge": merge_k(),
     "eq14_mean_bits": eq14_k(), "eq16_retained_fraction": eq16_k(), "project": project_k(), "prefill": prefill_k(),
+    "decode_slice": decode_slice_k(), "merge_slices": merge_slices_k(),
 }
 
 PLANTS = {
@@ -355,6 +402,10 @@ PLANTS = {
     "projection accumulated in fp32": ("project", project_k(fp32_accumulate=True)),
     "projection left in fp64": ("project", project_k(keep_fp64=True)),
     "prefill queries one position late": ("prefill", prefill_k(shift=1)),
+    "slice keys RoPE'd at local positions": ("decode_slice", decode_slice_k(ignore_pos0=True)),
+    "slice query at the slice's last position": ("decode_slice", decode_slice_k(q_at_end_of_slice=True)),
+    "slice merge without the slice sums": ("merge_slices", merge_slices_k(drop_l=True)),
+    "slice merge weights e^(M - m)": ("merge_slices", merge_slices_k(flip=True)),
     "eq. 14 bit widths swapped": ("eq14_mean_bits", eq14_k(swap=True)),
     "eq. 16 drops the exempt layers": ("eq16_retained_fraction", eq16_k(drop_exempt=True)),
 }

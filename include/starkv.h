@@ -242,6 +242,44 @@ STARKV_API starkv_status starkv_decode_attn_noalloc(starkv_ctx* ctx, const stark
                                                     int32_t max_pages, void* out,
                                                     starkv_stream_t stream);
 
+/* Decode over one slice of each sequence's context, for sequence (context)
+ * sharding across GPUs: the softmax partition identity of [CaliDrop] (the
+ * attention decomposition theorem, eq. 1) lets every GPU attend the query to
+ * the tokens it holds and a merge combine the slices exactly.  Same dataflow
+ * as starkv_decode_attn ([Review] Algorithm 2 steps 4-8); B_v is linear, so
+ * each slice projects through it locally and only d_h-wide rows cross GPUs.
+ * seq_lens: device int32 [batch], the tokens of the slice held in `cache`
+ *   (the block table maps them from local index 0);
+ * key_pos0: device int32 [batch], the position of the slice's first token
+ *   (its tokens are at key_pos0[b] .. key_pos0[b] + seq_lens[b] - 1);
+ * q_pos: device int32 [batch], the query's position (normally the last
+ *   position of the whole sequence).  Every position must be < max_position.
+ * out_o: device fp32 [batch][num_q_heads][head_dim], 16-byte aligned: the
+ *   attention output over the slice alone (normalised within the slice);
+ * out_ml: device fp32 [batch][num_q_heads][2], 8-byte aligned: the slice's
+ *   softmax statistics (m, l) with scores in log2 units,
+ *   m = max_j s_j * log2(e), l = sum_j 2^(s_j * log2(e) - m); an empty slice
+ *   gives (-inf, 0).
+ * workspace: as starkv_decode_attn.  Only shapes served by the tensor-core
+ * decode are supported (else UNSUPPORTED_SHAPE).
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, WORKSPACE_TOO_SMALL; device bits
+ * BAD_PAGE, BAD_SEQ_LEN (a position outside the RoPE table). */
+STARKV_API starkv_status starkv_decode_attn_slice(starkv_ctx* ctx, const starkv_cache* cache, const void* q,
+                                                  const int32_t* block_table, const int32_t* seq_lens,
+                                                  const int32_t* key_pos0, const int32_t* q_pos, int32_t batch,
+                                                  int32_t max_pages, float* out_o, float* out_ml, void* workspace,
+                                                  size_t workspace_bytes, starkv_stream_t stream);
+
+/* Merge n_parts slice results of the same queries (the partition identity,
+ * [CaliDrop] eq. 1): out = sum_r 2^(m_r - M) l_r o_r / sum_r 2^(m_r - M) l_r
+ * with M = max_r m_r over the slices with l_r > 0 (all-empty: a zero row).
+ * o_parts: device fp32 [n_parts][batch][num_q_heads][head_dim] (16-byte
+ * aligned), ml_parts: device fp32 [n_parts][batch][num_q_heads][2], both as
+ * starkv_decode_attn_slice writes them; out: device bf16
+ * [batch][num_q_heads][head_dim].  Errors: INVALID_ARG. */
+STARKV_API starkv_status starkv_merge_slices(starkv_ctx* ctx, const float* o_parts, const float* ml_parts,
+                                             int32_t n_parts, int32_t batch, void* out, starkv_stream_t stream);
+
 /* Causal chunk attention over the packed cache (the chunked form of the same
  * dataflow).  q: device bf16 [total_q][num_q_heads][head_dim], pre-RoPE, rows of
  * sequence b at cu_q[b] .. cu_q[b+1]-1 (cu_q: device int32 [batch+1], cu_q[0]=0,

@@ -400,6 +400,51 @@ starkv_status starkv_decode_attn_noalloc(starkv_ctx* ctx, const starkv_cache* ca
   return ok();
 }
 
+starkv_status starkv_decode_attn_slice(starkv_ctx* ctx, const starkv_cache* cache, const void* q,
+                                       const int32_t* block_table, const int32_t* seq_lens, const int32_t* key_pos0,
+                                       const int32_t* q_pos, int32_t batch, int32_t max_pages, float* out_o,
+                                       float* out_ml, void* workspace, size_t workspace_bytes,
+                                       starkv_stream_t stream) {
+  if (!ctx) return fail(STARKV_ERR_INVALID_ARG, "ctx is NULL");
+  Ctx* c = reinterpret_cast<Ctx*>(ctx);
+  starkv_status st = check_cache(c, cache);
+  if (st) return st;
+  if (batch < 0 || max_pages < 0) return fail(STARKV_ERR_INVALID_ARG, "negative size");
+  if (batch == 0) return ok();
+  if (max_pages == 0) return fail(STARKV_ERR_INVALID_ARG, "max_pages must be >= 1");
+  if (!q || !block_table || !seq_lens || !key_pos0 || !q_pos || !out_o || !out_ml)
+    return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
+  if (((uintptr_t)out_o & 15) != 0 || ((uintptr_t)out_ml & 7) != 0)
+    return fail(STARKV_ERR_INVALID_ARG, "out_o must be 16-byte and out_ml 8-byte aligned");
+  if (!c->tc)
+    return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "slice decode needs the tensor-core decode path for this shape");
+  const DecodePlan plan = plan_decode(*c, batch, max_pages);
+  if (!workspace || workspace_bytes < plan.ws_bytes)
+    return fail(STARKV_ERR_WORKSPACE_TOO_SMALL, "decode needs %zu workspace bytes, got %zu", plan.ws_bytes,
+                workspace ? workspace_bytes : (size_t)0);
+  if (((uintptr_t)workspace & 255) != 0) return fail(STARKV_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const DecodeSlice slice{key_pos0, q_pos, out_o, out_ml};
+  cudaError_t e = launch_decode_tc(*c, *cache, (const __nv_bfloat16*)q, block_table, seq_lens, batch, max_pages,
+                                   nullptr, workspace, plan, (cudaStream_t)stream, &slice);
+  if (e != cudaSuccess) return cuda_fail(e, "slice decode launch");
+  return ok();
+}
+
+starkv_status starkv_merge_slices(starkv_ctx* ctx, const float* o_parts, const float* ml_parts, int32_t n_parts,
+                                  int32_t batch, void* out, starkv_stream_t stream) {
+  if (!ctx) return fail(STARKV_ERR_INVALID_ARG, "ctx is NULL");
+  Ctx* c = reinterpret_cast<Ctx*>(ctx);
+  if (n_parts < 0 || batch < 0) return fail(STARKV_ERR_INVALID_ARG, "negative size");
+  if (n_parts == 0 || batch == 0) return ok();
+  if (!o_parts || !ml_parts || !out) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
+  if (((uintptr_t)o_parts & 15) != 0 || ((uintptr_t)ml_parts & 7) != 0 || ((uintptr_t)out & 7) != 0)
+    return fail(STARKV_ERR_INVALID_ARG, "o_parts must be 16-byte, ml_parts and out 8-byte aligned");
+  cudaError_t e = launch_merge_slices(o_parts, ml_parts, n_parts, (int64_t)batch * c->cfg.num_q_heads,
+                                      c->cfg.head_dim, (__nv_bfloat16*)out, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return ok();
+}
+
 starkv_status starkv_prefill_attn(starkv_ctx* ctx, const starkv_cache* cache, const void* q, const int32_t* cu_q,
                                   const int32_t* block_table, const int32_t* seq_lens, int32_t batch,
                                   int32_t max_pages, int64_t total_q, int32_t max_q_len, void* out,

@@ -62,6 +62,22 @@ __device__ __forceinline__ unsigned int ordered_bits(float f) {
 __device__ __forceinline__ float ordered_float(unsigned int o) {
   return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
 }
+
+// Token count of sequence b, or -1 when the call's arguments for it are not
+// valid.  The sequence's cached tokens sit at positions pos0 .. pos0 + L - 1
+// (pos0 = 0 without a key-position table) and its query at qpos (L - 1
+// without a query-position table); every position must lie in the RoPE table.
+__device__ __forceinline__ int decode_len(const int32_t* seq_lens, const int32_t* pos0, const int32_t* qpos, int b,
+                                          int max_pages, int max_position) {
+  const int L = seq_lens[b];
+  const int p0 = pos0 ? pos0[b] : 0;
+  if (L < 0 || L > max_pages * kPage || p0 < 0 || (int64_t)p0 + L > max_position) return -1;
+  if (qpos) {
+    const int qp = qpos[b];
+    if (qp < 0 || qp >= max_position) return -1;
+  }
+  return L;
+}
 }  // namespace
 
 // ===========================================================================
@@ -76,6 +92,8 @@ struct ScoreArgs {
   const __nv_bfloat16* q;
   const int32_t* block_table;
   const int32_t* seq_lens;
+  const int32_t* pos0;  // [B] position of each sequence's first cached token, or NULL (0)
+  const int32_t* qpos;  // [B] query positions, or NULL (seq_len - 1)
   const uint8_t* k_codes;
   const uint32_t* k_meta;
   const float* Bk;     // [h_kv][r_k][d] fp32 B'_k
@@ -109,6 +127,8 @@ constexpr int kWpSeq = 1;  // sequences per W-prep CTA
 template <int RK>
 __global__ void __launch_bounds__(128) decode_wprep_kernel(const __nv_bfloat16* __restrict__ q,
                                                            const int32_t* __restrict__ seq_lens,
+                                                           const int32_t* __restrict__ pos0,
+                                                           const int32_t* __restrict__ qpos,
                                                            const float* __restrict__ Bk, const float2* __restrict__ rope,
                                                            uint8_t* __restrict__ wimg, unsigned int* __restrict__ Mx,
                                                            int H, int group, int d, int hpc, int ncols, int batch,
@@ -125,9 +145,9 @@ __global__ void __launch_bounds__(128) decode_wprep_kernel(const __nv_bfloat16* 
     const int sb = e / half, i = e % half, b = b0 + sb;
     float qa = 0.f, qb = 0.f;
     if (b < batch) {
-      int L = seq_lens[b];
-      if (L <= 0 || L > max_pages * kPage || L > max_position) L = 1;  // unused (no tiles), keep reads in range
-      const float2 cs = rope[(int64_t)(L - 1) * half + i];
+      const int L = decode_len(seq_lens, pos0, qpos, b, max_pages, max_position);
+      const int qp = L <= 0 ? 0 : (qpos ? qpos[b] : L - 1);  // no tiles when L <= 0: keep reads in range
+      const float2 cs = rope[(int64_t)qp * half + i];
       const __nv_bfloat16* qv = q + ((int64_t)b * H + h) * d;
       const float x0 = __bfloat162float(qv[i]), x1 = __bfloat162float(qv[i + half]);
       qa = (x0 * cs.x - x1 * cs.y) * scale;
@@ -397,8 +417,10 @@ __global__ void __launch_bounds__(kAThreads, 1)
     const int tile_lo = item - bhg * a.tiles_per_seq;
     const int tile_hi = job_end - bhg * a.tiles_per_seq;
     item = job_end;
-    const int L = a.seq_lens[b];
-    const bool bad_len = L < 0 || L > a.max_pages * kPage || L > a.max_position;
+    const int Lv = decode_len(a.seq_lens, a.pos0, a.qpos, b, a.max_pages, a.max_position);
+    const bool bad_len = Lv < 0;
+    const int L = bad_len ? 0 : Lv;
+    const int p0 = a.pos0 ? a.pos0[b] : 0;  // position of the sequence's first cached token
     const int n_tiles = bad_len ? 0 : (L + kT - 1) / kT;
     const int t0 = tile_lo, t1 = min(tile_hi, n_tiles);
     if (t0 >= t1) continue;
@@ -445,7 +467,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
         if (lane == 0) mbar_arrive_expect_tx(&trfull[ts], a.trig_stage);
         __syncwarp();
         uint8_t* trig_dst = sm + a.off_trig + ts * a.trig_stage;
-        if (lane < nsub) tma_load_2d(trig_dst + lane * 16384, &trig_map, lane * 64, j0, &trfull[ts]);
+        if (lane < nsub) tma_load_2d(trig_dst + lane * 16384, &trig_map, lane * 64, p0 + j0, &trfull[ts]);
         // key codes and metadata of its pages
         if (!__all_sync(0xffffffffu, mbar_wait(&kempty[ks], kph ^ 1))) {
           if (lane == 0) {
@@ -618,6 +640,8 @@ struct ValueArgs {
   int64_t n_pages;
   const int32_t* block_table;
   const int32_t* seq_lens;
+  const int32_t* pos0;  // as ScoreArgs (only their validity matters here)
+  const int32_t* qpos;
   const uint8_t* v_codes;
   const uint32_t* v_meta;
   const unsigned int* Mx;  // [B][H] sequence-wide score maxima (ordered bits)
@@ -678,8 +702,8 @@ __global__ void __launch_bounds__(kVThreads, 1)
   pdl_wait();  // scores, their maxima and the appended codes (every CTA, even one that leaves early)
   pdl_launch_dependents();
 
-  int L = a.seq_lens[b];
-  const bool bad_len = L < 0 || L > a.max_pages * kPage || L > a.max_position;
+  int L = decode_len(a.seq_lens, a.pos0, a.qpos, b, a.max_pages, a.max_position);
+  const bool bad_len = L < 0;
   if (bad_len) {
     if (split == 0 && tid == 0) set_status(a.status, STARKV_DEV_BAD_SEQ_LEN);
     L = 0;
@@ -1007,9 +1031,16 @@ struct ProjArgs {
   float* oacc;           // [B][H][d] fp32 sums (zeroed by the score kernel)
   unsigned int* ocnt;    // [H][ceil(B/16)] arrival counters (zeroed by the score kernel)
   const int32_t* seq_lens;
+  const int32_t* pos0;  // as ScoreArgs (only their validity matters here)
+  const int32_t* qpos;
   int tpad, max_pages, max_position;
   const __half* Bv16;
   __nv_bfloat16* out;
+  // slice mode (sequence sharding): fp32 outputs normalised within the slice,
+  // and the slice's softmax statistics, instead of `out`
+  const unsigned int* Mx;  // [B][H] score maxima (ordered bits, log2 domain)
+  float* out_o;            // [B][H][d] or NULL
+  float* out_ml;           // [B][H][2]: (maximum, sum of 2^(s - maximum)) or NULL
 };
 
 constexpr int kProjM = 16;   // sequences per projection CTA (the MMA's M)
@@ -1027,6 +1058,7 @@ __global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, i
   __shared__ __align__(16) __half As[kProjM][kProjC + 8];
   __shared__ __align__(16) __half Bs[kProjC][128 + 8];
   __shared__ float linv[kProjM];
+  __shared__ float lsum[kProjM];
   __shared__ int nparts_s[kProjM];
   __shared__ int last;
   const int R = a.R, d = a.d;
@@ -1040,8 +1072,8 @@ __global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, i
     const int b = b0 + tid;
     int np = 0;
     if (b < batch) {
-      int L = a.seq_lens[b];
-      if (L < 0 || L > a.max_pages * kPage || L > a.max_position) L = 0;
+      int L = decode_len(a.seq_lens, a.pos0, a.qpos, b, a.max_pages, a.max_position);
+      if (L < 0) L = 0;
       const int nst = (L + a.st - 1) / a.st;
       const int nsp = nst > 0 ? min(a.splits, (int)(((int64_t)nst * a.splits - 1) / a.stages_total) + 1) : 0;
       np = (nsp + a.cs - 1) / a.cs;
@@ -1080,6 +1112,7 @@ __global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, i
       for (int u = 0; u < 4; ++u) l += v[u];
     }
     linv[tid] = l > 0.f ? 1.f / l : 0.f;
+    lsum[tid] = l;
   }
   // o_lat sums: 2 items of 4 channels per thread (16 sequences x 32 quads),
   // added in partial order; both items' loads of a round are in flight together
@@ -1169,14 +1202,73 @@ __global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, i
     for (int i = 0; i < 2; ++i) {
       const int e = (tid + i * 256) * 4, b = b0 + e / d;
       if (e < kProjM * d && b < batch) {
-        __nv_bfloat16* o = a.out + ((int64_t)b * a.H + h) * d + e % d;
-        o[0] = __float2bfloat16_rn(v[i].x);
-        o[1] = __float2bfloat16_rn(v[i].y);
-        o[2] = __float2bfloat16_rn(v[i].z);
-        o[3] = __float2bfloat16_rn(v[i].w);
+        if (a.out_o) {
+          *reinterpret_cast<float4*>(a.out_o + ((int64_t)b * a.H + h) * d + e % d) = v[i];
+        } else {
+          __nv_bfloat16* o = a.out + ((int64_t)b * a.H + h) * d + e % d;
+          o[0] = __float2bfloat16_rn(v[i].x);
+          o[1] = __float2bfloat16_rn(v[i].y);
+          o[2] = __float2bfloat16_rn(v[i].z);
+          o[3] = __float2bfloat16_rn(v[i].w);
+        }
       }
     }
+    if (a.out_ml && tid < kProjM && b0 + tid < batch) {
+      // the slice's softmax statistics: maximum (log2 domain) and sum; an empty slice has (-inf, 0)
+      const int b = b0 + tid;
+      const unsigned int mo = a.Mx[b * a.H + h];
+      const float m = (mo && lsum[tid] > 0.f) ? ordered_float(mo) : -INFINITY;
+      *reinterpret_cast<float2*>(a.out_ml + ((int64_t)b * a.H + h) * 2) = make_float2(m, lsum[tid] > 0.f ? lsum[tid] : 0.f);
+    }
   }
+}
+
+// ===========================================================================
+// merge of slice results (sequence sharding): the softmax partition identity
+//   o = sum_r 2^(m_r - M) l_r o_r / sum_r 2^(m_r - M) l_r,  M = max_r m_r
+// one thread per (sequence, head, 4 output columns)
+// ===========================================================================
+__global__ void merge_slices_kernel(const float* __restrict__ o_parts, const float* __restrict__ ml_parts, int n_parts,
+                                    int64_t bh, int d, __nv_bfloat16* __restrict__ out) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int q4 = d / 4;
+  if (idx >= bh * q4) return;
+  const int64_t r = idx / q4;
+  const int c = (int)(idx % q4) * 4;
+  float M = -INFINITY;
+  for (int p = 0; p < n_parts; ++p) {
+    const float2 ml = *reinterpret_cast<const float2*>(ml_parts + ((int64_t)p * bh + r) * 2);
+    if (ml.y > 0.f) M = fmaxf(M, ml.x);
+  }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float den = 0.f;
+  if (M != -INFINITY) {
+    for (int p = 0; p < n_parts; ++p) {
+      const float2 ml = *reinterpret_cast<const float2*>(ml_parts + ((int64_t)p * bh + r) * 2);
+      if (!(ml.y > 0.f)) continue;
+      const float w = exp2f(ml.x - M) * ml.y;
+      const float4 o = *reinterpret_cast<const float4*>(o_parts + ((int64_t)p * bh + r) * d + c);
+      acc.x = fmaf(w, o.x, acc.x);
+      acc.y = fmaf(w, o.y, acc.y);
+      acc.z = fmaf(w, o.z, acc.z);
+      acc.w = fmaf(w, o.w, acc.w);
+      den += w;
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  __nv_bfloat16* o = out + r * d + c;
+  o[0] = __float2bfloat16_rn(acc.x * inv);
+  o[1] = __float2bfloat16_rn(acc.y * inv);
+  o[2] = __float2bfloat16_rn(acc.z * inv);
+  o[3] = __float2bfloat16_rn(acc.w * inv);
+}
+
+cudaError_t launch_merge_slices(const float* o_parts, const float* ml_parts, int n_parts, int64_t bh, int d,
+                                __nv_bfloat16* out, cudaStream_t s) {
+  const int64_t n = bh * (d / 4);
+  if (n == 0) return cudaSuccess;
+  merge_slices_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(o_parts, ml_parts, n_parts, bh, d, out);
+  return cudaGetLastError();
 }
 
 // ===========================================================================
@@ -1453,8 +1545,11 @@ static cudaError_t launch_scores(const Ctx& c, const ScoreArgs& a, int grid, siz
 
 cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
                              const int32_t* block_table, const int32_t* seq_lens, int batch, int max_pages,
-                             __nv_bfloat16* out, void* ws, const DecodePlan&, cudaStream_t s) {
+                             __nv_bfloat16* out, void* ws, const DecodePlan&, cudaStream_t s,
+                             const DecodeSlice* slice) {
   if (batch == 0) return cudaSuccess;
+  const int32_t* pos0 = slice ? slice->pos0 : nullptr;
+  const int32_t* qpos = slice ? slice->qpos : nullptr;
   const starkv_config& f = c.cfg;
   const TcLayout t = tc_layout(c, batch, max_pages);
   char* w = (char*)ws;
@@ -1473,15 +1568,15 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
     cudaError_t e0 = cudaSuccess;
     switch (f.rank_k) {
       case 16:
-        e0 = launch_chained(decode_wprep_kernel<16>, g, dim3(128), 0, s, 1u, q, seq_lens, (const float*)c.Bk, (const float2*)c.rope, wimg, Mx,
+        e0 = launch_chained(decode_wprep_kernel<16>, g, dim3(128), 0, s, 1u, q, seq_lens, pos0, qpos, (const float*)c.Bk, (const float2*)c.rope, wimg, Mx,
                             (int)f.num_q_heads, c.group, d, t.hpc, t.ncols, batch, max_pages, (int)f.max_position);
         break;
       case 32:
-        e0 = launch_chained(decode_wprep_kernel<32>, g, dim3(128), 0, s, 1u, q, seq_lens, (const float*)c.Bk, (const float2*)c.rope, wimg, Mx,
+        e0 = launch_chained(decode_wprep_kernel<32>, g, dim3(128), 0, s, 1u, q, seq_lens, pos0, qpos, (const float*)c.Bk, (const float2*)c.rope, wimg, Mx,
                             (int)f.num_q_heads, c.group, d, t.hpc, t.ncols, batch, max_pages, (int)f.max_position);
         break;
       default:
-        e0 = launch_chained(decode_wprep_kernel<64>, g, dim3(128), 0, s, 1u, q, seq_lens, (const float*)c.Bk, (const float2*)c.rope, wimg, Mx,
+        e0 = launch_chained(decode_wprep_kernel<64>, g, dim3(128), 0, s, 1u, q, seq_lens, pos0, qpos, (const float*)c.Bk, (const float2*)c.rope, wimg, Mx,
                             (int)f.num_q_heads, c.group, d, t.hpc, t.ncols, batch, max_pages, (int)f.max_position);
         break;
     }
@@ -1517,6 +1612,8 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   A.q = q;
   A.block_table = block_table;
   A.seq_lens = seq_lens;
+  A.pos0 = pos0;
+  A.qpos = qpos;
   A.k_codes = (const uint8_t*)cache.k_codes;
   A.k_meta = (const uint32_t*)cache.k_meta;
   A.Bk = c.Bk;
@@ -1590,6 +1687,8 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   B.n_pages = cache.n_pages;
   B.block_table = block_table;
   B.seq_lens = seq_lens;
+  B.pos0 = pos0;
+  B.qpos = qpos;
   B.v_codes = (const uint8_t*)cache.v_codes;
   B.v_meta = (const uint32_t*)cache.v_meta;
   B.Mx = Mx;
@@ -1648,6 +1747,11 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   P.part = acc;
   P.lpart = lsum;
   P.seq_lens = seq_lens;
+  P.pos0 = pos0;
+  P.qpos = qpos;
+  P.Mx = Mx;
+  P.out_o = slice ? slice->out_o : nullptr;
+  P.out_ml = slice ? slice->out_ml : nullptr;
   P.tpad = t.tpad;
   P.max_pages = max_pages;
   P.max_position = f.max_position;

@@ -301,9 +301,22 @@ cudaError_t launch_decode_simt(const Ctx& c, const starkv_cache& cache, const __
 // tensor-core decode (decode_tc.cu)
 bool tc_decode_supported(const starkv_config& cfg);
 DecodePlan plan_decode_tc(const Ctx& c, int batch, int max_pages);
+// Decode over one slice of each sequence's context (sequence sharding): the
+// slice's tokens sit at positions pos0[b] .. pos0[b] + seq_lens[b] - 1, the
+// query at qpos[b]; the results are fp32 outputs normalised within the slice
+// (out_o [B][H][d]) and the slice's softmax statistics (out_ml [B][H][2]).
+struct DecodeSlice {
+  const int32_t* pos0;
+  const int32_t* qpos;
+  float* out_o;
+  float* out_ml;
+};
 cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
                              const int32_t* block_table, const int32_t* seq_lens, int batch, int max_pages,
-                             __nv_bfloat16* out, void* ws, const DecodePlan& plan, cudaStream_t s);
+                             __nv_bfloat16* out, void* ws, const DecodePlan& plan, cudaStream_t s,
+                             const DecodeSlice* slice = nullptr);
+cudaError_t launch_merge_slices(const float* o_parts, const float* ml_parts, int n_parts, int64_t bh, int d,
+                                __nv_bfloat16* out, cudaStream_t s);
 cudaError_t launch_prepare_tc_factors(const Ctx& c, cudaStream_t s);
 cudaError_t launch_decode(const Ctx& c, const starkv_cache& cache, const __nv_bfloat16* q,
                           const int32_t* block_table, const int32_t* seq_lens, int batch,

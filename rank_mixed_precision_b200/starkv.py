@@ -25,7 +25,7 @@ LATENT_KEY, LATENT_VALUE = 0, 1
 EXPORTS = [
     "starkv_version", "starkv_last_error", "starkv_cache_layout", "starkv_create", "starkv_destroy",
     "starkv_get_config", "starkv_append", "starkv_workspace_bytes", "starkv_decode_attn",
-    "starkv_decode_attn_noalloc",
+    "starkv_decode_attn_noalloc", "starkv_decode_attn_slice", "starkv_merge_slices",
     "starkv_prefill_attn", "starkv_quantize_pack", "starkv_dequantize", "starkv_read_device_status",
     "starkv_selftest_wait_timeout",
 ]
@@ -73,6 +73,9 @@ _SIGS = {
     "starkv_workspace_bytes": ([_vp, _i32, _i32, _i32, _i64, ctypes.POINTER(_sz)], _i32),
     "starkv_decode_attn": ([_vp, ctypes.POINTER(starkv_cache), _vp, _vp, _vp, _i32, _i32, _vp, _vp, _sz, _vp], _i32),
     "starkv_decode_attn_noalloc": ([_vp, ctypes.POINTER(starkv_cache), _vp, _vp, _vp, _i32, _i32, _vp, _vp], _i32),
+    "starkv_decode_attn_slice": ([_vp, ctypes.POINTER(starkv_cache), _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp,
+                                  _vp, _sz, _vp], _i32),
+    "starkv_merge_slices": ([_vp, _vp, _vp, _i32, _i32, _vp, _vp], _i32),
     "starkv_prefill_attn": ([_vp, ctypes.POINTER(starkv_cache), _vp, _vp, _vp, _vp, _i32, _i32, _i64, _i32, _vp,
                              _vp, _sz, _vp], _i32),
     "starkv_quantize_pack": ([_vp, _i32, _vp, _i64, _vp, _vp, _vp], _i32),
@@ -216,6 +219,37 @@ def starkv_decode_attn_noalloc(ctx, cache: starkv_cache, q, block_table, seq_len
         raise ValueError("q / block_table / seq_lens / out disagree on the batch")
     _check(lib().starkv_decode_attn_noalloc(ctx, ctypes.byref(cache), _p(q), _p(block_table), _p(seq_lens), B,
                                             block_table.shape[1], _p(out), _stream(stream)))
+
+
+def starkv_decode_attn_slice(ctx, cache: starkv_cache, q, block_table, seq_lens, key_pos0, q_pos, out_o, out_ml,
+                             workspace, stream=None):
+    """Decode over one slice of each sequence's context (sequence sharding):
+    fp32 output normalised within the slice and its (m, l) statistics."""
+    _need(q, torch.bfloat16, "q", 3)
+    _need(block_table, torch.int32, "block_table", 2)
+    for t, n in ((seq_lens, "seq_lens"), (key_pos0, "key_pos0"), (q_pos, "q_pos")):
+        _need(t, torch.int32, n, 1)
+    _need(out_o, torch.float32, "out_o", 3)
+    _need(out_ml, torch.float32, "out_ml", 3)
+    _need(workspace, torch.uint8, "workspace", 1)
+    B = q.shape[0]
+    if any(t.shape[0] != B for t in (block_table, seq_lens, key_pos0, q_pos, out_ml)) or \
+            tuple(out_o.shape) != tuple(q.shape) or tuple(out_ml.shape) != (B, q.shape[1], 2):
+        raise ValueError("slice decode arguments disagree on the shapes")
+    _check(lib().starkv_decode_attn_slice(ctx, ctypes.byref(cache), _p(q), _p(block_table), _p(seq_lens),
+                                          _p(key_pos0), _p(q_pos), B, block_table.shape[1], _p(out_o), _p(out_ml),
+                                          _p(workspace), workspace.numel(), _stream(stream)))
+
+
+def starkv_merge_slices(ctx, o_parts, ml_parts, out, stream=None):
+    """Merge slice results [n, B, H, d] / [n, B, H, 2] into the bf16 output [B, H, d]."""
+    _need(o_parts, torch.float32, "o_parts", 4)
+    _need(ml_parts, torch.float32, "ml_parts", 4)
+    _need(out, torch.bfloat16, "out", 3)
+    n, B = o_parts.shape[0], o_parts.shape[1]
+    if tuple(o_parts.shape[1:]) != tuple(out.shape) or tuple(ml_parts.shape) != (n, B, out.shape[1], 2):
+        raise ValueError("merge arguments disagree on the shapes")
+    _check(lib().starkv_merge_slices(ctx, _p(o_parts), _p(ml_parts), n, B, _p(out), _stream(stream)))
 
 
 def starkv_prefill_attn(ctx, cache: starkv_cache, q, cu_q, block_table, seq_lens, max_q_len, out, workspace,

@@ -146,7 +146,7 @@ typedef struct starkv_cache_sizes {
 
 typedef struct starkv_ctx starkv_ctx;
 
-enum { STARKV_OP_DECODE = 0, STARKV_OP_PREFILL = 1 };
+enum { STARKV_OP_DECODE = 0, STARKV_OP_PREFILL = 1, STARKV_OP_DECODE_OUT = 2 };
 enum { STARKV_LATENT_KEY = 0, STARKV_LATENT_VALUE = 1 };
 
 /* Library version string (static storage). */
@@ -194,9 +194,10 @@ STARKV_API starkv_status starkv_append(starkv_ctx* ctx, const starkv_cache* cach
                             const int64_t* slot_mapping, int64_t n, float* latents_out,
                             starkv_stream_t stream);
 
-/* Workspace bytes needed by decode (op = STARKV_OP_DECODE; total_q ignored) or
- * prefill (op = STARKV_OP_PREFILL) for `batch` sequences whose block tables
- * have max_pages columns.  out: host. */
+/* Workspace bytes needed by decode (op = STARKV_OP_DECODE; total_q ignored),
+ * decode with the output projection (op = STARKV_OP_DECODE_OUT; needs
+ * starkv_set_output_projection first) or prefill (op = STARKV_OP_PREFILL) for
+ * `batch` sequences whose block tables have max_pages columns.  out: host. */
 STARKV_API starkv_status starkv_workspace_bytes(const starkv_ctx* ctx, int32_t op, int32_t batch,
                                      int32_t max_pages, int64_t total_q, size_t* out);
 
@@ -215,6 +216,31 @@ STARKV_API starkv_status starkv_decode_attn(starkv_ctx* ctx, const starkv_cache*
                                  const int32_t* block_table, const int32_t* seq_lens,
                                  int32_t batch, int32_t max_pages, void* out, void* workspace,
                                  size_t workspace_bytes, starkv_stream_t stream);
+
+/* Give the context the attention block's output projection W_o, so that
+ * decode can emit the block's output directly ([Review] Algorithm 2 steps 7-8:
+ * apply the prepared head-specific value/output factors and sum the head
+ * contributions; section 5.3 eq. 12).  W_o: device bf16 [num_q_heads*head_dim]
+ * [model_dim], the rows of query head h at h*head_dim .. (h+1)*head_dim - 1.
+ * Copied into context-owned memory (synchronises `stream`); a later call
+ * replaces it.  model_dim: a positive multiple of 8, <= 65536.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, CUDA. */
+STARKV_API starkv_status starkv_set_output_projection(starkv_ctx* ctx, const void* W_o, int32_t model_dim,
+                                                      starkv_stream_t stream);
+
+/* Decode attention followed by the output projection: the same arguments as
+ * starkv_decode_attn, but the result is the attention block's output
+ * y[b] = sum_h o_h[b] W_o,h, device bf16 [batch][model_dim], where o_h is what
+ * starkv_decode_attn returns.  The value factor B_v is applied first (in the
+ * R-dim latent, then d_h wide) and W_o second: with R > d_h that is cheaper
+ * than the fused factor U_h^T O_h of eq. 12 (R x model_dim per query head).
+ * workspace: >= starkv_workspace_bytes(STARKV_OP_DECODE_OUT, ...), 256-byte
+ * aligned.  Errors: as starkv_decode_attn, plus INVALID_ARG without an output
+ * projection. */
+STARKV_API starkv_status starkv_decode_attn_out(starkv_ctx* ctx, const starkv_cache* cache, const void* q,
+                                                const int32_t* block_table, const int32_t* seq_lens, int32_t batch,
+                                                int32_t max_pages, void* y, void* workspace, size_t workspace_bytes,
+                                                starkv_stream_t stream);
 
 /* Decode without any device allocation: the same computation and arguments as
  * starkv_decode_attn, minus the workspace.  (The paper has no counterpart; this

@@ -463,6 +463,18 @@ def decode(cache: Cache, q, B_k, B_v, block_table, seq_lens, seqs=None, heads=No
     return out
 
 
+def decode_out(cache: Cache, q, B_k, B_v, W_o, block_table, seq_lens):
+    """starkv_decode_attn_out: the attention block's output, decode dataflow
+    steps 7-8 ([Review] Algorithm 2: apply the head-specific value/output
+    factors, sum the head contributions; eq. 12):
+    y[b] = sum_h o_h[b] W_o[h d_h : (h + 1) d_h, :] with o from ``decode``.
+    W_o: [H d_h, model_dim].  Returns y [B, model_dim] (fp64)."""
+    cfg = cache.cfg
+    o = decode(cache, q, B_k, B_v, block_table, seq_lens)
+    W_o = np.asarray(W_o, np.float64)
+    return o.reshape(o.shape[0], cfg.H * cfg.d_h) @ W_o
+
+
 def decode_slice(cache: Cache, q, B_k, B_v, block_table, seq_lens, key_pos0, q_pos, heads=None):
     """starkv_decode_attn_slice: sequence b's cache holds one slice of its context,
     seq_lens[b] tokens at positions key_pos0[b] .. key_pos0[b] + seq_lens[b] - 1

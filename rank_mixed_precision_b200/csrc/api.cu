@@ -123,6 +123,20 @@ starkv_status check_cache(const Ctx* c, const starkv_cache* cache) {
   return STARKV_OK;
 }
 
+struct DecodeOutWs {
+  size_t decode, o, zpart, total;
+};
+
+DecodeOutWs decode_out_ws(const Ctx& c, int batch, int max_pages) {
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  DecodeOutWs w;
+  w.decode = al(plan_decode(c, batch, max_pages).ws_bytes);
+  w.o = al((size_t)batch * c.cfg.num_q_heads * c.cfg.head_dim * 2);
+  w.zpart = al((size_t)(c.wo_splits > 0 ? c.wo_splits : 1) * kSmallAppend * (c.model_dim > 0 ? c.model_dim : 1) * 4);
+  w.total = w.decode + w.o + w.zpart;
+  return w;
+}
+
 }  // namespace
 
 namespace starkv {
@@ -208,6 +222,7 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
     cudaFree(c->status);
     cudaFree(c->Bk16);
     cudaFree(c->Bv16p);
+    cudaFree(c->Wo);
     delete c;
   };
   // small appends: K splits of the projection so that about every SM streams a
@@ -313,7 +328,56 @@ starkv_status starkv_destroy(starkv_ctx* ctx) {
   cudaFree(c->status);
   cudaFree(c->Bk16);
   cudaFree(c->Bv16p);
+  cudaFree(c->Wo);
   delete c;
+  return ok();
+}
+
+starkv_status starkv_set_output_projection(starkv_ctx* ctx, const void* W_o, int32_t model_dim,
+                                           starkv_stream_t stream) {
+  if (!ctx) return fail(STARKV_ERR_INVALID_ARG, "ctx is NULL");
+  Ctx* c = reinterpret_cast<Ctx*>(ctx);
+  if (!W_o) return fail(STARKV_ERR_INVALID_ARG, "W_o is NULL");
+  if (model_dim <= 0 || model_dim % 8 != 0 || model_dim > (1 << 16))
+    return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "model_dim %d: need a positive multiple of 8, <= 65536", model_dim);
+  const int K = c->cfg.num_q_heads * c->cfg.head_dim;
+  // K splits so that about every SM streams a slice of W_o (slices of 64..512 rows)
+  int splits = 0;
+  {
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, c->device);
+    const int col_blocks = (model_dim + 127) / 128;
+    for (int kl = 512; kl >= 64; kl >>= 1) {
+      if (K % kl != 0) continue;
+      if (K / kl > 64) break;
+      splits = K / kl;
+      if ((int64_t)splits * col_blocks * 4 >= (int64_t)sms * 3) break;
+    }
+  }
+  if (splits == 0) return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "num_q_heads*head_dim must be a multiple of 64");
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t bytes = (size_t)K * model_dim * 2;
+  __nv_bfloat16* w = nullptr;
+  cudaError_t e = cudaMalloc(&w, bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc (output projection)");
+  e = cudaMemcpyAsync(w, W_o, bytes, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    cudaFree(w);
+    return cuda_fail(e, "starkv_set_output_projection");
+  }
+  const int kl = K / splits;
+  CUtensorMap map;
+  if (!starkv::encode_map_2d(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, (uint64_t)model_dim, (uint64_t)K,
+                             (uint64_t)model_dim * 2, 64, kl < 256 ? kl : 256, CU_TENSOR_MAP_SWIZZLE_128B)) {
+    cudaFree(w);
+    return fail(STARKV_ERR_CUDA, "tensor map of the output projection");
+  }
+  cudaFree(c->Wo);
+  c->Wo = w;
+  c->model_dim = model_dim;
+  c->wo_splits = splits;
+  c->wo_map = map;
   return ok();
 }
 
@@ -344,6 +408,9 @@ starkv_status starkv_workspace_bytes(const starkv_ctx* ctx, int32_t op, int32_t 
   const Ctx* c = reinterpret_cast<const Ctx*>(ctx);
   if (op == STARKV_OP_DECODE) {
     *out = plan_decode(*c, batch, max_pages).ws_bytes;
+  } else if (op == STARKV_OP_DECODE_OUT) {
+    if (c->model_dim <= 0) return fail(STARKV_ERR_INVALID_ARG, "no output projection set");
+    *out = decode_out_ws(*c, batch, max_pages).total;
   } else if (op == STARKV_OP_PREFILL) {
     *out = plan_prefill(*c, batch, max_pages, total_q).ws_bytes;
   } else {
@@ -371,6 +438,35 @@ starkv_status starkv_decode_attn(starkv_ctx* ctx, const starkv_cache* cache, con
   cudaError_t e = launch_decode(*c, *cache, (const __nv_bfloat16*)q, block_table, seq_lens, batch, max_pages,
                                 (__nv_bfloat16*)out, workspace, plan, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return ok();
+}
+
+starkv_status starkv_decode_attn_out(starkv_ctx* ctx, const starkv_cache* cache, const void* q,
+                                     const int32_t* block_table, const int32_t* seq_lens, int32_t batch,
+                                     int32_t max_pages, void* y, void* workspace, size_t workspace_bytes,
+                                     starkv_stream_t stream) {
+  if (!ctx) return fail(STARKV_ERR_INVALID_ARG, "ctx is NULL");
+  Ctx* c = reinterpret_cast<Ctx*>(ctx);
+  starkv_status st = check_cache(c, cache);
+  if (st) return st;
+  if (c->model_dim <= 0) return fail(STARKV_ERR_INVALID_ARG, "no output projection set (starkv_set_output_projection)");
+  if (batch < 0 || max_pages < 0) return fail(STARKV_ERR_INVALID_ARG, "negative size");
+  if (batch == 0) return ok();
+  if (max_pages == 0) return fail(STARKV_ERR_INVALID_ARG, "max_pages must be >= 1");
+  if (!q || !block_table || !seq_lens || !y) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
+  const DecodeOutWs w = decode_out_ws(*c, batch, max_pages);
+  if (!workspace || workspace_bytes < w.total)
+    return fail(STARKV_ERR_WORKSPACE_TOO_SMALL, "decode with output projection needs %zu workspace bytes, got %zu",
+                w.total, workspace ? workspace_bytes : (size_t)0);
+  if (((uintptr_t)workspace & 255) != 0) return fail(STARKV_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  char* base = (char*)workspace;
+  __nv_bfloat16* o = (__nv_bfloat16*)(base + w.decode);
+  float* zpart = (float*)(base + w.decode + w.o);
+  const DecodePlan plan = plan_decode(*c, batch, max_pages);
+  cudaError_t e = launch_decode(*c, *cache, (const __nv_bfloat16*)q, block_table, seq_lens, batch, max_pages, o,
+                                workspace, plan, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = launch_outproj(*c, o, batch, (__nv_bfloat16*)y, zpart, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode with output projection");
   return ok();
 }
 

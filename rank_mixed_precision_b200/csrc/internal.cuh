@@ -57,6 +57,11 @@ struct Ctx {
   bool tc_prefill;        // tensor-core prefill available for this shape
   CUtensorMap a_map64;    // TMA map of `A`: box 64 columns x 64 rows, 128-byte swizzle (tensor-core append)
   bool tc_append;         // tensor-core append (more than 64 tokens) available
+  // output projection (set by starkv_set_output_projection; model_dim 0 = none)
+  __nv_bfloat16* Wo;      // [H*d_h][model_dim] bf16
+  int model_dim;
+  int wo_splits;          // K splits of the output projection GEMM
+  CUtensorMap wo_map;     // TMA map of Wo: box 64 columns x min(256, K / wo_splits) rows, 128-byte swizzle
 };
 
 // 2-D TMA map over a row-major [rows][inner] array (no interleave, zero fill).
@@ -322,6 +327,11 @@ cudaError_t launch_decode(const Ctx& c, const starkv_cache& cache, const __nv_bf
                           const int32_t* block_table, const int32_t* seq_lens, int batch,
                           int max_pages, __nv_bfloat16* out, void* ws, const DecodePlan& plan,
                           cudaStream_t s);
+
+// Output projection y = o W_o of a decode step's bf16 output o [batch][H*d_h]
+// (quant.cu); zpart: [wo_splits][kSmallAppend][model_dim] fp32 scratch.
+cudaError_t launch_outproj(const Ctx& c, const __nv_bfloat16* o, int batch, __nv_bfloat16* y, float* zpart,
+                           cudaStream_t s);
 
 // Built-in scratch of starkv_decode_attn_noalloc (see decode.cu).
 constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;  // 16 MiB

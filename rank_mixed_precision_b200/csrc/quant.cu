@@ -293,6 +293,55 @@ __global__ void __launch_bounds__(256, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Output projection of a decode step (the attention block's output, [Review]
+// Algorithm 2 steps 7-8: apply the head-specific output factors and sum the
+// head contributions): y[b] = sum_h o_h[b] W_o[h d : (h + 1) d, :], a thin GEMM
+// [B x H d] . [H d x model_dim] bound by reading W_o once.  The same split-K
+// kernel as the small appends (A slice by TMA, mma.sync), then a reduction of
+// the split sums in a fixed order.
+// ---------------------------------------------------------------------------
+__global__ void outproj_reduce_kernel(const float* __restrict__ zpart, int splits, int rows, int cols,
+                                      __nv_bfloat16* __restrict__ y) {
+  sm100::pdl_wait();  // the split sums
+  sm100::pdl_launch_dependents();
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)rows * cols) return;
+  const int r = (int)(idx / cols), col = (int)(idx % cols);
+  float v = 0.f;
+  for (int sp = 0; sp < splits; ++sp) v += __ldcg(zpart + ((int64_t)sp * kSmallAppend + r) * cols + col);
+  y[idx] = __float2bfloat16_rn(v);
+}
+
+cudaError_t launch_outproj(const Ctx& c, const __nv_bfloat16* o, int batch, __nv_bfloat16* y, float* zpart,
+                           cudaStream_t s) {
+  const int K = c.cfg.num_q_heads * c.cfg.head_dim, N = c.model_dim;
+  const int KL = K / c.wo_splits;
+  const size_t smem_max = (size_t)2 * KL * 128 + (size_t)kSmallAppend * (KL + 8) * 2 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(append_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
+  if (e != cudaSuccess) return e;
+  for (int b0 = 0; b0 < batch; b0 += kSmallAppend) {
+    const int n = batch - b0 < kSmallAppend ? batch - b0 : kSmallAppend;
+    AppendArgs a = {};
+    a.hidden = K;
+    a.lat_cols = N;
+    a.n = n;
+    a.X = o + (int64_t)b0 * K;
+    a.status = c.status;
+    const size_t smem = (size_t)2 * KL * 128 + (size_t)((n + 15) / 16) * 16 * (KL + 8) * 2 + 1024;
+    dim3 g1((unsigned)((N + kAgCols - 1) / kAgCols), (unsigned)c.wo_splits);
+    // a plain launch: the kernel reads o without waiting on a programmatic edge
+    append_gemm_kernel<<<g1, 256, smem, s>>>(c.wo_map, a, KL, zpart);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t total = (int64_t)n * N;
+    e = launch_chained(outproj_reduce_kernel, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, s, 1u,
+                       (const float*)zpart, c.wo_splits, n, N, y + (int64_t)b0 * N);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaGetLastError();
+}
+
 // One thread per (token, 4 columns): it adds its columns' split sums (every
 // load in flight at once), then the group's leader gathers the group's g values
 // from its neighbours by shuffles (groups never straddle a warp: they start on

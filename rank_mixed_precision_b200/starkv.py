@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libstarkv.s
 PAGE_TOKENS = 16
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_WORKSPACE_TOO_SMALL, ERR_CUDA, ERR_DEVICE_STATUS = range(6)
 DEV_BAD_PAGE, DEV_BAD_SEQ_LEN, DEV_QUANT_OVERFLOW, DEV_BAD_SLOT, DEV_BAD_QUERY_SPAN, DEV_WAIT_TIMEOUT = 1, 2, 4, 8, 16, 32
-OP_DECODE, OP_PREFILL = 0, 1
+OP_DECODE, OP_PREFILL, OP_DECODE_OUT = 0, 1, 2
 LATENT_KEY, LATENT_VALUE = 0, 1
 
 # every function include/starkv.h declares
@@ -26,6 +26,7 @@ EXPORTS = [
     "starkv_version", "starkv_last_error", "starkv_cache_layout", "starkv_create", "starkv_destroy",
     "starkv_get_config", "starkv_append", "starkv_workspace_bytes", "starkv_decode_attn",
     "starkv_decode_attn_noalloc", "starkv_decode_attn_slice", "starkv_merge_slices",
+    "starkv_set_output_projection", "starkv_decode_attn_out",
     "starkv_prefill_attn", "starkv_quantize_pack", "starkv_dequantize", "starkv_read_device_status",
     "starkv_selftest_wait_timeout",
 ]
@@ -76,6 +77,9 @@ _SIGS = {
     "starkv_decode_attn_slice": ([_vp, ctypes.POINTER(starkv_cache), _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp,
                                   _vp, _sz, _vp], _i32),
     "starkv_merge_slices": ([_vp, _vp, _vp, _i32, _i32, _vp, _vp], _i32),
+    "starkv_set_output_projection": ([_vp, _vp, _i32, _vp], _i32),
+    "starkv_decode_attn_out": ([_vp, ctypes.POINTER(starkv_cache), _vp, _vp, _vp, _i32, _i32, _vp, _vp, _sz, _vp],
+                               _i32),
     "starkv_prefill_attn": ([_vp, ctypes.POINTER(starkv_cache), _vp, _vp, _vp, _vp, _i32, _i32, _i64, _i32, _vp,
                              _vp, _sz, _vp], _i32),
     "starkv_quantize_pack": ([_vp, _i32, _vp, _i64, _vp, _vp, _vp], _i32),
@@ -239,6 +243,27 @@ def starkv_decode_attn_slice(ctx, cache: starkv_cache, q, block_table, seq_lens,
     _check(lib().starkv_decode_attn_slice(ctx, ctypes.byref(cache), _p(q), _p(block_table), _p(seq_lens),
                                           _p(key_pos0), _p(q_pos), B, block_table.shape[1], _p(out_o), _p(out_ml),
                                           _p(workspace), workspace.numel(), _stream(stream)))
+
+
+def starkv_set_output_projection(ctx, W_o, stream=None):
+    """W_o: bf16 [num_q_heads * head_dim, model_dim] (copied by the library)."""
+    _need(W_o, torch.bfloat16, "W_o", 2)
+    _check(lib().starkv_set_output_projection(ctx, _p(W_o), W_o.shape[1], _stream(stream)))
+
+
+def starkv_decode_attn_out(ctx, cache: starkv_cache, q, block_table, seq_lens, y, workspace, stream=None):
+    """Decode attention and the output projection: y bf16 [batch, model_dim]."""
+    _need(q, torch.bfloat16, "q", 3)
+    _need(block_table, torch.int32, "block_table", 2)
+    _need(seq_lens, torch.int32, "seq_lens", 1)
+    _need(y, torch.bfloat16, "y", 2)
+    _need(workspace, torch.uint8, "workspace", 1)
+    B = q.shape[0]
+    if block_table.shape[0] != B or seq_lens.shape[0] != B or y.shape[0] != B:
+        raise ValueError("q / block_table / seq_lens / y disagree on the batch")
+    _check(lib().starkv_decode_attn_out(ctx, ctypes.byref(cache), _p(q), _p(block_table), _p(seq_lens), B,
+                                        block_table.shape[1], _p(y), _p(workspace), workspace.numel(),
+                                        _stream(stream)))
 
 
 def starkv_merge_slices(ctx, o_parts, ml_parts, out, stream=None):

@@ -115,6 +115,9 @@ def test_every_entry_point_rejects_a_null_context_before_any_device_work(S):
         "starkv_decode_attn_slice": lambda: L.starkv_decode_attn_slice(None, None, None, None, None, None, None, 1, 1,
                                                                       None, None, None, 0, None),
         "starkv_merge_slices": lambda: L.starkv_merge_slices(None, None, None, 1, 1, None, None),
+        "starkv_set_output_projection": lambda: L.starkv_set_output_projection(None, None, 64, None),
+        "starkv_decode_attn_out": lambda: L.starkv_decode_attn_out(None, None, None, None, None, 1, 1, None, None, 0,
+                                                                  None),
         "starkv_prefill_attn": lambda: L.starkv_prefill_attn(None, None, None, None, None, None, 1, 1, 1, 1, None, None,
                                                             0, None),
         "starkv_workspace_bytes": lambda: L.starkv_workspace_bytes(None, 0, 1, 1, 0, ctypes.byref(sz)),

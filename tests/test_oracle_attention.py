@@ -273,3 +273,36 @@ def test_one_slice_is_the_whole_decode():
     c, sbt, _, _ = slices[0]
     o, m, l = O.decode_slice(c, q, f.B_k, f.B_v, sbt, [n], [0], [n - 1])
     np.testing.assert_allclose(o, O.decode(whole, q, f.B_k, f.B_v, bt, [n]), atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("H,h_kv", [(4, 4), (8, 2)])
+def test_output_projection_equals_fused_factor_and_dense(H, h_kv):
+    # [Review] eq. 12: p_h (Z_V U_h^T) O_h = (p_h Z_V) (U_h^T O_h).  The oracle's
+    # two-stage y = sum_h o_h W_o,h equals the fused factor form (latent row times
+    # the offline product B_v,h W_o,h) and the dense form (materialised V, torch
+    # SDPA, then W_o)
+    cfg, zk, zv, Bk, Bv, q = _rand_case(H=H, h_kv=h_kv, m=1, n=60)
+    n, d, model = zk.shape[0], cfg.d_h, 48
+    rng = np.random.default_rng(7)
+    W_o = rng.standard_normal((H * d, model)) / np.sqrt(H * d)
+    bt, n_pages = gen.make_block_table([n])
+    cache = O.new_cache(cfg, n_pages)
+    # unquantised comparison: write latents and compare against the dequantised ones
+    O.write_latents(cache, gen.slots_for(bt, 0, np.arange(n)), zk.astype(np.float32), zv.astype(np.float32))
+    y = O.decode_out(cache, q, Bk, Bv, W_o, bt, [n])
+    zkh, zvh = O.gather_sequence(cache, bt[0], n)
+    zkh, zvh = O.unrotate_fp64(zkh, cfg.key.g), O.unrotate_fp64(zvh, cfg.val.g)
+    dense = _sdpa_materialised(cfg, zkh, zvh, Bk, Bv, q, [n - 1]).reshape(1, H * d) @ W_o
+    np.testing.assert_allclose(y, dense, atol=1e-12, rtol=0)
+    # fused factor: for each head, (p_h Z_v) (B_v[:, kv] W_o,h)
+    fused = np.zeros((1, model))
+    for h in range(H):
+        kv = h // cfg.group
+        k = hf_rope(zkh[:, kv] @ Bk[kv], np.arange(n), cfg.rope_base)
+        qr = hf_rope(q[:, h], [n - 1], cfg.rope_base)
+        s = (qr @ k.T) / np.sqrt(d)
+        p = np.exp(s - s.max())
+        p /= p.sum()
+        F = Bv[:, kv * d:(kv + 1) * d] @ W_o[h * d:(h + 1) * d]
+        fused += (p @ zvh) @ F
+    np.testing.assert_allclose(y, fused, atol=1e-12, rtol=0)

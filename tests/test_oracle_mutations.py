@@ -285,6 +285,18 @@ def merge_slices_k(drop_l=False, flip=False):
     return merge_slices
 
 
+def decode_out_k(kv_rows=False):
+    def decode_out(cache, q, B_k, B_v, W_o, block_table, seq_lens):
+        cfg = cache.cfg
+        o = OM.decode(cache, q, B_k, B_v, block_table, seq_lens)
+        W_o = np.asarray(W_o, np.float64)
+        if not kv_rows:
+            return o.reshape(o.shape[0], cfg.H * cfg.d_h) @ W_o
+        d = cfg.d_h
+        return sum(o[:, h] @ W_o[(h // cfg.group) * d:(h // cfg.group + 1) * d] for h in range(cfg.H))
+    return decode_out
+
+
 def prefill_k(shift=0):
     def prefill(cache, q, cu_q, B_k, B_v, block_table, seq_lens, select=None, heads=None):
         cfg = cache.cfg
@@ -354,6 +366,7 @@ PINS = {
     "decode_slice": [lambda: TA.test_slices_merge_to_the_whole_decode(0),
                      lambda: TA.test_slice_statistics_against_materialised_scores()],
     "merge_slices": [lambda: TA.test_slices_merge_to_the_whole_decode(0)],
+    "decode_out": [lambda: TA.test_output_projection_equals_fused_factor_and_dense(8, 2)],
     "eq14_mean_bits": [lambda: TB.test_eq14_printed_values()],
     "eq16_retained_fraction": [lambda: TB.test_eq16_printed_values()],
 }
@@ -365,7 +378,7 @@ FAITHFUL = {
     "pack_region": pack_k(), "write_latents": write_k(), "gather_sequence": gather_k(),
     "attend_latents": attend_k(), "partial_softmax": partial_k(), "lse_merge": merge_k(),
     "eq14_mean_bits": eq14_k(), "eq16_retained_fraction": eq16_k(), "project": project_k(), "prefill": prefill_k(),
-    "decode_slice": decode_slice_k(), "merge_slices": merge_slices_k(),
+    "decode_slice": decode_slice_k(), "merge_slices": merge_slices_k(), "decode_out": decode_out_k(),
 }
 
 PLANTS = {
@@ -406,6 +419,7 @@ PLANTS = {
     "slice query at the slice's last position": ("decode_slice", decode_slice_k(q_at_end_of_slice=True)),
     "slice merge without the slice sums": ("merge_slices", merge_slices_k(drop_l=True)),
     "slice merge weights e^(M - m)": ("merge_slices", merge_slices_k(flip=True)),
+    "output projection rows of the KV head": ("decode_out", decode_out_k(kv_rows=True)),
     "eq. 14 bit widths swapped": ("eq14_mean_bits", eq14_k(swap=True)),
     "eq. 16 drops the exempt layers": ("eq16_retained_fraction", eq16_k(drop_exempt=True)),
 }

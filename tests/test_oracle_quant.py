@@ -259,3 +259,17 @@ def test_quantize_latent_scale_per_group_on_hand_built_input():
         assert zp[0, gi] == np.float16(np.float32(seg.min()))
         # the range is the ramp's (gi + 1) * 0.25 * 15 to within the rotation's rounding
         assert abs((seg.max() - seg.min()) - (gi + 1) * 0.25 * 15) < 1e-4
+
+
+@pytest.mark.parametrize("r", [16, 64, 512])
+def test_uniform_4bit_variant_quantises_every_group_at_4_bits(r):
+    # the review's four-bit cache (section 6.1, the speed ablation of section 8.1):
+    # top_fraction 1.0 puts every channel in the 4-bit block; mean width 4 bits
+    rng = np.random.default_rng(r + 1)
+    lat = O.latent_split(r, 1.0)
+    assert (lat.n_top, lat.n_bot, lat.g) == (r, 0, 16)
+    z = (rng.standard_normal((32, r)) * rng.uniform(0.5, 4.0, (32, 1))).astype(np.float32)
+    codes, s, zp = O.quantize_latent(z, lat)
+    assert np.all(codes.reshape(32, -1, 16).max(axis=2) == 15)
+    assert O.eq14_mean_bits(1.0) == 4.0
+    assert lat.payload_bytes == 16 * r * 4 // 8

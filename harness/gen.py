@@ -85,6 +85,7 @@ class Workload:
     top_fraction: float = 0.25
     steps: int = 0    # decode steps with one appended token each (long-context run)
     chunk: int = 0    # prefill: tokens appended then attended causally
+    fp16_latent: bool = False  # the unquantised storage variant
 
 
 WORKLOADS = {

@@ -82,6 +82,18 @@ enum {
 /* Opaque stream handle: pass a cudaStream_t. */
 typedef struct CUstream_st* starkv_stream_t;
 
+/* Latent storage variants (starkv_config.flags).
+ * 0: mixed precision, the leading top_fraction of each latent's channels at 4
+ *    bits and the rest at 3 bits ([Review] section 6.1, eq. 14); top_fraction
+ *    1.0 gives the uniform 4-bit cache of the review's speed ablation.
+ * STARKV_FLAG_FP16_LATENT: the unquantised variant, every rotated latent value
+ *    stored as fp16 ([Review] section 8.1, the unquantised rank-75% rows);
+ *    top_fraction is ignored, the rotation group is 16 channels, and a region
+ *    of a page is group tiles of 16 tokens x 16 channels, element (t, c) at
+ *    fp16 index t*16 + c (512 bytes per tile, no metadata: the k_meta and
+ *    v_meta pools have 0 bytes and may be NULL). */
+#define STARKV_FLAG_FP16_LATENT 1
+
 /* Model shape and quantisation settings.
  * top_fraction: share of each latent's leading channels (singular-value order)
  *   stored at 4 bits; the rest are stored at 3 bits ([Review] eq. 14; the
@@ -103,7 +115,7 @@ typedef struct starkv_config {
   int32_t rank_k;       /* r_k: key latent rank per KV head             */
   int32_t rank_v;       /* R: joint value latent rank                   */
   int32_t max_position; /* positions [0, max_position) are supported    */
-  int32_t flags;        /* reserved, must be 0                          */
+  int32_t flags;        /* 0, or STARKV_FLAG_FP16_LATENT                */
   double top_fraction;  /* 0.25                                         */
   double rope_base;     /* RoPE theta base (1e4 Llama-2, 5e5 Llama-3)   */
 } starkv_config;

@@ -45,11 +45,13 @@ class QuantError(ValueError):
 # ----------------------------------------------------------------------------
 @dataclasses.dataclass(frozen=True)
 class Latent:
-    """Geometry of one latent: a KV head's key latent, or the joint value latent."""
+    """Geometry of one latent: a KV head's key latent, or the joint value latent.
+    fp16: the unquantised variant ([Review] section 8.1): rotated values stored as fp16."""
     r: int
     n_top: int
     n_bot: int
     g: int
+    fp16: bool = False
 
     @property
     def n_groups(self) -> int:
@@ -60,11 +62,15 @@ class Latent:
         return self.n_top // self.g
 
     def group_bits(self, gi: int) -> int:
+        if self.fp16:
+            return 16
         return 4 if gi < self.n_top_groups else 3
 
     @property
     def payload_bytes(self) -> int:
-        """Packed code bytes of one page (16 tokens): 16 * (4 n_top + 3 n_bot) / 8."""
+        """Packed bytes of one page (16 tokens): 16 * (4 n_top + 3 n_bot) / 8, or 16 r fp16 values."""
+        if self.fp16:
+            return 32 * self.r
         return 2 * (4 * self.n_top + 3 * self.n_bot)
 
     @property
@@ -74,8 +80,8 @@ class Latent:
 
     @property
     def meta_bytes(self) -> int:
-        """fp16 (scale, zero) per group per token, for one page."""
-        return self.n_groups * PAGE * 4
+        """fp16 (scale, zero) per group per token, for one page (none for fp16 latents)."""
+        return 0 if self.fp16 else self.n_groups * PAGE * 4
 
 
 def latent_split(r: int, top_fraction: float = 0.25) -> Latent:
@@ -84,6 +90,14 @@ def latent_split(r: int, top_fraction: float = 0.25) -> Latent:
     n_bot = r - n_top
     g = gcd(16, gcd(n_top, n_bot))
     return Latent(r, n_top, n_bot, g)
+
+
+def latent_fp16(r: int) -> Latent:
+    """The unquantised variant ([Review] section 8.1, the unquantised rows of the
+    attention-speed ablation): every rotated value stored as fp16; the rotation
+    groups are 16 channels (the rotation is exact in real arithmetic and folded
+    into the up-projections either way, eq. 13)."""
+    return Latent(r, 0, r, 16, True)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -96,14 +110,15 @@ class Config:
     R: int
     top_fraction: float = 0.25
     rope_base: float = 10000.0
+    fp16_latent: bool = False
 
     @property
     def key(self) -> Latent:
-        return latent_split(self.r_k, self.top_fraction)
+        return latent_fp16(self.r_k) if self.fp16_latent else latent_split(self.r_k, self.top_fraction)
 
     @property
     def val(self) -> Latent:
-        return latent_split(self.R, self.top_fraction)
+        return latent_fp16(self.R) if self.fp16_latent else latent_split(self.R, self.top_fraction)
 
     @property
     def group(self) -> int:
@@ -113,7 +128,8 @@ class Config:
 def config_of(w) -> Config:
     """Oracle config from a workload description (shape numbers only)."""
     return Config(H=w.H, h_kv=w.h_kv, d_h=w.d_h, hidden=w.hidden, r_k=w.r_k, R=w.R,
-                  top_fraction=w.top_fraction, rope_base=w.rope_base)
+                  top_fraction=w.top_fraction, rope_base=w.rope_base,
+                  fp16_latent=bool(getattr(w, "fp16_latent", False)))
 
 
 # ----------------------------------------------------------------------------
@@ -202,6 +218,13 @@ def quantize_latent(z, lat: Latent):
     """
     z = np.asarray(z, np.float32)
     n = z.shape[0]
+    if lat.fp16:
+        # unquantised variant: fl16 of the rotated values; no scale or zero
+        with np.errstate(over="ignore"):
+            v = rotate_fl32(z, lat.g).astype(np.float16)
+        if not np.isfinite(v).all():
+            raise QuantError("fp16 latent overflow")
+        return v, None, None
     zr = rotate_fl32(z, lat.g).reshape(n, lat.n_groups, lat.g)
     codes = np.empty((n, lat.n_groups, lat.g), np.uint8)
     s = np.empty((n, lat.n_groups), np.float16)
@@ -215,7 +238,10 @@ def quantize_latent(z, lat: Latent):
 
 
 def dequantize_codes(codes, s, zp, lat: Latent) -> np.ndarray:
-    """z^ = fl32(code * s + zp) per element (rotated domain).  code*s is exact in fp32."""
+    """z^ = fl32(code * s + zp) per element (rotated domain).  code*s is exact in fp32.
+    fp16 latents: the stored fp16 value."""
+    if lat.fp16:
+        return np.asarray(codes, np.float16).astype(np.float32)
     n = codes.shape[0]
     c = codes.reshape(n, lat.n_groups, lat.g).astype(np.float32)
     zh = c * s.astype(np.float32)[..., None] + zp.astype(np.float32)[..., None]
@@ -238,6 +264,13 @@ def pack_region(codes, s, zp, lat: Latent):
     1-bit plane of the high bit (element i at bit i mod 8 of byte i // 8).
     meta[p, group, t] = fp16 scale in the low half, fp16 zero in the high half.
     """
+    if lat.fp16:
+        # tiles of 16 tokens x g channels in channel order; element (t, c) at fp16 index t g + c
+        v = np.asarray(codes, np.float16)
+        P = v.shape[0] // PAGE
+        tiles = v.reshape(P, PAGE, lat.n_groups, lat.g).transpose(0, 2, 1, 3)       # [P, G, 16, g]
+        out = np.ascontiguousarray(tiles).view(np.uint8).reshape(P, lat.region_bytes)
+        return out.copy(), np.zeros((P, 0, PAGE), np.uint32)
     codes = np.asarray(codes, np.uint8)
     P = codes.shape[0] // PAGE
     g = lat.g
@@ -267,6 +300,9 @@ def unpack_region(data, meta, lat: Latent):
     data = np.asarray(data, np.uint8)
     P = data.shape[0]
     g = lat.g
+    if lat.fp16:
+        tiles = np.ascontiguousarray(data[:, :lat.payload_bytes]).view(np.float16).reshape(P, lat.n_groups, PAGE, g)
+        return tiles.transpose(0, 2, 1, 3).reshape(P * PAGE, lat.r).copy(), None, None
     c = np.empty((P, lat.n_groups, PAGE * g), np.uint8)
     off = 0
     for gi in range(lat.n_groups):
@@ -299,6 +335,10 @@ def quantize_pack_region(z, lat: Latent):
     n = z.shape[0]
     P = (n + PAGE - 1) // PAGE
     codes, s, zp = quantize_latent(z, lat)
+    if lat.fp16:
+        vv = np.zeros((P * PAGE, lat.r), np.float16)
+        vv[:n] = codes
+        return pack_region(vv, None, None, lat)
     cc = np.zeros((P * PAGE, lat.r), np.uint8)
     ss = np.zeros((P * PAGE, lat.n_groups), np.float16)
     zz = np.zeros((P * PAGE, lat.n_groups), np.float16)
@@ -309,6 +349,8 @@ def quantize_pack_region(z, lat: Latent):
 def dequantize_region(data, meta, lat: Latent, n: int) -> np.ndarray:
     """z^ (rotated domain, fp32) of the first n tokens of packed pages."""
     codes, s, zp = unpack_region(data, meta, lat)
+    if lat.fp16:
+        return dequantize_codes(codes[:n], None, None, lat)
     return dequantize_codes(codes[:n], s[:n], zp[:n], lat)
 
 
@@ -326,11 +368,13 @@ class Cache:
 
 def new_cache(cfg: Config, n_pages: int) -> Cache:
     k, v = cfg.key, cfg.val
+    mk = 0 if k.fp16 else k.n_groups   # fp16 latents carry no metadata
+    mv = 0 if v.fp16 else v.n_groups
     return Cache(cfg,
                  np.zeros((n_pages, cfg.h_kv, k.region_bytes), np.uint8),
                  np.zeros((n_pages, v.region_bytes), np.uint8),
-                 np.zeros((n_pages, cfg.h_kv, k.n_groups, PAGE), np.uint32),
-                 np.zeros((n_pages, v.n_groups, PAGE), np.uint32))
+                 np.zeros((n_pages, cfg.h_kv, mk, PAGE), np.uint32),
+                 np.zeros((n_pages, mv, PAGE), np.uint32))
 
 
 def write_latents(cache: Cache, slots, z_k, z_v) -> None:
@@ -346,6 +390,17 @@ def write_latents(cache: Cache, slots, z_k, z_v) -> None:
     pages, offs = slots // PAGE, slots % PAGE
     upages, inv = np.unique(pages, return_inverse=True)
     rows = inv * PAGE + offs
+    if cfg.fp16_latent:
+        for h in range(cfg.h_kv):
+            v, _, _ = quantize_latent(np.asarray(z_k)[:, h], cfg.key)
+            vv, _, _ = unpack_region(cache.k_codes[upages, h], None, cfg.key)
+            vv[rows] = v
+            cache.k_codes[upages, h] = pack_region(vv, None, None, cfg.key)[0]
+        v, _, _ = quantize_latent(z_v, cfg.val)
+        vv, _, _ = unpack_region(cache.v_codes[upages], None, cfg.val)
+        vv[rows] = v
+        cache.v_codes[upages] = pack_region(vv, None, None, cfg.val)[0]
+        return
     for h in range(cfg.h_kv):
         codes, s, zp = quantize_latent(np.asarray(z_k)[:, h], cfg.key)
         cc, ss, zz = unpack_region(cache.k_codes[upages, h], cache.k_meta[upages, h], cfg.key)

@@ -49,7 +49,20 @@ int gcd_int(int a, int b) {
 
 // Channel split of an r-channel latent: n_top = floor(top_fraction * r + 0.5),
 // g = gcd(16, n_top, r - n_top).
-bool make_geom(int r, double frac, LatentGeom* L) {
+bool make_geom(int r, double frac, bool fp16, LatentGeom* L) {
+  if (fp16) {
+    if (r % 16 != 0) return false;
+    L->r = r;
+    L->n_top = 0;
+    L->g = 16;
+    L->groups = r / 16;
+    L->top_groups = 0;
+    L->payload_bytes = 32 * r;
+    L->region_bytes = 32 * r;
+    L->fp16 = 1;
+    return true;
+  }
+  L->fp16 = 0;
   const int n_top = (int)floor(frac * r + 0.5);
   const int n_bot = r - n_top;
   if (n_top < 0 || n_bot < 0) return false;
@@ -70,7 +83,8 @@ starkv_status check_config(const starkv_config* c, LatentGeom* key, LatentGeom* 
   if (c->num_q_heads <= 0 || c->num_kv_heads <= 0 || c->head_dim <= 0 || c->hidden <= 0 ||
       c->rank_k <= 0 || c->rank_v <= 0 || c->max_position <= 0)
     return fail(STARKV_ERR_INVALID_ARG, "config sizes must be positive");
-  if (c->flags != 0) return fail(STARKV_ERR_INVALID_ARG, "config.flags must be 0");
+  if (c->flags != 0 && c->flags != STARKV_FLAG_FP16_LATENT)
+    return fail(STARKV_ERR_INVALID_ARG, "config.flags must be 0 or STARKV_FLAG_FP16_LATENT");
   if (c->num_q_heads > kMaxHeads || c->num_kv_heads > kMaxHeads || c->hidden > kMaxHidden)
     return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "num_q_heads, num_kv_heads <= %d and hidden <= %d", kMaxHeads,
                 kMaxHidden);
@@ -88,9 +102,10 @@ starkv_status check_config(const starkv_config* c, LatentGeom* key, LatentGeom* 
   if (c->hidden % 64 != 0) return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "hidden %% 64 != 0");
   if (c->max_position > (1 << 24)) return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "max_position too large");
   LatentGeom k, v;
-  if (!make_geom(c->rank_k, c->top_fraction, &k))
+  const bool fp16 = c->flags == STARKV_FLAG_FP16_LATENT;
+  if (!make_geom(c->rank_k, c->top_fraction, fp16, &k))
     return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "key latent: group size gcd(16, n_top, n_bot) must be 4, 8 or 16");
-  if (!make_geom(c->rank_v, c->top_fraction, &v))
+  if (!make_geom(c->rank_v, c->top_fraction, fp16, &v))
     return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "value latent: group size gcd(16, n_top, n_bot) must be 4, 8 or 16");
   if (key) *key = k;
   if (val) *val = v;
@@ -114,12 +129,12 @@ bool make_trig_map(Ctx* c) {
 starkv_status check_cache(const Ctx* c, const starkv_cache* cache) {
   if (!cache) return fail(STARKV_ERR_INVALID_ARG, "cache is NULL");
   if (cache->n_pages < 0) return fail(STARKV_ERR_INVALID_ARG, "cache.n_pages < 0");
-  if (cache->n_pages > 0 && (!cache->k_codes || !cache->v_codes || !cache->k_meta || !cache->v_meta))
+  const bool meta = !c->key.fp16;  // fp16 latents carry no metadata
+  if (cache->n_pages > 0 && (!cache->k_codes || !cache->v_codes || (meta && (!cache->k_meta || !cache->v_meta))))
     return fail(STARKV_ERR_INVALID_ARG, "cache pool pointer is NULL");
   if (!aligned16(cache->k_codes) || !aligned16(cache->v_codes) || !aligned16(cache->k_meta) ||
       !aligned16(cache->v_meta))
     return fail(STARKV_ERR_INVALID_ARG, "cache pools must be 16-byte aligned");
-  (void)c;
   return STARKV_OK;
 }
 
@@ -182,8 +197,8 @@ starkv_status starkv_cache_layout(const starkv_config* cfg, int64_t n_pages, sta
   out->value_groups = v.groups;
   out->k_codes_bytes = n_pages * cfg->num_kv_heads * (int64_t)k.region_bytes;
   out->v_codes_bytes = n_pages * (int64_t)v.region_bytes;
-  out->k_meta_bytes = n_pages * cfg->num_kv_heads * (int64_t)k.groups * kPage * 4;
-  out->v_meta_bytes = n_pages * (int64_t)v.groups * kPage * 4;
+  out->k_meta_bytes = k.fp16 ? 0 : n_pages * cfg->num_kv_heads * (int64_t)k.groups * kPage * 4;
+  out->v_meta_bytes = v.fp16 ? 0 : n_pages * (int64_t)v.groups * kPage * 4;
   return ok();
 }
 
@@ -573,9 +588,9 @@ starkv_status starkv_quantize_pack(starkv_ctx* ctx, int32_t which, const float* 
   Ctx* c = reinterpret_cast<Ctx*>(ctx);
   if (which != STARKV_LATENT_KEY && which != STARKV_LATENT_VALUE) return fail(STARKV_ERR_INVALID_ARG, "bad latent kind");
   if (n < 0) return fail(STARKV_ERR_INVALID_ARG, "n < 0");
-  if (n > 0 && (!z || !codes || !meta)) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
-  if (!aligned16(codes) || !aligned16(meta)) return fail(STARKV_ERR_INVALID_ARG, "codes/meta must be 16-byte aligned");
   const LatentGeom& L = which == STARKV_LATENT_KEY ? c->key : c->val;
+  if (n > 0 && (!z || !codes || (!meta && !L.fp16))) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
+  if (!aligned16(codes) || !aligned16(meta)) return fail(STARKV_ERR_INVALID_ARG, "codes/meta must be 16-byte aligned");
   cudaError_t e = launch_quantize_pack(*c, L, z, n, (uint8_t*)codes, (uint32_t*)meta, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "quantize_pack launch");
   return ok();
@@ -587,8 +602,8 @@ starkv_status starkv_dequantize(starkv_ctx* ctx, int32_t which, const void* code
   Ctx* c = reinterpret_cast<Ctx*>(ctx);
   if (which != STARKV_LATENT_KEY && which != STARKV_LATENT_VALUE) return fail(STARKV_ERR_INVALID_ARG, "bad latent kind");
   if (n < 0) return fail(STARKV_ERR_INVALID_ARG, "n < 0");
-  if (n > 0 && (!z_out || !codes || !meta)) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
   const LatentGeom& L = which == STARKV_LATENT_KEY ? c->key : c->val;
+  if (n > 0 && (!z_out || !codes || (!meta && !L.fp16))) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
   cudaError_t e = launch_dequantize(*c, L, (const uint8_t*)codes, (const uint32_t*)meta, n, z_out, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
   return ok();

@@ -145,8 +145,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeArgs a)
 #pragma unroll
         for (int c = 0; c < RK; ++c) {
           const int gi = c / a.key.g;
-          const float2 sz = unpack_meta(meta[gi * kPage + t]);
-          z[c] = __fmaf_rn((float)load_code(region, a.key, gi, t, c % a.key.g), sz.x, sz.y);
+          z[c] = latent_value(region, meta, a.key, gi, t, c % a.key.g);
         }
         const float2* rr = a.rope + (int64_t)j * half;
         float acc_s = 0.f;
@@ -191,8 +190,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeArgs a)
         const int ch = tid + k * kDecThreads;
         if (ch < R) {
           const int gi = ch / a.val.g;
-          const float2 sz = unpack_meta(meta[gi * kPage + t]);
-          const float zv = __fmaf_rn((float)load_code(region, a.val, gi, t, ch % a.val.g), sz.x, sz.y);
+          const float zv = latent_value(region, meta, a.val, gi, t, ch % a.val.g);
           acc[k] = fmaf(pt, zv, acc[k]);
         }
       }

@@ -353,6 +353,28 @@ __device__ __forceinline__ float key_dot(const uint8_t* region, const uint32_t* 
   return score;
 }
 
+// sum_c z_c G_c over one token's unquantised (fp16) key latent: tiles of 16
+// tokens x 16 channels, row t16 of tile gi holds channels 16 gi .. 16 gi + 15.
+template <int RK>
+__device__ __forceinline__ float key_dot_fp16(const uint8_t* region, int t16, const uint32_t (&raw)[RK]) {
+  const float* Gv = reinterpret_cast<const float*>(raw);
+  float acc[2] = {0.f, 0.f};
+#pragma unroll
+  for (int gi = 0; gi < RK / 16; ++gi) {
+    const uint4* row = reinterpret_cast<const uint4*>(region + gi * 512 + t16 * 32);
+    const uint4 u0 = row[0], u1 = row[1];
+    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+      acc[k & 1] = fmaf(f.x, Gv[gi * 16 + 2 * k], acc[k & 1]);
+      acc[k & 1] = fmaf(f.y, Gv[gi * 16 + 2 * k + 1], acc[k & 1]);
+    }
+  }
+  return acc[0] + acc[1];
+}
+
+// G: the key group size of quantised latents (4, 8, 16), or 0 for fp16 latents.
 template <int RK, int G>
 __global__ void __launch_bounds__(kAThreads, 1)
     decode_scores_kernel(const __grid_constant__ CUtensorMap trig_map, const ScoreArgs a) {
@@ -502,7 +524,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
             if ((lane & 1) == 0)
               bulk_g2s(sm + a.off_codes + ks * a.codes_stage + p * a.codes_pitch,
                        a.k_codes + ((int64_t)pid * a.h_kv + kv0) * a.key.region_bytes, a.codes_page, &kfull[ks]);
-            else
+            else if (a.meta_page)  // fp16 latents carry no metadata
               bulk_g2s(sm + a.off_meta + ks * a.meta_stage + p * a.meta_pitch,
                        a.k_meta + ((int64_t)pid * a.h_kv + kv0) * a.key.groups * kPage, a.meta_page, &kfull[ks]);
           }
@@ -564,8 +586,8 @@ __global__ void __launch_bounds__(kAThreads, 1)
           mloc[i] = fmaxf(mloc[i], score);
         };
         const int hl0 = hq * hper;
-        if constexpr (RK >= 64) {
-          // one 64-column row per head (a 256-column accumulator holds 4 heads: one per warp)
+        if constexpr (RK >= 64 || G == 0) {
+          // one RK-column row per head at a time
 #pragma unroll
           for (int hh = 0; hh < 4; ++hh) {
             if (hh >= hper) break;
@@ -575,8 +597,11 @@ __global__ void __launch_bounds__(kAThreads, 1)
             float sc = -INFINITY;
             if (valid) {
               const int kA = (h0 + hl0 + hh) / a.group - kv0;
-              sc = key_dot<RK, G>(cstage + kA * a.key.region_bytes, mstage + kA * a.key.groups * kPage,
-                                  a.key.top_groups, t16, rA);
+              if constexpr (G == 0)
+                sc = key_dot_fp16<RK>(cstage + kA * a.key.region_bytes, t16, rA);
+              else
+                sc = key_dot<RK, G>(cstage + kA * a.key.region_bytes, mstage + kA * a.key.groups * kPage,
+                                    a.key.top_groups, t16, rA);
             }
             finish(hh, sc);
           }
@@ -793,7 +818,7 @@ __global__ void __launch_bounds__(kVThreads, 1)
               if (((i - nbox) & 1) == 0)
                 bulk_g2s(sm + a.off_codes + cs * a.codes_stage + p * a.codes_pitch,
                          a.v_codes + (int64_t)pid * V.region_bytes, a.codes_page, &cfull[cs]);
-              else
+              else if (a.meta_page)  // fp16 latents carry no metadata
                 bulk_g2s(sm + a.off_meta + cs * a.meta_stage + p * a.meta_pitch,
                          a.v_meta + (int64_t)pid * V.groups * kPage, a.meta_page, &cfull[cs]);
             }
@@ -888,7 +913,12 @@ __global__ void __launch_bounds__(kVThreads, 1)
           const int gi = mt * 8 + gsel + 2 * i;
           cz[2 * i] = make_uint4(0, 0, 0, 0);
           cz[2 * i + 1] = make_uint4(0, 0, 0, 0);
-          if (tvalid && gi < V.groups) {
+          if (tvalid && gi < V.groups && V.fp16) {
+            // unquantised latents: the row of the group's tile, channels in order
+            const uint4* row = reinterpret_cast<const uint4*>(region + gi * 512 + t16 * 32);
+            cz[2 * i] = row[0];
+            cz[2 * i + 1] = row[1];
+          } else if (tvalid && gi < V.groups) {
             const uint32_t mw = meta[gi * kPage + t16];
             if (gi < V.top_groups)
               dequant16_4bit(region + gi * 128 + 8 * t16, mw, cz[2 * i], cz[2 * i + 1]);
@@ -940,7 +970,7 @@ __global__ void __launch_bounds__(kVThreads, 1)
       for (int mt = warp >> 2; mt < a.MT; mt += groups4) {
         const int mpos = mt * 128 + q4 * 32 + lane;
         const int gidx = mpos >> 4;
-        const int ch = gidx * 16 + value_channel_of_position(mpos & 15, gidx < V.top_groups);
+        const int ch = V.fp16 ? mpos : gidx * 16 + value_channel_of_position(mpos & 15, gidx < V.top_groups);
         for (int c0 = 0; c0 < a.N; c0 += 16) {
           float acc[16];
 #pragma unroll
@@ -1274,10 +1304,21 @@ cudaError_t launch_merge_slices(const float* o_parts, const float* ml_parts, int
 // ===========================================================================
 // host side
 // ===========================================================================
+// Query heads per score CTA: up to 256 accumulator columns (hpc * r_k); with
+// fp16 key latents also at most 32 KiB of key pages per 128-token stage.
+static int score_hpc(const starkv_config& cfg) {
+  const int rk = cfg.rank_k;
+  const int group = cfg.num_q_heads / cfg.num_kv_heads;
+  int hpc = (256 / rk) < cfg.num_q_heads ? 256 / rk : cfg.num_q_heads;
+  if (cfg.flags & STARKV_FLAG_FP16_LATENT)
+    while (hpc > 4 && hpc > group && kPagesPerTile * (hpc / group) * 32 * rk > 32768) hpc /= 2;
+  return hpc;
+}
+
 bool tc_decode_supported(const starkv_config& cfg) {
   const int rk = cfg.rank_k;
   if (rk != 16 && rk != 32 && rk != 64) return false;
-  const int hpc = (256 / rk) < cfg.num_q_heads ? 256 / rk : cfg.num_q_heads;
+  const int hpc = score_hpc(cfg);
   const int group = cfg.num_q_heads / cfg.num_kv_heads;
   if (cfg.num_q_heads % hpc != 0 || hpc % 4 != 0) return false;
   if (hpc % group != 0 && group % hpc != 0) return false;
@@ -1315,7 +1356,7 @@ struct VSmem {
 bool value_smem(const Ctx& c, int N, int nW, int PS, int ST, int stages_total, int splits, VSmem& v) {
   const starkv_config& f = c.cfg;
   v.codes_page = c.val.region_bytes;
-  v.meta_page = c.val.groups * kPage * 4;
+  v.meta_page = c.val.fp16 ? 0 : c.val.groups * kPage * 4;
   v.codes_pitch = v.codes_page + 64;
   v.meta_pitch = v.meta_page + 64;
   v.codes_stage = PS * v.codes_pitch;
@@ -1410,7 +1451,7 @@ struct TcLayout {
 TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
   TcLayout t;
   const starkv_config& f = c.cfg;
-  t.hpc = (256 / f.rank_k) < f.num_q_heads ? 256 / f.rank_k : f.num_q_heads;
+  t.hpc = score_hpc(f);
   t.kvpc = t.hpc / c.group;
   t.ncols = t.hpc * f.rank_k;
   t.HG = f.num_q_heads / t.hpc;
@@ -1441,7 +1482,8 @@ TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
     int s0 = sms / bt;
     if (s0 > t.stages_total) s0 = t.stages_total;
     if (s0 < 1) s0 = 1;
-    const double tok_bytes = (double)c.val.region_bytes / kPage + c.val.groups * 4.0 + f.num_q_heads * 4.0;
+    const double tok_bytes =
+        (double)c.val.region_bytes / kPage + (c.val.fp16 ? 0.0 : c.val.groups * 4.0) + f.num_q_heads * 4.0;
     const double work = (double)bt * t.tpad * tok_bytes;
     const double part_unit = 2.0 * f.num_q_heads * f.rank_v * 4.0;
     const int threads = (kVRoleWarps + t.nW) * 32;
@@ -1536,6 +1578,7 @@ static cudaError_t launch_scores_g(const Ctx& c, const ScoreArgs& a, int grid, s
 
 template <int RK>
 static cudaError_t launch_scores(const Ctx& c, const ScoreArgs& a, int grid, size_t smem, cudaStream_t s) {
+  if (c.key.fp16) return launch_scores_g<RK, 0>(c, a, grid, smem, s);
   switch (c.key.g) {
     case 4: return launch_scores_g<RK, 4>(c, a, grid, smem, s);
     case 8: return launch_scores_g<RK, 8>(c, a, grid, smem, s);
@@ -1629,7 +1672,7 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   A.status = c.status;
   A.trig_stage = kT * d * 2;
   A.codes_page = t.kvpc * c.key.region_bytes;
-  A.meta_page = t.kvpc * c.key.groups * kPage * 4;
+  A.meta_page = c.key.fp16 ? 0 : t.kvpc * c.key.groups * kPage * 4;
   A.codes_pitch = (A.codes_page + 64 + 127) / 128 * 128 - 64;  // = 64 mod 128: the two pages a warp reads
   A.meta_pitch = (A.meta_page + 64 + 127) / 128 * 128 - 64;    // fall on different banks
   A.codes_stage = kPagesPerTile * A.codes_pitch;

@@ -16,16 +16,18 @@ constexpr int kPage = STARKV_PAGE_TOKENS;
 // Geometry of one latent (a KV head's key latent, or the joint value latent).
 struct LatentGeom {
   int r;             // channels
-  int n_top;         // leading 4-bit channels
-  int g;             // rotation / quantisation group size (4, 8 or 16)
+  int n_top;         // leading 4-bit channels (0 for fp16 latents)
+  int g;             // rotation / quantisation group size (4, 8 or 16; 16 for fp16 latents)
   int groups;        // r / g
   int top_groups;    // n_top / g
-  int payload_bytes; // 2 * (4 n_top + 3 (r - n_top)) per page
+  int payload_bytes; // 2 * (4 n_top + 3 (r - n_top)) per page; 32 r for fp16 latents
   int region_bytes;  // payload rounded up to 16
+  int fp16;          // 1: unquantised fp16 latents (tiles of 16 tokens x g channels, no metadata)
 };
 
 // Byte offset of group tile `gi` inside a page region.
 __host__ __device__ inline int tile_offset(const LatentGeom& L, int gi) {
+  if (L.fp16) return gi * 32 * L.g;
   return gi < L.top_groups ? gi * 8 * L.g : L.top_groups * 8 * L.g + (gi - L.top_groups) * 6 * L.g;
 }
 
@@ -250,6 +252,16 @@ __device__ inline float2 unpack_meta(uint32_t m) {
   return make_float2(__half2float(__half(s)), __half2float(__half(z)));
 }
 
+// Stored value of element (t, c) of group gi of a page region, rotated domain:
+// code * s + zp (fp32, exact product) for quantised latents, the fp16 value for
+// unquantised ones.  meta_page: the region's [groups][16] metadata (unused for fp16).
+__device__ inline float latent_value(const uint8_t* region, const uint32_t* meta_page, const LatentGeom& L, int gi,
+                                     int t, int c) {
+  if (L.fp16) return __half2float(reinterpret_cast<const __half*>(region + tile_offset(L, gi))[t * L.g + c]);
+  const float2 sz = unpack_meta(meta_page[gi * kPage + t]);
+  return __fmaf_rn((float)load_code(region, L, gi, t, c), sz.x, sz.y);
+}
+
 // ---------------------------------------------------------------------------
 // Rotate + quantise + store one group of one token (shared by append and the
 // quantise entry).  x: the group's g pre-rotation latents.
@@ -262,6 +274,26 @@ __device__ inline void rotate_quantize_store(const float* x_in, const LatentGeom
 #pragma unroll
   for (int i = 0; i < G; ++i) x[i] = x_in[i];
   fwht_fl32<G>(x);
+  if (L.fp16) {
+    // unquantised latent: fl16 of the rotated values, row t of the group's tile
+    uint32_t h[G / 2];
+    bool finite = true;
+#pragma unroll
+    for (int i = 0; i < G; i += 2) {
+      const __half2 v = __floats2half2_rn(x[i], x[i + 1]);
+      finite = finite && isfinite(__low2float(v)) && isfinite(__high2float(v));
+      h[i / 2] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    if (!finite) {
+      set_status(status, STARKV_DEV_QUANT_OVERFLOW);
+#pragma unroll
+      for (int i = 0; i < G / 2; ++i) h[i] = 0u;
+    }
+    uint4* dst = reinterpret_cast<uint4*>(region + tile_offset(L, gi) + t * G * 2);
+#pragma unroll
+    for (int i = 0; i < G / 8; ++i) dst[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+    return;
+  }
   uint8_t code[G];
   __half s16, zp16;
   const int bits = gi < L.top_groups ? 4 : 3;

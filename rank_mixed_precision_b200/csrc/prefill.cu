@@ -85,8 +85,8 @@ __global__ void __launch_bounds__(256) prefill_simt_expand_kernel(PrefillArgs a,
     if (ok_len && j0 + t2 < L && page >= 0) {
       const int t = (j0 + t2) % kPage, gi = c / a.key.g;
       const uint8_t* region = a.k_codes + ((int64_t)page * a.h_kv + kv) * a.key.region_bytes;
-      const float2 sz = unpack_meta(a.k_meta[(((int64_t)page * a.h_kv + kv) * a.key.groups + gi) * kPage + t]);
-      z = __fmaf_rn((float)load_code(region, a.key, gi, t, c % a.key.g), sz.x, sz.y);
+      z = latent_value(region, a.k_meta + ((int64_t)page * a.h_kv + kv) * a.key.groups * kPage, a.key, gi, t,
+                       c % a.key.g);
     }
     Zk[t2][c] = z;
   }
@@ -127,8 +127,7 @@ __global__ void __launch_bounds__(256) prefill_simt_expand_kernel(PrefillArgs a,
       if (ch < R && ok_len && j0 + t2 < L && page >= 0) {
         const int t = (j0 + t2) % kPage, gi = ch / a.val.g;
         const uint8_t* region = a.v_codes + (int64_t)page * a.val.region_bytes;
-        const float2 sz = unpack_meta(a.v_meta[((int64_t)page * a.val.groups + gi) * kPage + t]);
-        z = __fmaf_rn((float)load_code(region, a.val, gi, t, ch % a.val.g), sz.x, sz.y);
+        z = latent_value(region, a.v_meta + (int64_t)page * a.val.groups * kPage, a.val, gi, t, ch % a.val.g);
       }
       Zv[t2][c] = z;
     }

@@ -174,9 +174,9 @@ __global__ void __launch_bounds__(kXThreadsW, 1)
     // ---------------- copies ----------------
     const int npg = __popc(__ballot_sync(0xffffffffu, lane < 8 && pg[lane < 8 ? lane : 0] >= 0));
     // key pages of the CTA's heads: codes (padded region) and metadata, one lane per copy
+    const uint32_t kmeta = a.kc_page - a.kc_codes;  // 0 for fp16 latents
     if (lane == 0) {
-      mbar_arrive_expect_tx(kfull, (uint32_t)(npg * nh) * (a.kc_codes + (uint32_t)a.key.groups * kPage * 4) +
-                                       (uint32_t)(nh * nsub * rk * 128));
+      mbar_arrive_expect_tx(kfull, (uint32_t)(npg * nh) * a.kc_page + (uint32_t)(nh * nsub * rk * 128));
       for (int hh = 0; hh < nh; ++hh)
         for (int i = 0; i < nsub; ++i)
           tma_load_2d(Bk + hh * a.bk_head + i * rk * 128, &bk_map, i * 64, (kv0 + hh) * rk, kfull);
@@ -190,8 +190,8 @@ __global__ void __launch_bounds__(kXThreadsW, 1)
       uint8_t* dst = Kc + (hh * 8 + p) * a.kc_page;
       if ((e & 1) == 0)
         bulk_g2s(dst, a.k_codes + reg * a.key.region_bytes, a.kc_codes, kfull);
-      else
-        bulk_g2s(dst + a.kc_codes, a.k_meta + reg * a.key.groups * kPage, (uint32_t)a.key.groups * kPage * 4, kfull);
+      else if (kmeta)
+        bulk_g2s(dst + a.kc_codes, a.k_meta + reg * a.key.groups * kPage, kmeta, kfull);
     }
     // value chunks
     for (int c = 0; c < nchunk; ++c) {
@@ -203,7 +203,8 @@ __global__ void __launch_bounds__(kXThreadsW, 1)
       }
       uint32_t coff, cbytes;
       value_chunk_span(V, c, coff, cbytes);
-      if (lane == 0) mbar_arrive_expect_tx(&cfull[s], (uint32_t)npg * (cbytes + 4 * kPage * 4));
+      const uint32_t vmeta = V.fp16 ? 0u : 4 * kPage * 4;
+      if (lane == 0) mbar_arrive_expect_tx(&cfull[s], (uint32_t)npg * (cbytes + vmeta));
       __syncwarp();
       if (lane < 16) {
         const int p = lane >> 1;
@@ -212,9 +213,8 @@ __global__ void __launch_bounds__(kXThreadsW, 1)
           uint8_t* dst = Vc + s * vstage + p * a.vc_page;
           if ((lane & 1) == 0)
             bulk_g2s(dst, a.v_codes + (int64_t)pid * V.region_bytes + coff, cbytes, &cfull[s]);
-          else
-            bulk_g2s(dst + a.vc_codes_max, a.v_meta + ((int64_t)pid * V.groups + 4 * c) * kPage, 4 * kPage * 4,
-                     &cfull[s]);
+          else if (vmeta)
+            bulk_g2s(dst + a.vc_codes_max, a.v_meta + ((int64_t)pid * V.groups + 4 * c) * kPage, vmeta, &cfull[s]);
         }
       }
       const int bs = c & 1;
@@ -274,8 +274,8 @@ __global__ void __launch_bounds__(kXThreadsW, 1)
           if (pg[p] >= 0 && tile * kTile + t < L) {
             const int t16 = t % kPage, gi = c / a.key.g;
             const uint8_t* page = Kc + (hh * 8 + p) * a.kc_page;
-            const float2 sz = unpack_meta(reinterpret_cast<const uint32_t*>(page + a.kc_codes)[gi * kPage + t16]);
-            z = __fmaf_rn((float)load_code(page, a.key, gi, t16, c % a.key.g), sz.x, sz.y);
+            z = latent_value(page, reinterpret_cast<const uint32_t*>(page + a.kc_codes), a.key, gi, t16,
+                             c % a.key.g);
           }
           *reinterpret_cast<__half*>(tileA + sw128_kmajor_offset(t, c, kTile)) = __float2half_rn(z);
         }
@@ -302,7 +302,12 @@ __global__ void __launch_bounds__(kXThreadsW, 1)
         const int gi = c * 4 + gq;
         const int p = t / kPage, t16 = t % kPage;
         uint4 c0 = make_uint4(0, 0, 0, 0), c1 = make_uint4(0, 0, 0, 0);
-        if (pg[p] >= 0 && tile * kTile + t < L) {
+        if (pg[p] >= 0 && tile * kTile + t < L && V.fp16) {
+          // unquantised latents: the row of the group's tile, channels in order
+          const uint4* row = reinterpret_cast<const uint4*>(st + p * a.vc_page + gq * 512 + t16 * 32);
+          c0 = row[0];
+          c1 = row[1];
+        } else if (pg[p] >= 0 && tile * kTile + t < L) {
           const uint8_t* page = st + p * a.vc_page;
           const uint32_t mw = reinterpret_cast<const uint32_t*>(page + a.vc_codes_max)[gq * kPage + t16];
           const uint32_t toff = (uint32_t)(tile_offset(V, gi) - tile_offset(V, c * 4));
@@ -735,10 +740,10 @@ XLayout expand_layout(const Ctx& c) {
   x.bk_head = (uint32_t)(d / 64) * rk * 128;
   x.bv_stage = (uint32_t)(x.HP * d / 64) * 8192;
   x.kc_codes = (uint32_t)c.key.region_bytes;                        // a multiple of 16
-  x.kc_page = x.kc_codes + (uint32_t)c.key.groups * kPage * 4;
-  // the largest 4-group span of the value region (all 4-bit groups)
-  x.vc_codes_max = 4 * 8 * (uint32_t)c.val.g;
-  x.vc_page = x.vc_codes_max + 4 * kPage * 4;
+  x.kc_page = x.kc_codes + (c.key.fp16 ? 0u : (uint32_t)c.key.groups * kPage * 4);
+  // the largest 4-group span of the value region (all 4-bit groups, or fp16 tiles)
+  x.vc_codes_max = c.val.fp16 ? 4 * 512u : 4 * 8 * (uint32_t)c.val.g;
+  x.vc_page = x.vc_codes_max + (c.val.fp16 ? 0u : 4 * kPage * 4);
   uint32_t o = 0;
   x.off_ak = o;
   o += x.HP * kTile * 128;
@@ -807,7 +812,10 @@ bool make_prefill_maps(Ctx* c) {
                      (uint64_t)f.num_kv_heads * f.rank_k, (uint64_t)f.head_dim * 2, 64, (uint32_t)f.rank_k,
                      CU_TENSOR_MAP_SWIZZLE_128B))
     return false;
-  return encode_map_2d(&c->bvp_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, c->Bv16p, (uint64_t)f.num_kv_heads * f.head_dim,
+  // the value A tiles hold channels in the order the dequantiser emits them
+  // (value_channel_of_position) for quantised latents, in plain order for fp16 ones
+  return encode_map_2d(&c->bvp_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, c->val.fp16 ? c->Bv16 : c->Bv16p,
+                       (uint64_t)f.num_kv_heads * f.head_dim,
                        (uint64_t)f.rank_v, (uint64_t)f.num_kv_heads * f.head_dim * 2, 64, 64,
                        CU_TENSOR_MAP_SWIZZLE_128B);
 }

@@ -72,8 +72,10 @@ cudaError_t launch_quantize_pack(const Ctx& c, const LatentGeom& L, const float*
   const int64_t pages = (n + kPage - 1) / kPage;
   cudaError_t e = cudaMemsetAsync(codes, 0, (size_t)pages * L.region_bytes, s);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(meta, 0, (size_t)pages * L.groups * kPage * 4, s);
-  if (e != cudaSuccess) return e;
+  if (!L.fp16) {  // fp16 latents carry no metadata
+    e = cudaMemsetAsync(meta, 0, (size_t)pages * L.groups * kPage * 4, s);
+    if (e != cudaSuccess) return e;
+  }
   const int64_t total = n * L.groups;
   if (total == 0) return cudaSuccess;
   quantize_pack_kernel<<<(unsigned)((total + 127) / 128), 128, 0, s>>>(L, z, n, codes, meta, c.status);
@@ -90,9 +92,7 @@ __global__ void dequantize_kernel(LatentGeom L, const uint8_t* __restrict__ code
   const int64_t page = tok / kPage;
   const int t = (int)(tok % kPage);
   const int gi = ch / L.g;
-  const int code = load_code(codes + page * L.region_bytes, L, gi, t, ch % L.g);
-  const float2 sz = unpack_meta(meta[(page * L.groups + gi) * kPage + t]);
-  z[idx] = __fmaf_rn((float)code, sz.x, sz.y);
+  z[idx] = latent_value(codes + page * L.region_bytes, meta + page * L.groups * kPage, L, gi, t, ch % L.g);
 }
 
 cudaError_t launch_dequantize(const Ctx&, const LatentGeom& L, const uint8_t* codes,

@@ -135,8 +135,11 @@ def _need(t, dtype, name, ndim=None):
 
 
 # ---------------------------------------------------------------------------
-def make_config(H, h_kv, d_h, hidden, r_k, R, max_position, top_fraction=0.25, rope_base=10000.0):
-    return starkv_config(H, h_kv, d_h, hidden, r_k, R, max_position, 0, top_fraction, rope_base)
+FLAG_FP16_LATENT = 1
+
+
+def make_config(H, h_kv, d_h, hidden, r_k, R, max_position, top_fraction=0.25, rope_base=10000.0, flags=0):
+    return starkv_config(H, h_kv, d_h, hidden, r_k, R, max_position, flags, top_fraction, rope_base)
 
 
 def starkv_version() -> str:

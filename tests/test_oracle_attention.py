@@ -306,3 +306,27 @@ def test_output_projection_equals_fused_factor_and_dense(H, h_kv):
         F = Bv[:, kv * d:(kv + 1) * d] @ W_o[h * d:(h + 1) * d]
         fused += (p @ zvh) @ F
     np.testing.assert_allclose(y, fused, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("wi", [0, 3])
+def test_fp16_variant_attention_close_to_unquantised(wi):
+    # the unquantised variant differs from exact latents only by fp16 rounding of
+    # the rotated values (relative 2^-11): far tighter than the 4/3-bit cache
+    w = gen.shrink(gen.workload(wi), ctx=200, fp16_latent=True)
+    cfg = O.config_of(w)
+    f = gen.make_factors(w)
+    zk, zv = gen.make_latents(w, 200)
+    bt, n_pages = gen.make_block_table([200])
+    cache = O.new_cache(cfg, n_pages)
+    O.write_latents(cache, gen.slots_for(bt, 0, np.arange(200)), zk, zv)
+    q = gen.make_queries(1, w.H, w.d_h)
+    got = O.decode(cache, q, f.B_k, f.B_v, bt, [200])
+    ref = O.attend_latents(cfg, zk, zv, q, [199], f.B_k, f.B_v)
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel < 2e-3
+    # and the 4/3-bit cache of the same latents is much further off
+    w43 = gen.shrink(w, fp16_latent=False)
+    c43 = O.new_cache(O.config_of(w43), n_pages)
+    O.write_latents(c43, gen.slots_for(bt, 0, np.arange(200)), zk, zv)
+    rel43 = np.linalg.norm(O.decode(c43, q, f.B_k, f.B_v, bt, [200]) - ref) / np.linalg.norm(ref)
+    assert rel43 > 4 * rel

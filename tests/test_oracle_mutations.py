@@ -105,10 +105,13 @@ def dequantize_k(zp_sign=1.0, half_step=False):
     return dequantize_codes
 
 
-def quantize_latent_k(all_bits=None, top_shift=0):
+def quantize_latent_k(all_bits=None, top_shift=0, fp16_unrotated=False):
     def quantize_latent(z, lat):
         z = np.asarray(z, np.float32)
         n = z.shape[0]
+        if lat.fp16:
+            v = (z if fp16_unrotated else OM.rotate_fl32(z, lat.g)).astype(np.float16)
+            return v, None, None
         zr = OM.rotate_fl32(z, lat.g).reshape(n, lat.n_groups, lat.g)
         codes = np.empty((n, lat.n_groups, lat.g), np.uint8)
         s = np.empty((n, lat.n_groups), np.float16)
@@ -124,8 +127,16 @@ def quantize_latent_k(all_bits=None, top_shift=0):
     return quantize_latent
 
 
-def pack_k(hi_first=False, planes_swapped=False, meta_swapped=False):
+def pack_k(hi_first=False, planes_swapped=False, meta_swapped=False, fp16_channel_major=False):
     def pack_region(codes, s, zp, lat):
+        if lat.fp16:
+            v = np.asarray(codes, np.float16)
+            P = v.shape[0] // OM.PAGE
+            tiles = v.reshape(P, OM.PAGE, lat.n_groups, lat.g).transpose(0, 2, 1, 3)
+            if fp16_channel_major:
+                tiles = tiles.transpose(0, 1, 3, 2)
+            return (np.ascontiguousarray(tiles).view(np.uint8).reshape(P, lat.region_bytes).copy(),
+                    np.zeros((P, 0, OM.PAGE), np.uint32))
         codes = np.asarray(codes, np.uint8)
         P = codes.shape[0] // OM.PAGE
         g = lat.g
@@ -352,9 +363,11 @@ PINS = {
                          lambda: TQ.test_constant_group_has_zero_scale()],
     "quantize_latent": [lambda: TQ.test_quantize_latent_bit_width_per_group(64),
                         lambda: TQ.test_quantize_latent_bit_width_per_group(32),
-                        lambda: TQ.test_quantize_latent_scale_per_group_on_hand_built_input()],
+                        lambda: TQ.test_quantize_latent_scale_per_group_on_hand_built_input(),
+                        lambda: TA.test_fp16_variant_attention_close_to_unquantised(0)],
     "pack_region": [lambda: TQ.test_pack_matches_hand_derived_bytes(),
-                    lambda: TQ.test_pack_unpack_exhaustive(32, 0.25)],
+                    lambda: TQ.test_pack_unpack_exhaustive(32, 0.25),
+                    lambda: TQ.test_fp16_variant_page_bytes_by_hand()],
     "write_latents": [lambda: TQ.test_write_latents_partial_pages_keep_other_rows()],
     "gather_sequence": [lambda: TA.test_decode_through_paged_cache_equals_direct()],
     "attend_latents": [lambda: TA.test_reassociated_equals_materialised(8, 2),
@@ -400,6 +413,8 @@ PLANTS = {
     "every group quantised at 4 bits": ("quantize_latent", quantize_latent_k(all_bits=4)),
     "4-bit block one group too wide": ("quantize_latent", quantize_latent_k(top_shift=1)),
     "4-bit block one group too narrow": ("quantize_latent", quantize_latent_k(top_shift=-1)),
+    "fp16 variant stores the unrotated latent": ("quantize_latent", quantize_latent_k(fp16_unrotated=True)),
+    "fp16 variant tiles channel-major": ("pack_region", pack_k(fp16_channel_major=True)),
     "4-bit tile: high nibble first": ("pack_region", pack_k(hi_first=True)),
     "3-bit tile: 1-bit plane before 2-bit plane": ("pack_region", pack_k(planes_swapped=True)),
     "metadata: zero in the low half": ("pack_region", pack_k(meta_swapped=True)),

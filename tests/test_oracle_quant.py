@@ -13,6 +13,7 @@ import pytest
 import scipy.linalg
 
 import oracle as O
+from harness import gen
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -273,3 +274,44 @@ def test_uniform_4bit_variant_quantises_every_group_at_4_bits(r):
     assert np.all(codes.reshape(32, -1, 16).max(axis=2) == 15)
     assert O.eq14_mean_bits(1.0) == 4.0
     assert lat.payload_bytes == 16 * r * 4 // 8
+
+
+def test_fp16_variant_page_bytes_by_hand():
+    # the unquantised variant's page layout (the library's own specification):
+    # group tiles of 16 tokens x 16 channels in channel order, element (t, c) at
+    # fp16 index t * 16 + c, little-endian; no metadata
+    lat = O.latent_fp16(32)
+    assert (lat.g, lat.n_groups, lat.region_bytes, lat.meta_bytes) == (16, 2, 1024, 0)
+    v = np.zeros((16, 32), np.float16)
+    v[3, 5] = 1.0          # 0x3C00 -> tile 0, index 53 -> bytes 106, 107
+    v[0, 18] = -2.0        # 0xC000 -> tile 1, index 2 -> bytes 512 + 4, 5
+    v[15, 31] = 0.5        # 0x3800 -> tile 1, index 255 -> bytes 1022, 1023
+    data, meta = O.pack_region(v, None, None, lat)
+    want = np.zeros(1024, np.uint8)
+    want[107], want[517], want[1023] = 0x3C, 0xC0, 0x38
+    np.testing.assert_array_equal(data[0], want)
+    assert meta.size == 0
+    back, _, _ = O.unpack_region(data, None, lat)
+    np.testing.assert_array_equal(back.view(np.uint16), v.view(np.uint16))
+
+
+def test_fp16_variant_keeps_exact_rotated_values():
+    # latents whose rotated values are small integers: the rotation is exact in
+    # fp32 and every rotated value is an fp16 number, so the store is lossless
+    rng = np.random.default_rng(8)
+    lat = O.latent_fp16(64)
+    k = rng.integers(-300, 301, (20, 64)).astype(np.float64)
+    z = O.unrotate_fp64(k, 16).astype(np.float32)          # H_g is its own inverse
+    data, _ = O.quantize_pack_region(z, lat)
+    zh = O.dequantize_region(data, None, lat, 20)
+    np.testing.assert_array_equal(zh, k.astype(np.float32))
+
+
+def test_fp16_variant_payload_against_eq1():
+    # unquantised latents at rank fraction rho: 16-bit payload, compression 1 / rho against eq. 1
+    w = gen.workload(1)
+    cfg = O.config_of(gen.shrink(w, fp16_latent=True))
+    dense = O.eq1_dense_payload_bytes(1, 1, 1, w.h_kv, w.d_h, 16)
+    rho = (w.h_kv * w.r_k + w.R) / (2 * w.h_kv * w.d_h)
+    assert dense / O.payload_bytes_per_token(cfg) == pytest.approx(1 / rho)
+    assert O.cache_bytes_per_token(cfg) == O.payload_bytes_per_token(cfg) == 2 * (w.h_kv * w.r_k + w.R)

@@ -86,6 +86,7 @@ class Workload:
     steps: int = 0    # decode steps with one appended token each (long-context run)
     chunk: int = 0    # prefill: tokens appended then attended causally
     fp16_latent: bool = False  # the unquantised storage variant
+    key_ranks: tuple = None    # ragged key ranks, one per KV head (r_k = their maximum)
 
 
 WORKLOADS = {
@@ -140,9 +141,18 @@ class Factors:
         return {k: bf16_bits(getattr(self, k)) for k in ("A_k", "A_v", "B_k", "B_v")}
 
 
+def key_ranks_of(w: Workload):
+    return list(w.key_ranks) if w.key_ranks is not None else [w.r_k] * w.h_kv
+
+
 def make_factors(w: Workload, seed: int = 0, a_std: float | None = None) -> Factors:
+    """Factors in the library's layout.  With ragged key ranks, A_k holds
+    sum_h r_h columns and B_k is [sum_h r_h, d_h] (head h's rows after the
+    earlier heads'); with uniform ranks B_k is [h_kv, r_k, d_h]."""
     hidden = w.hidden
     std = (1.0 / np.sqrt(hidden)) if a_std is None else a_std
+    if w.key_ranks is not None:
+        return _make_factors_ragged(w, seed, std)
     rk = rng_for("A_k", seed)
     ok = rng_for("outlier_k", seed)
     A_k = np.empty((hidden, w.h_kv * w.r_k), np.float64)
@@ -165,6 +175,28 @@ def make_factors(w: Workload, seed: int = 0, a_std: float | None = None) -> Fact
     return Factors(f(A_k), f(A_v), f(B_k), f(B_v), outk, outv.tolist())
 
 
+def _make_factors_ragged(w: Workload, seed: int, std: float) -> Factors:
+    ranks = key_ranks_of(w)
+    hidden = w.hidden
+    rk, ok, rb = rng_for("A_k", seed), rng_for("outlier_k", seed), rng_for("B_k", seed)
+    A_k = np.empty((hidden, sum(ranks)), np.float64)
+    B_k = np.empty((sum(ranks), w.d_h), np.float64)
+    outk, col = [], 0
+    for r in ranks:
+        sc, o = _latent_scale(r, ok)
+        A_k[:, col:col + r] = rk.standard_normal((hidden, r)) * std * sc
+        Q, _ = np.linalg.qr(rb.standard_normal((w.d_h, r)))
+        B_k[col:col + r] = Q.T
+        outk.append(o.tolist())
+        col += r
+    rv = rng_for("A_v", seed)
+    sc, outv = _latent_scale(w.R, rng_for("outlier_v", seed))
+    A_v = rv.standard_normal((hidden, w.R)) * std * sc
+    Q, _ = np.linalg.qr(rng_for("B_v", seed).standard_normal((w.h_kv * w.d_h, w.R)))
+    f = lambda a: to_bf16(a.astype(np.float32))[0]
+    return Factors(f(A_k), f(A_v), f(B_k), f(Q.T), outk, outv.tolist())
+
+
 def make_hidden(n: int, hidden: int, seed: int = 0, name: str = "X", sub: int = 0):
     """Hidden states X ~ N(0,1), bf16 values as float32 [n, hidden]."""
     x = rng_for(name, seed, sub).standard_normal((n, hidden), dtype=np.float32)
@@ -183,7 +215,13 @@ def make_latents(w: Workload, n: int, seed: int = 0, sub: int = 0):
     Returns (z_k [n, h_kv, r_k], z_v [n, R]).
     """
     ok = rng_for("outlier_k", seed)
-    sk = np.stack([_latent_scale(w.r_k, ok)[0] for _ in range(w.h_kv)])
+    if w.key_ranks is not None:
+        # ragged ranks: head h's first r_h channels, zero past its rank
+        sk = np.zeros((w.h_kv, w.r_k))
+        for h, r in enumerate(key_ranks_of(w)):
+            sk[h, :r] = _latent_scale(r, ok)[0]
+    else:
+        sk = np.stack([_latent_scale(w.r_k, ok)[0] for _ in range(w.h_kv)])
     sv = _latent_scale(w.R, rng_for("outlier_v", seed))[0]
     zk = rng_for("latent_k", seed, sub).standard_normal((n, w.h_kv, w.r_k)) * sk
     zv = rng_for("latent_v", seed, sub).standard_normal((n, w.R)) * sv

@@ -118,7 +118,25 @@ typedef struct starkv_config {
   int32_t flags;        /* 0, or STARKV_FLAG_FP16_LATENT                */
   double top_fraction;  /* 0.25                                         */
   double rope_base;     /* RoPE theta base (1e4 Llama-2, 5e5 Llama-3)   */
+  const int32_t* key_ranks; /* host [num_kv_heads] learned key rank of each
+                               KV head, or NULL for rank_k everywhere (see
+                               "Ragged key ranks" below)                */
 } starkv_config;
+
+/* Ragged key ranks ([Review] section 3 and its figure of learned rank
+ * profiles: the key rank is learned per head and layer; the checkpoint card's
+ * calibration caps it at max_rank_k = 64).  With key_ranks set, KV head h keeps
+ * r_h = key_ranks[h] latent channels: 16 <= r_h <= rank_k, r_h a multiple of
+ * 16, and rank_k is the largest of them.  Each head's channel split and group
+ * size follow from its own r_h (n_top = floor(top_fraction r_h + 0.5),
+ * g = gcd(16, n_top, r_h - n_top)).  A_k holds sum_h r_h columns, head h's at
+ * col0_h = r_0 + ... + r_{h-1}; B_k is [sum_h r_h][head_dim], head h's rows at
+ * col0_h.  A page of the key-code pool holds the heads' regions back to back
+ * (head h at sum_{h' < h} region_bytes(r_h')), and a page of the key-meta pool
+ * their metadata likewise; starkv_cache_sizes.key_page_bytes and
+ * key_page_meta_bytes give the per-page strides.  The joint value rank R is
+ * per layer (one context per layer).  Decode and prefill of ragged ranks run
+ * on the CUDA-core kernels; append on every kernel. */
 
 /* The four caller-allocated page pools of a paged latent cache.
  *   k_codes: [n_pages][num_kv_heads][key_region_bytes]    packed key codes
@@ -154,12 +172,17 @@ typedef struct starkv_cache_sizes {
   int32_t value_top;          /* n_top of the value latent                     */
   int32_t key_groups;         /* r_k / g                                       */
   int32_t value_groups;       /* R / g                                         */
+  int32_t key_page_bytes;     /* key-code bytes of one page, all KV heads      */
+  int32_t key_page_meta_bytes;/* key-meta bytes of one page, all KV heads      */
 } starkv_cache_sizes;
 
 typedef struct starkv_ctx starkv_ctx;
 
 enum { STARKV_OP_DECODE = 0, STARKV_OP_PREFILL = 1, STARKV_OP_DECODE_OUT = 2 };
 enum { STARKV_LATENT_KEY = 0, STARKV_LATENT_VALUE = 1 };
+/* starkv_quantize_pack / starkv_dequantize: the key latent of KV head h
+ * (needed with ragged key ranks; STARKV_LATENT_KEY is head 0). */
+#define STARKV_LATENT_KEY_HEAD(h) (2 + (h))
 
 /* Library version string (static storage). */
 STARKV_API const char* starkv_version(void);

@@ -111,10 +111,34 @@ class Config:
     top_fraction: float = 0.25
     rope_base: float = 10000.0
     fp16_latent: bool = False
+    key_ranks: tuple = None   # ragged ranks: r_k,h per KV head ([Review] section 3), r_k their maximum
 
     @property
     def key(self) -> Latent:
         return latent_fp16(self.r_k) if self.fp16_latent else latent_split(self.r_k, self.top_fraction)
+
+    @property
+    def ragged(self) -> bool:
+        return self.key_ranks is not None
+
+    def key_rank(self, h: int) -> int:
+        return self.r_k if self.key_ranks is None else int(self.key_ranks[h])
+
+    def key_head(self, h: int) -> Latent:
+        """Geometry of KV head h's key latent (its own rank with ragged ranks)."""
+        r = self.key_rank(h)
+        return latent_fp16(r) if self.fp16_latent else latent_split(r, self.top_fraction)
+
+    def key_layout(self):
+        """Per head (latent column, byte offset in a key-code page, word offset in a
+        key-meta page), and the page strides (code bytes, meta words): the heads'
+        regions back to back in head order."""
+        heads, col, code, meta = [], 0, 0, 0
+        for h in range(self.h_kv):
+            L = self.key_head(h)
+            heads.append((col, code, meta))
+            col, code, meta = col + L.r, code + L.region_bytes, meta + L.meta_bytes // 4
+        return heads, code, meta
 
     @property
     def val(self) -> Latent:
@@ -127,9 +151,11 @@ class Config:
 
 def config_of(w) -> Config:
     """Oracle config from a workload description (shape numbers only)."""
+    kr = getattr(w, "key_ranks", None)
     return Config(H=w.H, h_kv=w.h_kv, d_h=w.d_h, hidden=w.hidden, r_k=w.r_k, R=w.R,
                   top_fraction=w.top_fraction, rope_base=w.rope_base,
-                  fp16_latent=bool(getattr(w, "fp16_latent", False)))
+                  fp16_latent=bool(getattr(w, "fp16_latent", False)),
+                  key_ranks=tuple(int(r) for r in kr) if kr is not None else None)
 
 
 # ----------------------------------------------------------------------------
@@ -370,6 +396,11 @@ def new_cache(cfg: Config, n_pages: int) -> Cache:
     k, v = cfg.key, cfg.val
     mk = 0 if k.fp16 else k.n_groups   # fp16 latents carry no metadata
     mv = 0 if v.fp16 else v.n_groups
+    if cfg.ragged:
+        # ragged ranks: one flat key page per page id, the heads' regions back to back
+        _, kb, km = cfg.key_layout()
+        return Cache(cfg, np.zeros((n_pages, kb), np.uint8), np.zeros((n_pages, v.region_bytes), np.uint8),
+                     np.zeros((n_pages, km), np.uint32), np.zeros((n_pages, mv, PAGE), np.uint32))
     return Cache(cfg,
                  np.zeros((n_pages, cfg.h_kv, k.region_bytes), np.uint8),
                  np.zeros((n_pages, v.region_bytes), np.uint8),
@@ -390,6 +421,22 @@ def write_latents(cache: Cache, slots, z_k, z_v) -> None:
     pages, offs = slots // PAGE, slots % PAGE
     upages, inv = np.unique(pages, return_inverse=True)
     rows = inv * PAGE + offs
+    if cfg.ragged:
+        # per head: its own rank (the first r_k,h channels of z_k[:, h]) and geometry
+        for h, (_, co, mo) in enumerate(cfg.key_layout()[0]):
+            L = cfg.key_head(h)
+            codes, s_, zp = quantize_latent(np.asarray(z_k)[:, h, :L.r], L)
+            cb = cache.k_codes[upages, co:co + L.region_bytes]
+            mb = cache.k_meta[upages, mo:mo + L.meta_bytes // 4].reshape(len(upages), -1, PAGE)
+            cc, ss, zz = unpack_region(cb, mb, L)
+            cc[rows] = codes
+            if not L.fp16:
+                ss[rows], zz[rows] = s_, zp
+            nb, nm = pack_region(cc, ss, zz, L)
+            cache.k_codes[upages, co:co + L.region_bytes] = nb
+            cache.k_meta[upages, mo:mo + L.meta_bytes // 4] = nm.reshape(len(upages), -1)
+        _write_values(cache, upages, rows, z_v)
+        return
     if cfg.fp16_latent:
         for h in range(cfg.h_kv):
             v, _, _ = quantize_latent(np.asarray(z_k)[:, h], cfg.key)
@@ -412,13 +459,58 @@ def write_latents(cache: Cache, slots, z_k, z_v) -> None:
     cache.v_codes[upages], cache.v_meta[upages] = pack_region(cc, ss, zz, cfg.val)
 
 
+def _write_values(cache: Cache, upages, rows, z_v) -> None:
+    cfg = cache.cfg
+    codes, s, zp = quantize_latent(z_v, cfg.val)
+    cc, ss, zz = unpack_region(cache.v_codes[upages], None if cfg.val.fp16 else cache.v_meta[upages], cfg.val)
+    cc[rows] = codes
+    if not cfg.val.fp16:
+        ss[rows], zz[rows] = s, zp
+    nb, nm = pack_region(cc, ss, zz, cfg.val)
+    cache.v_codes[upages] = nb
+    if not cfg.val.fp16:
+        cache.v_meta[upages] = nm
+
+
+def pad_key_latents(cfg: Config, z) -> np.ndarray:
+    """Key latents of the library's ragged layout, [n, sum_h r_k,h] (head h's
+    columns at its offset), as [n, h_kv, r_k] with zeros past each head's rank."""
+    z = np.asarray(z)
+    out = np.zeros((z.shape[0], cfg.h_kv, cfg.r_k), z.dtype)
+    for h, (col, _, _) in enumerate(cfg.key_layout()[0]):
+        out[:, h, :cfg.key_rank(h)] = z[:, col:col + cfg.key_rank(h)]
+    return out
+
+
+def pad_key_factor(cfg: Config, B_k) -> np.ndarray:
+    """B_k of the ragged layout, [sum_h r_k,h, d_h], as [h_kv, r_k, d_h] with zero
+    rows past each head's rank (the padded channels then contribute nothing)."""
+    B_k = np.asarray(B_k)
+    out = np.zeros((cfg.h_kv, cfg.r_k, cfg.d_h), B_k.dtype)
+    for h, (col, _, _) in enumerate(cfg.key_layout()[0]):
+        out[h, :cfg.key_rank(h)] = B_k[col:col + cfg.key_rank(h)]
+    return out
+
+
+def unrotate_keys(cfg: Config, zk) -> np.ndarray:
+    """Undo the key rotation of [n, h_kv, r_k] latents, each head with its own group size."""
+    if not cfg.ragged:
+        return unrotate_fp64(zk, cfg.key.g)
+    out = np.zeros(np.shape(zk))
+    for h in range(cfg.h_kv):
+        L = cfg.key_head(h)
+        out[:, h, :L.r] = unrotate_fp64(np.asarray(zk)[:, h, :L.r], L.g)
+    return out
+
+
 def append(cache: Cache, X, A_k, A_v, slots):
     """Decode dataflow steps 1-3: Z_k = X A_k, Z_v = X A_v, rotate, quantise, store.
 
     Returns the pre-quantisation latents (z_k [n, h_kv, r_k], z_v [n, R]) as fp32.
     """
     cfg = cache.cfg
-    z_k = project(X, A_k).reshape(-1, cfg.h_kv, cfg.r_k)
+    z_k = project(X, A_k)
+    z_k = pad_key_latents(cfg, z_k) if cfg.ragged else z_k.reshape(-1, cfg.h_kv, cfg.r_k)
     z_v = project(X, A_v)
     write_latents(cache, slots, z_k, z_v)
     return z_k, z_v
@@ -432,6 +524,14 @@ def gather_sequence(cache: Cache, block_table_row, n: int):
     cfg = cache.cfg
     P = (n + PAGE - 1) // PAGE
     pages = np.asarray(block_table_row[:P], np.int64)
+    if cfg.ragged:
+        zk = np.zeros((n, cfg.h_kv, cfg.r_k), np.float32)
+        for h, (_, co, mo) in enumerate(cfg.key_layout()[0]):
+            L = cfg.key_head(h)
+            mb = cache.k_meta[pages, mo:mo + L.meta_bytes // 4].reshape(P, -1, PAGE)
+            zk[:, h, :L.r] = dequantize_region(cache.k_codes[pages, co:co + L.region_bytes], mb, L, n)
+        zv = dequantize_region(cache.v_codes[pages], cache.v_meta[pages], cfg.val, n)
+        return zk, zv
     zk = np.stack([dequantize_region(cache.k_codes[pages, h], cache.k_meta[pages, h], cfg.key, n)
                    for h in range(cfg.h_kv)], axis=1)
     zv = dequantize_region(cache.v_codes[pages], cache.v_meta[pages], cfg.val, n)
@@ -512,7 +612,7 @@ def decode(cache: Cache, q, B_k, B_v, block_table, seq_lens, seqs=None, heads=No
             out[b, heads] = 0.0
             continue
         zk, zv = gather_sequence(cache, block_table[b], n)
-        zk = unrotate_fp64(zk, cfg.key.g)
+        zk = unrotate_keys(cfg, zk)
         zv = unrotate_fp64(zv, cfg.val.g)
         out[b, heads] = attend_latents(cfg, zk, zv, q[b:b + 1], [n - 1], B_k, B_v, heads)[0]
     return out
@@ -557,7 +657,7 @@ def decode_slice(cache: Cache, q, B_k, B_v, block_table, seq_lens, key_pos0, q_p
             o[b, heads], m[b, heads], l[b, heads] = 0.0, -np.inf, 0.0
             continue
         zk, zv = gather_sequence(cache, block_table[b], n)
-        zk = unrotate_fp64(zk, cfg.key.g)
+        zk = unrotate_keys(cfg, zk)
         zv = unrotate_fp64(zv, cfg.val.g)
         pos = int(key_pos0[b]) + np.arange(n)
         for h in heads:
@@ -608,7 +708,7 @@ def prefill(cache: Cache, q, cu_q, B_k, B_v, block_table, seq_lens, select=None,
             continue
         n = int(seq_lens[b])
         zk, zv = gather_sequence(cache, block_table[b], n)
-        zk = unrotate_fp64(zk, cfg.key.g)
+        zk = unrotate_keys(cfg, zk)
         zv = unrotate_fp64(zv, cfg.val.g)
         rows = int(cu_q[b]) + idx
         out[np.ix_(rows, heads)] = attend_latents(cfg, zk, zv, q[rows], n - nb + idx, B_k, B_v, heads)
@@ -668,9 +768,10 @@ def eq16_retained_fraction(L=32, exempt=3, compressed_fraction=0.25 * 3.2 / 16) 
 def layout_sizes(cfg: Config, n_pages: int) -> dict:
     """Bytes of the four cache pools for n_pages pages (the packed layout above)."""
     k, v = cfg.key, cfg.val
-    return dict(k_codes=n_pages * cfg.h_kv * k.region_bytes,
+    _, kb, km = cfg.key_layout()
+    return dict(k_codes=n_pages * kb,
                 v_codes=n_pages * v.region_bytes,
-                k_meta=n_pages * cfg.h_kv * k.meta_bytes,
+                k_meta=n_pages * km * 4,
                 v_meta=n_pages * v.meta_bytes)
 
 
@@ -679,4 +780,4 @@ def cache_bytes_per_token(cfg: Config) -> float:
 
 
 def payload_bytes_per_token(cfg: Config) -> float:
-    return (cfg.h_kv * cfg.key.payload_bytes + cfg.val.payload_bytes) / PAGE
+    return (sum(cfg.key_head(h).payload_bytes for h in range(cfg.h_kv)) + cfg.val.payload_bytes) / PAGE

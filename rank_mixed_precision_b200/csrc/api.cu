@@ -107,12 +107,54 @@ starkv_status check_config(const starkv_config* c, LatentGeom* key, LatentGeom* 
     return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "key latent: group size gcd(16, n_top, n_bot) must be 4, 8 or 16");
   if (!make_geom(c->rank_v, c->top_fraction, fp16, &v))
     return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "value latent: group size gcd(16, n_top, n_bot) must be 4, 8 or 16");
+  if (c->key_ranks) {
+    int widest = 0;
+    for (int h = 0; h < c->num_kv_heads; ++h) {
+      const int r = c->key_ranks[h];
+      LatentGeom kh;
+      if (r < 16 || r > c->rank_k || r % 16 != 0)
+        return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "key_ranks[%d] = %d: need a multiple of 16 in [16, rank_k = %d]", h,
+                    r, c->rank_k);
+      if (!make_geom(r, c->top_fraction, fp16, &kh))
+        return fail(STARKV_ERR_UNSUPPORTED_SHAPE, "key_ranks[%d] = %d: group size must be 4, 8 or 16", h, r);
+      widest = r > widest ? r : widest;
+    }
+    if (widest != c->rank_k)
+      return fail(STARKV_ERR_INVALID_ARG, "rank_k (%d) must equal the largest of key_ranks (%d)", c->rank_k, widest);
+  }
   if (key) *key = k;
   if (val) *val = v;
   return STARKV_OK;
 }
 
+// Per-head key geometry and page offsets (uniform ranks: every head is `uniform`).
+// heads: host [h_kv]; returns the page strides (code bytes, meta words) and the key columns.
+void build_key_heads(const starkv_config* c, const LatentGeom& uniform, KeyHead* heads, int* page_bytes,
+                     int* page_meta, int* cols) {
+  const bool fp16 = c->flags == STARKV_FLAG_FP16_LATENT;
+  int col = 0, code = 0, meta = 0;
+  for (int h = 0; h < c->num_kv_heads; ++h) {
+    LatentGeom L = uniform;
+    if (c->key_ranks) make_geom(c->key_ranks[h], c->top_fraction, fp16, &L);
+    if (heads) heads[h] = KeyHead{L, col, code, meta};
+    col += L.r;
+    code += L.region_bytes;
+    meta += L.fp16 ? 0 : L.groups * kPage;
+  }
+  *page_bytes = code;
+  *page_meta = meta;
+  *cols = col;
+}
+
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+// Geometry of a latent kind of the quantise / dequantise entries.
+const LatentGeom* latent_of(const Ctx* c, int which) {
+  if (which == STARKV_LATENT_VALUE) return &c->val;
+  if (which == STARKV_LATENT_KEY) return &c->khead_host[0].L;
+  if (which >= 2 && which - 2 < c->cfg.num_kv_heads) return &c->khead_host[which - 2].L;
+  return nullptr;
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -195,9 +237,13 @@ starkv_status starkv_cache_layout(const starkv_config* cfg, int64_t n_pages, sta
   out->value_top = v.n_top;
   out->key_groups = k.groups;
   out->value_groups = v.groups;
-  out->k_codes_bytes = n_pages * cfg->num_kv_heads * (int64_t)k.region_bytes;
+  int kpage = 0, kmeta = 0, kcols = 0;
+  build_key_heads(cfg, k, nullptr, &kpage, &kmeta, &kcols);
+  out->key_page_bytes = kpage;
+  out->key_page_meta_bytes = kmeta * 4;
+  out->k_codes_bytes = n_pages * (int64_t)kpage;
   out->v_codes_bytes = n_pages * (int64_t)v.region_bytes;
-  out->k_meta_bytes = k.fp16 ? 0 : n_pages * cfg->num_kv_heads * (int64_t)k.groups * kPage * 4;
+  out->k_meta_bytes = n_pages * (int64_t)kmeta * 4;
   out->v_meta_bytes = v.fp16 ? 0 : n_pages * (int64_t)v.groups * kPage * 4;
   return ok();
 }
@@ -217,11 +263,28 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
   c->key = k;
   c->val = v;
   c->group = cfg->num_q_heads / cfg->num_kv_heads;
-  c->lat_cols = cfg->num_kv_heads * cfg->rank_k + cfg->rank_v;
+  c->khead_host = new (std::nothrow) KeyHead[cfg->num_kv_heads];
+  c->key_ranks = cfg->key_ranks ? new (std::nothrow) int32_t[cfg->num_kv_heads] : nullptr;
+  if (!c->khead_host || (cfg->key_ranks && !c->key_ranks)) {
+    delete[] c->khead_host;
+    delete[] c->key_ranks;
+    delete c;
+    return fail(STARKV_ERR_CUDA, "out of host memory");
+  }
+  build_key_heads(cfg, k, c->khead_host, &c->kpage_bytes, &c->kpage_meta, &c->key_cols);
+  c->ragged = false;
+  if (cfg->key_ranks) {
+    for (int h = 0; h < cfg->num_kv_heads; ++h) {
+      c->key_ranks[h] = cfg->key_ranks[h];
+      c->ragged = c->ragged || cfg->key_ranks[h] != cfg->rank_k;
+    }
+    c->cfg.key_ranks = c->key_ranks;  // the context's own copy
+  }
+  c->lat_cols = c->key_cols + cfg->rank_v;
   cudaGetDevice(&c->device);
   const int d = cfg->head_dim, half = d / 2;
   const size_t a_bytes = (size_t)cfg->hidden * c->lat_cols * 2;
-  const size_t bk_bytes = (size_t)cfg->num_kv_heads * cfg->rank_k * d * 4;
+  const size_t bk_bytes = (size_t)c->key_cols * d * 4;
   const size_t bv_bytes = (size_t)cfg->rank_v * cfg->num_kv_heads * d * 4;
   const size_t rope_bytes = (size_t)cfg->max_position * half * sizeof(float2);
   const size_t trig_bytes = (size_t)cfg->max_position * d * sizeof(__half);
@@ -238,6 +301,9 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
     cudaFree(c->Bk16);
     cudaFree(c->Bv16p);
     cudaFree(c->Wo);
+    cudaFree(c->khead);
+    delete[] c->khead_host;
+    delete[] c->key_ranks;
     delete c;
   };
   // small appends: K splits of the projection so that about every SM streams a
@@ -262,12 +328,18 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
       (e = cudaMalloc(&c->zpart, (size_t)(c->app_splits > 0 ? c->app_splits : 1) * kSmallAppend * c->lat_cols * 4)) !=
           cudaSuccess ||
       (e = cudaMalloc(&c->status, sizeof(unsigned int))) != cudaSuccess ||
-      (e = cudaMalloc(&c->Bk16, bk_bytes / 2)) != cudaSuccess || (e = cudaMalloc(&c->Bv16p, bv_bytes / 2)) != cudaSuccess) {
+      (e = cudaMalloc(&c->Bk16, bk_bytes / 2)) != cudaSuccess || (e = cudaMalloc(&c->Bv16p, bv_bytes / 2)) != cudaSuccess ||
+      (e = cudaMalloc(&c->khead, (size_t)cfg->num_kv_heads * sizeof(KeyHead))) != cudaSuccess) {
     cleanup();
     return cuda_fail(e, "cudaMalloc (context factors)");
   }
   // A = [A_k | A_v], row-major [hidden][lat_cols]
-  const size_t kcols = (size_t)cfg->num_kv_heads * cfg->rank_k;
+  const size_t kcols = (size_t)c->key_cols;
+  e = cudaMemcpyAsync(c->khead, c->khead_host, (size_t)cfg->num_kv_heads * sizeof(KeyHead), cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) {
+    cleanup();
+    return cuda_fail(e, "starkv_create");
+  }
   e = cudaMemcpy2DAsync(c->A, c->lat_cols * 2, A_k, kcols * 2, kcols * 2, cfg->hidden, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess)
     e = cudaMemcpy2DAsync((char*)c->A + kcols * 2, c->lat_cols * 2, A_v, (size_t)cfg->rank_v * 2,
@@ -308,10 +380,10 @@ starkv_status starkv_create(const starkv_config* cfg, const void* A_k, const voi
   }
   const char* path = getenv("STARKV_DECODE_PATH");
   const bool want_simt = path && strcmp(path, "simt") == 0;
-  c->tc = !want_simt && tc_decode_supported(c->cfg) && c->val.g == 16 && make_trig_map(c);
+  c->tc = !want_simt && !c->ragged && tc_decode_supported(c->cfg) && c->val.g == 16 && make_trig_map(c);
   const char* ppath = getenv("STARKV_PREFILL_PATH");
   const bool want_simt_prefill = ppath && strcmp(ppath, "simt") == 0;
-  c->tc_prefill = !want_simt_prefill && tc_prefill_supported(*c) && make_prefill_maps(c);
+  c->tc_prefill = !want_simt_prefill && !c->ragged && tc_prefill_supported(*c) && make_prefill_maps(c);
   if (c->app_splits > 0) {
     const int kl = cfg->hidden / c->app_splits;
     if (!starkv::encode_map_2d(&c->a_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c->A, (uint64_t)c->lat_cols,
@@ -344,6 +416,9 @@ starkv_status starkv_destroy(starkv_ctx* ctx) {
   cudaFree(c->Bk16);
   cudaFree(c->Bv16p);
   cudaFree(c->Wo);
+  cudaFree(c->khead);
+  delete[] c->khead_host;
+  delete[] c->key_ranks;
   delete c;
   return ok();
 }
@@ -586,9 +661,10 @@ starkv_status starkv_quantize_pack(starkv_ctx* ctx, int32_t which, const float* 
                                    void* meta, starkv_stream_t stream) {
   if (!ctx) return fail(STARKV_ERR_INVALID_ARG, "ctx is NULL");
   Ctx* c = reinterpret_cast<Ctx*>(ctx);
-  if (which != STARKV_LATENT_KEY && which != STARKV_LATENT_VALUE) return fail(STARKV_ERR_INVALID_ARG, "bad latent kind");
+  const LatentGeom* Lp = latent_of(c, which);
+  if (!Lp) return fail(STARKV_ERR_INVALID_ARG, "bad latent kind %d", which);
   if (n < 0) return fail(STARKV_ERR_INVALID_ARG, "n < 0");
-  const LatentGeom& L = which == STARKV_LATENT_KEY ? c->key : c->val;
+  const LatentGeom& L = *Lp;
   if (n > 0 && (!z || !codes || (!meta && !L.fp16))) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
   if (!aligned16(codes) || !aligned16(meta)) return fail(STARKV_ERR_INVALID_ARG, "codes/meta must be 16-byte aligned");
   cudaError_t e = launch_quantize_pack(*c, L, z, n, (uint8_t*)codes, (uint32_t*)meta, (cudaStream_t)stream);
@@ -600,9 +676,10 @@ starkv_status starkv_dequantize(starkv_ctx* ctx, int32_t which, const void* code
                                 float* z_out, starkv_stream_t stream) {
   if (!ctx) return fail(STARKV_ERR_INVALID_ARG, "ctx is NULL");
   Ctx* c = reinterpret_cast<Ctx*>(ctx);
-  if (which != STARKV_LATENT_KEY && which != STARKV_LATENT_VALUE) return fail(STARKV_ERR_INVALID_ARG, "bad latent kind");
+  const LatentGeom* Lp = latent_of(c, which);
+  if (!Lp) return fail(STARKV_ERR_INVALID_ARG, "bad latent kind %d", which);
   if (n < 0) return fail(STARKV_ERR_INVALID_ARG, "n < 0");
-  const LatentGeom& L = which == STARKV_LATENT_KEY ? c->key : c->val;
+  const LatentGeom& L = *Lp;
   if (n > 0 && (!z_out || !codes || (!meta && !L.fp16))) return fail(STARKV_ERR_INVALID_ARG, "NULL argument");
   cudaError_t e = launch_dequantize(*c, L, (const uint8_t*)codes, (const uint32_t*)meta, n, z_out, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");

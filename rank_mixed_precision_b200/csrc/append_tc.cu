@@ -37,6 +37,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
 
 struct AppendTcArgs {
   LatentGeom key, val;
+  const KeyHead* kh;       // [h_kv] per-head key geometry and page offsets
+  int key_cols, kpage_bytes, kpage_meta;
   int h_kv, hidden, lat_cols;
   int64_t n, n_pages;
   const int64_t* slots;
@@ -139,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           slot = -1;
         }
       }
-      const int key_cols = a.h_kv * a.key.r;
+      const int key_cols = a.key_cols;
       for (int c0 = 0; c0 < N; c0 += 16) {
         uint32_t v[16];
         tmem_ld16(tmem + lane_off + c0, v);
@@ -155,16 +157,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (slot < 0) continue;
         const int64_t page = slot / kPage;
         const int t = (int)(slot % kPage);
-        // the 16 columns hold whole groups of one latent (h_kv r_k and R are multiples of 16, g divides 16)
+        // the 16 columns hold whole groups of one latent (every head's rank and R are
+        // multiples of 16, g divides 16)
         const bool is_key = col < key_cols;
-        const LatentGeom& L = is_key ? a.key : a.val;
-        const int cin = is_key ? col % a.key.r : col - key_cols;
+        const int kv = is_key ? key_head_of(a.kh, a.h_kv, col) : 0;
+        const LatentGeom L = is_key ? a.kh[kv].L : a.val;
+        const int cin = is_key ? col - a.kh[kv].col0 : col - key_cols;
         for (int j = 0; j < 16; j += L.g) {
           const int gi = (cin + j) / L.g;
           if (is_key) {
-            const int kv = col / a.key.r;
-            rotate_quantize_store_any(x + j, L, gi, a.k_codes + (page * a.h_kv + kv) * L.region_bytes,
-                                        a.k_meta + (page * a.h_kv + kv) * L.groups * kPage, t, a.status);
+            rotate_quantize_store_any(x + j, L, gi, a.k_codes + page * a.kpage_bytes + a.kh[kv].code_off,
+                                      a.k_meta + page * a.kpage_meta + a.kh[kv].meta_off, t, a.status);
           } else {
             rotate_quantize_store_any(x + j, L, gi, a.v_codes + page * L.region_bytes,
                                         a.v_meta + page * L.groups * kPage, t, a.status);
@@ -197,6 +200,10 @@ cudaError_t launch_append_tc(const Ctx& c, const starkv_cache& cache, const __nv
   AppendTcArgs a;
   a.key = c.key;
   a.val = c.val;
+  a.kh = c.khead;
+  a.key_cols = c.key_cols;
+  a.kpage_bytes = c.kpage_bytes;
+  a.kpage_meta = c.kpage_meta;
   a.h_kv = c.cfg.num_kv_heads;
   a.hidden = c.cfg.hidden;
   a.lat_cols = c.lat_cols;

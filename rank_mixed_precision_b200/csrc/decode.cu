@@ -28,6 +28,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 struct DecodeArgs {
   LatentGeom key, val;
+  const KeyHead* kh;    // [h_kv] per-head key geometry and page offsets
+  int kpage_bytes, kpage_meta;
   int H, h_kv, group, d, max_position;
   int max_pages, pages_per_split, splits;
   int64_t n_pages;
@@ -84,6 +86,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeArgs a)
   const int tid = threadIdx.x;
   const int kv = h / a.group;
   const int R = a.val.r;
+  const KeyHead khd = a.kh[kv];  // this KV head's rank r_h <= RK, its B'_k rows and page offsets
+  const LatentGeom& KL = khd.L;
   float* part = a.part + (((int64_t)b * a.H + h) * a.splits + split) * (R + 2);
 
   const int seq_len = a.seq_lens[b];
@@ -104,12 +108,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeArgs a)
       qr[i + half] = (x1 * cs.x + x0 * cs.y) * scale;
     }
     __syncthreads();
-    const float* Bk = a.Bk + (int64_t)kv * RK * a.d;
+    const float* Bk = a.Bk + (int64_t)khd.col0 * a.d;
     for (int e = tid; e < half * RK; e += kDecThreads) {
       const int i = e / RK, c = e % RK;
-      const float ba = Bk[c * a.d + i], bb = Bk[c * a.d + i + half];
-      Wa[e] = qr[i] * ba + qr[i + half] * bb;
-      Wb[e] = qr[i + half] * ba - qr[i] * bb;
+      float wa = 0.f, wb = 0.f;  // channels past this head's rank weigh nothing
+      if (c < KL.r) {
+        const float ba = Bk[c * a.d + i], bb = Bk[c * a.d + i + half];
+        wa = qr[i] * ba + qr[i + half] * bb;
+        wb = qr[i + half] * ba - qr[i] * bb;
+      }
+      Wa[e] = wa;
+      Wb[e] = wb;
     }
   }
   __syncthreads();
@@ -139,14 +148,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeArgs a)
       const int page = pg[tid / kPage];
       if (page >= 0) {
         const int t = j % kPage;
-        const uint8_t* region = a.k_codes + ((int64_t)page * a.h_kv + kv) * a.key.region_bytes;
-        const uint32_t* meta = a.k_meta + ((int64_t)page * a.h_kv + kv) * a.key.groups * kPage;
+        const uint8_t* region = a.k_codes + (int64_t)page * a.kpage_bytes + khd.code_off;
+        const uint32_t* meta = a.k_meta + (int64_t)page * a.kpage_meta + khd.meta_off;
         float z[RK];
 #pragma unroll
-        for (int c = 0; c < RK; ++c) {
-          const int gi = c / a.key.g;
-          z[c] = latent_value(region, meta, a.key, gi, t, c % a.key.g);
-        }
+        for (int c = 0; c < RK; ++c) z[c] = c < KL.r ? latent_value(region, meta, KL, c / KL.g, t, c % KL.g) : 0.f;
         const float2* rr = a.rope + (int64_t)j * half;
         float acc_s = 0.f;
         for (int i = 0; i < half; ++i) {
@@ -279,6 +285,9 @@ cudaError_t launch_decode_simt(const Ctx& c, const starkv_cache& cache, const __
   DecodeArgs a;
   a.key = c.key;
   a.val = c.val;
+  a.kh = c.khead;
+  a.kpage_bytes = c.kpage_bytes;
+  a.kpage_meta = c.kpage_meta;
   a.H = c.cfg.num_q_heads;
   a.h_kv = c.cfg.num_kv_heads;
   a.group = c.group;

@@ -31,9 +31,37 @@ __host__ __device__ inline int tile_offset(const LatentGeom& L, int gi) {
   return gi < L.top_groups ? gi * 8 * L.g : L.top_groups * 8 * L.g + (gi - L.top_groups) * 6 * L.g;
 }
 
+// One KV head's key latent: its geometry (its own rank r_k,h), its columns in
+// the latent row (and rows of B'_k), and where its region sits in a page of the
+// key pools.  Uniform ranks give col0 = h r_k, code_off = h region_bytes.
+struct KeyHead {
+  LatentGeom L;
+  int col0;      // first latent column (and B'_k row) of the head
+  int code_off;  // byte offset of the head's region within a page of the key-code pool
+  int meta_off;  // 4-byte word offset of the head's metadata within a page of the key-meta pool
+};
+
+// Head whose key columns hold latent column col (col < total key columns).
+__host__ __device__ inline int key_head_of(const KeyHead* kh, int h_kv, int col) {
+  int lo = 0, hi = h_kv - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (kh[mid].col0 <= col) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
 struct Ctx {
   starkv_config cfg;
-  LatentGeom key, val;
+  LatentGeom key, val;    // key: the geometry of every head at uniform ranks, of the widest head otherwise
+  KeyHead* khead;         // device [h_kv]
+  KeyHead* khead_host;    // host [h_kv]
+  int32_t* key_ranks;     // host [h_kv] copy of the rank table (cfg.key_ranks points here), or NULL
+  bool ragged;            // per-head key ranks differ
+  int key_cols;           // sum over heads of r_k,h
+  int kpage_bytes;        // key-code bytes of one page (all heads)
+  int kpage_meta;         // key-meta words of one page (all heads)
   int group;              // H / h_kv
   int lat_cols;           // h_kv * r_k + R
   int device;

@@ -21,6 +21,8 @@ constexpr float kLog2eP = 1.4426950408889634f;
 
 struct PrefillArgs {
   LatentGeom key, val;
+  const KeyHead* kh;    // [h_kv] per-head key geometry and page offsets
+  int kpage_bytes, kpage_meta;
   int H, h_kv, group, d, max_position;
   int batch, max_pages, chunk, max_q_len;
   int64_t n_pages, total_q;
@@ -76,23 +78,23 @@ __global__ void __launch_bounds__(256) prefill_simt_expand_kernel(PrefillArgs a,
   }
   __syncthreads();
   const bool valid = ok_len && j < L && pg[tt / 16] >= 0;
-  // ---- keys: dequantise this position's r_k latents, re-expand, RoPE
-  const int rk = a.key.r;
+  // ---- keys: dequantise this position's r_k,h latents, re-expand, RoPE
+  const KeyHead khd = a.kh[kv];
+  const int rk = khd.L.r;
   for (int e = tid; e < 32 * rk; e += 256) {
     const int t2 = e / rk, c = e % rk;
     float z = 0.f;
     const int page = pg[t2 / 16];
     if (ok_len && j0 + t2 < L && page >= 0) {
-      const int t = (j0 + t2) % kPage, gi = c / a.key.g;
-      const uint8_t* region = a.k_codes + ((int64_t)page * a.h_kv + kv) * a.key.region_bytes;
-      z = latent_value(region, a.k_meta + ((int64_t)page * a.h_kv + kv) * a.key.groups * kPage, a.key, gi, t,
-                       c % a.key.g);
+      const int t = (j0 + t2) % kPage, gi = c / khd.L.g;
+      const uint8_t* region = a.k_codes + (int64_t)page * a.kpage_bytes + khd.code_off;
+      z = latent_value(region, a.k_meta + (int64_t)page * a.kpage_meta + khd.meta_off, khd.L, gi, t, c % khd.L.g);
     }
     Zk[t2][c] = z;
   }
   __syncthreads();
   {
-    const float* Bk = a.Bk + (int64_t)kv * rk * a.d;
+    const float* Bk = a.Bk + (int64_t)khd.col0 * a.d;
     const int per = half / 8;
     for (int u = 0; u < per; ++u) {
       const int i = sub * per + u;
@@ -308,6 +310,9 @@ cudaError_t launch_prefill_simt(const Ctx& c, const starkv_cache& cache, const _
   PrefillArgs a;
   a.key = c.key;
   a.val = c.val;
+  a.kh = c.khead;
+  a.kpage_bytes = c.kpage_bytes;
+  a.kpage_meta = c.kpage_meta;
   a.H = c.cfg.num_q_heads;
   a.h_kv = c.cfg.num_kv_heads;
   a.group = c.group;

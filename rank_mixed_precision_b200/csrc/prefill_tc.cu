@@ -794,7 +794,7 @@ __global__ void to_half_prefill_kernel(const float* __restrict__ x, __half* __re
 
 cudaError_t launch_prepare_prefill_factors(const Ctx& c, cudaStream_t s) {
   const starkv_config& f = c.cfg;
-  const int64_t nk = (int64_t)f.num_kv_heads * f.rank_k * f.head_dim;
+  const int64_t nk = (int64_t)c.key_cols * f.head_dim;
   to_half_prefill_kernel<<<(unsigned)((nk + 255) / 256), 256, 0, s>>>(c.Bk, c.Bk16, nk);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

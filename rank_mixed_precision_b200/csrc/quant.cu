@@ -36,10 +36,18 @@ __global__ void fold_rotation_kernel(const __nv_bfloat16* __restrict__ B, float*
 cudaError_t launch_prepare_factors(const Ctx& c, const __nv_bfloat16* Bk, const __nv_bfloat16* Bv,
                                    cudaStream_t s) {
   const starkv_config& f = c.cfg;
-  {
+  if (!c.ragged) {
     const int64_t rows = (int64_t)f.num_kv_heads * f.rank_k;  // groups never cross heads (g | r_k)
     const int64_t total = rows * f.head_dim;
     fold_rotation_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(Bk, c.Bk, rows, f.head_dim, c.key.g);
+  } else {
+    for (int h = 0; h < f.num_kv_heads; ++h) {  // each head with its own rank and group size
+      const KeyHead& kh = c.khead_host[h];
+      const int64_t total = (int64_t)kh.L.r * f.head_dim;
+      const int64_t off = (int64_t)kh.col0 * f.head_dim;
+      fold_rotation_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(Bk + off, c.Bk + off, kh.L.r, f.head_dim,
+                                                                          kh.L.g);
+    }
   }
   {
     const int64_t rows = f.rank_v;
@@ -112,6 +120,8 @@ cudaError_t launch_dequantize(const Ctx&, const LatentGeom& L, const uint8_t* co
 // ---------------------------------------------------------------------------
 struct AppendArgs {
   LatentGeom key, val;
+  const KeyHead* kh;       // [h_kv] per-head key geometry and page offsets
+  int key_cols, kpage_bytes, kpage_meta;
   int h_kv, hidden, lat_cols;
   int64_t n, n_pages;
   const __nv_bfloat16* X;
@@ -173,7 +183,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
     }
   }
   // epilogue: one item per (token, 4-column unit); the unit that starts a group does the group
-  const int key_cols = a.h_kv * a.key.r;
+  const int key_cols = a.key_cols;
   for (int e = tid; e < kAppBM * (kAppBN / 4); e += 256) {
     const int m = e / (kAppBN / 4);
     const int cc = (e % (kAppBN / 4)) * 4;
@@ -181,8 +191,9 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
     const int64_t row = row0 + m;
     if (row >= a.n || col >= a.lat_cols) continue;
     const bool is_key = col < key_cols;
-    const LatentGeom& L = is_key ? a.key : a.val;
-    const int cin = is_key ? col % a.key.r : col - key_cols;
+    const int kv = is_key ? key_head_of(a.kh, a.h_kv, col) : 0;
+    const LatentGeom L = is_key ? a.kh[kv].L : a.val;
+    const int cin = is_key ? col - a.kh[kv].col0 : col - key_cols;
     if (cin % L.g != 0) continue;
     const int64_t slot = a.slots[row];
     if (slot < 0) continue;
@@ -194,9 +205,8 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
     const int t = (int)(slot % kPage);
     const int gi = cin / L.g;
     if (is_key) {
-      const int kv = col / a.key.r;
-      rotate_quantize_store_any(&Zs[m][cc], L, gi, a.k_codes + (page * a.h_kv + kv) * L.region_bytes,
-                                a.k_meta + (page * a.h_kv + kv) * L.groups * kPage, t, a.status);
+      rotate_quantize_store_any(&Zs[m][cc], L, gi, a.k_codes + page * a.kpage_bytes + a.kh[kv].code_off,
+                                a.k_meta + page * a.kpage_meta + a.kh[kv].meta_off, t, a.status);
     } else {
       rotate_quantize_store_any(&Zs[m][cc], L, gi, a.v_codes + page * L.region_bytes,
                                 a.v_meta + page * L.groups * kPage, t, a.status);
@@ -374,10 +384,11 @@ __global__ void __launch_bounds__(128) append_quant_kernel(AppendArgs a, const f
       }
     }
   }
-  const int key_cols = a.h_kv * a.key.r;
+  const int key_cols = a.key_cols;
   const bool is_key = col < key_cols;
-  const LatentGeom& L = is_key ? a.key : a.val;
-  const int cin = is_key ? col % a.key.r : col - key_cols;
+  const int kv = is_key ? key_head_of(a.kh, a.h_kv, col) : 0;
+  const LatentGeom L = is_key ? a.kh[kv].L : a.val;
+  const int cin = is_key ? col - a.kh[kv].col0 : col - key_cols;
   const int lane = threadIdx.x & 31;
   float x[16];
 #pragma unroll
@@ -399,9 +410,8 @@ __global__ void __launch_bounds__(128) append_quant_kernel(AppendArgs a, const f
     const int t = (int)(slot % kPage);
     const int gi = cin / L.g;
     if (is_key) {
-      const int kv = col / a.key.r;
-      rotate_quantize_store_any(x, L, gi, a.k_codes + (page * a.h_kv + kv) * L.region_bytes,
-                                a.k_meta + (page * a.h_kv + kv) * L.groups * kPage, t, a.status);
+      rotate_quantize_store_any(x, L, gi, a.k_codes + page * a.kpage_bytes + a.kh[kv].code_off,
+                                a.k_meta + page * a.kpage_meta + a.kh[kv].meta_off, t, a.status);
     } else {
       rotate_quantize_store_any(x, L, gi, a.v_codes + page * L.region_bytes, a.v_meta + page * L.groups * kPage,
                                 t, a.status);
@@ -415,6 +425,10 @@ cudaError_t launch_append(const Ctx& c, const starkv_cache& cache, const __nv_bf
   AppendArgs a;
   a.key = c.key;
   a.val = c.val;
+  a.kh = c.khead;
+  a.key_cols = c.key_cols;
+  a.kpage_bytes = c.kpage_bytes;
+  a.kpage_meta = c.kpage_meta;
   a.h_kv = c.cfg.num_kv_heads;
   a.hidden = c.cfg.hidden;
   a.lat_cols = c.lat_cols;

@@ -37,7 +37,8 @@ class starkv_config(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("hidden", ctypes.c_int32),
                 ("rank_k", ctypes.c_int32), ("rank_v", ctypes.c_int32),
                 ("max_position", ctypes.c_int32), ("flags", ctypes.c_int32),
-                ("top_fraction", ctypes.c_double), ("rope_base", ctypes.c_double)]
+                ("top_fraction", ctypes.c_double), ("rope_base", ctypes.c_double),
+                ("key_ranks", ctypes.POINTER(ctypes.c_int32))]
 
 
 class starkv_cache(ctypes.Structure):
@@ -52,7 +53,8 @@ class starkv_cache_sizes(ctypes.Structure):
                 ("key_region_bytes", ctypes.c_int32), ("value_region_bytes", ctypes.c_int32),
                 ("key_group_size", ctypes.c_int32), ("value_group_size", ctypes.c_int32),
                 ("key_top", ctypes.c_int32), ("value_top", ctypes.c_int32),
-                ("key_groups", ctypes.c_int32), ("value_groups", ctypes.c_int32)]
+                ("key_groups", ctypes.c_int32), ("value_groups", ctypes.c_int32),
+                ("key_page_bytes", ctypes.c_int32), ("key_page_meta_bytes", ctypes.c_int32)]
 
 
 class StarKVError(RuntimeError):
@@ -138,8 +140,20 @@ def _need(t, dtype, name, ndim=None):
 FLAG_FP16_LATENT = 1
 
 
-def make_config(H, h_kv, d_h, hidden, r_k, R, max_position, top_fraction=0.25, rope_base=10000.0, flags=0):
-    return starkv_config(H, h_kv, d_h, hidden, r_k, R, max_position, flags, top_fraction, rope_base)
+def make_config(H, h_kv, d_h, hidden, r_k, R, max_position, top_fraction=0.25, rope_base=10000.0, flags=0,
+                key_ranks=None):
+    """key_ranks: optional per-KV-head key ranks (ragged ranks; r_k must be their maximum)."""
+    cfg = starkv_config(H, h_kv, d_h, hidden, r_k, R, max_position, flags, top_fraction, rope_base, None)
+    if key_ranks is not None:
+        arr = (ctypes.c_int32 * len(key_ranks))(*[int(r) for r in key_ranks])
+        cfg.key_ranks = ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32))
+        cfg._key_ranks_keepalive = arr
+    return cfg
+
+
+def LATENT_KEY_HEAD(h: int) -> int:
+    """Latent kind of KV head h's key latent for starkv_quantize_pack / starkv_dequantize."""
+    return 2 + h
 
 
 def starkv_version() -> str:
@@ -159,11 +173,17 @@ def starkv_cache_layout(cfg: starkv_config, n_pages: int) -> dict:
 def starkv_create(cfg: starkv_config, A_k, A_v, B_k, B_v, stream=None):
     for t, n in ((A_k, "A_k"), (A_v, "A_v"), (B_k, "B_k"), (B_v, "B_v")):
         _need(t, torch.bfloat16, n)
-    if tuple(A_k.shape) != (cfg.hidden, cfg.num_kv_heads * cfg.rank_k):
+    if cfg.key_ranks:
+        kcols = sum(cfg.key_ranks[h] for h in range(cfg.num_kv_heads))
+        want_bk = (kcols, cfg.head_dim)          # ragged ranks: head h's rows after the earlier heads'
+    else:
+        kcols = cfg.num_kv_heads * cfg.rank_k
+        want_bk = (cfg.num_kv_heads, cfg.rank_k, cfg.head_dim)
+    if tuple(A_k.shape) != (cfg.hidden, kcols):
         raise ValueError(f"A_k shape {tuple(A_k.shape)}")
     if tuple(A_v.shape) != (cfg.hidden, cfg.rank_v):
         raise ValueError(f"A_v shape {tuple(A_v.shape)}")
-    if tuple(B_k.shape) != (cfg.num_kv_heads, cfg.rank_k, cfg.head_dim):
+    if tuple(B_k.shape) != want_bk:
         raise ValueError(f"B_k shape {tuple(B_k.shape)}")
     if tuple(B_v.shape) != (cfg.rank_v, cfg.num_kv_heads * cfg.head_dim):
         raise ValueError(f"B_v shape {tuple(B_v.shape)}")

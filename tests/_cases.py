@@ -33,7 +33,7 @@ def make_ctx(w: gen.Workload, seed=0, max_position=None):
     f = gen.make_factors(w, seed)
     mp = max_position or (w.ctx + max(w.steps, w.chunk) + 16)
     cfg = S.make_config(w.H, w.h_kv, w.d_h, w.hidden, w.r_k, w.R, mp, w.top_fraction, w.rope_base,
-                        S.FLAG_FP16_LATENT if w.fp16_latent else 0)
+                        S.FLAG_FP16_LATENT if w.fp16_latent else 0, w.key_ranks)
     kv = S.StarKV(cfg, bf16_tensor(f.A_k), bf16_tensor(f.A_v), bf16_tensor(f.B_k), bf16_tensor(f.B_v))
     return kv, f
 

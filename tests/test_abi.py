@@ -68,7 +68,7 @@ def test_top_fraction_0_2_rejected_for_supported_key_ranks(S):
 
 @pytest.mark.parametrize("field,value,code", [
     ("head_dim", 96, 2), ("num_kv_heads", 3, 2), ("rank_k", 24, 2), ("rank_v", 0, 1),
-    ("hidden", 100, 2), ("flags", 1, 1), ("rope_base", 1.0, 1), ("top_fraction", 1.5, 1),
+    ("hidden", 100, 2), ("flags", 2, 1), ("rope_base", 1.0, 1), ("top_fraction", 1.5, 1),
     ("max_position", 0, 1), ("max_position", (1 << 24) + 1, 2),
     ("num_kv_heads", 1 << 30, 2), ("num_q_heads", 2048, 2), ("hidden", 1 << 17, 2),
 ])

@@ -330,3 +330,30 @@ def test_fp16_variant_attention_close_to_unquantised(wi):
     O.write_latents(c43, gen.slots_for(bt, 0, np.arange(200)), zk, zv)
     rel43 = np.linalg.norm(O.decode(c43, q, f.B_k, f.B_v, bt, [200]) - ref) / np.linalg.norm(ref)
     assert rel43 > 4 * rel
+
+
+def test_ragged_ranks_decode_against_materialised():
+    # ragged key ranks ([Review] section 3: learned per head): each head's keys
+    # are its own r_h latents times its own B_k rows; brute force on the
+    # dequantised latents (per-head rotation undone) with torch SDPA
+    ranks = (64, 48, 32, 16, 64, 32, 48, 16)
+    w = gen.shrink(gen.workload(3), key_ranks=ranks, ctx=90)
+    cfg = O.config_of(w)
+    f = gen.make_factors(w)
+    Bk = O.pad_key_factor(cfg, f.B_k)
+    zk, zv = gen.make_latents(w, 90)
+    bt, n_pages = gen.make_block_table([90])
+    cache = O.new_cache(cfg, n_pages)
+    O.write_latents(cache, gen.slots_for(bt, 0, np.arange(90)), zk, zv)
+    q = gen.make_queries(1, w.H, w.d_h)
+    got = O.decode(cache, q, Bk, f.B_v, bt, [90])
+    zkh, zvh = O.gather_sequence(cache, bt[0], 90)
+    Kh = np.zeros((90, cfg.h_kv, cfg.r_k))
+    for h, r in enumerate(ranks):      # per-head unrotation with the head's own group size
+        g = O.latent_split(r).g
+        Kh[:, h, :r] = (zkh[:, h, :r].astype(np.float64).reshape(90, r // g, g) @ O.hadamard_fp64(g)).reshape(90, r)
+    ref = _sdpa_materialised(cfg, Kh, O.unrotate_fp64(zvh, cfg.val.g), Bk, f.B_v, q, [89])
+    np.testing.assert_allclose(got, ref, atol=1e-12, rtol=0)
+    # padded channels carry nothing: the padded B_k rows are zero
+    for h, r in enumerate(ranks):
+        assert np.all(Bk[h, r:] == 0)

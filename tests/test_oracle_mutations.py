@@ -164,8 +164,12 @@ def pack_k(hi_first=False, planes_swapped=False, meta_swapped=False, fp16_channe
 
 
 def write_k(drop_offsets=False):
+    real = OM.write_latents
+
     def write_latents(cache, slots, z_k, z_v):
         cfg = cache.cfg
+        if cfg.ragged:
+            return real(cache, slots, z_k, z_v)
         slots = np.asarray(slots, np.int64)
         if slots.size == 0:
             return
@@ -308,6 +312,53 @@ def decode_out_k(kv_rows=False):
     return decode_out
 
 
+def write_ragged_k(reverse_heads=False):
+    real = OM.write_latents
+
+    def write_latents(cache, slots, z_k, z_v):
+        cfg = cache.cfg
+        if not cfg.ragged:
+            return real(cache, slots, z_k, z_v)
+        slots = np.asarray(slots, np.int64)
+        pages, offs = slots // OM.PAGE, slots % OM.PAGE
+        upages, inv = np.unique(pages, return_inverse=True)
+        rows = inv * OM.PAGE + offs
+        rev = {}
+        if reverse_heads:   # the heads' regions placed in reverse head order
+            co_, mo_ = 0, 0
+            for h in reversed(range(cfg.h_kv)):
+                L = cfg.key_head(h)
+                rev[h] = (co_, mo_)
+                co_, mo_ = co_ + L.region_bytes, mo_ + L.meta_bytes // 4
+        for h, (_, co, mo) in enumerate(cfg.key_layout()[0]):
+            L = cfg.key_head(h)
+            if reverse_heads:
+                co, mo = rev[h]
+            codes, s_, zp = OM.quantize_latent(np.asarray(z_k)[:, h, :L.r], L)
+            cb = cache.k_codes[upages, co:co + L.region_bytes]
+            mb = cache.k_meta[upages, mo:mo + L.meta_bytes // 4].reshape(len(upages), -1, OM.PAGE)
+            cc, ss, zz = OM.unpack_region(cb, mb, L)
+            cc[rows], ss[rows], zz[rows] = codes, s_, zp
+            nb, nm = OM.pack_region(cc, ss, zz, L)
+            cache.k_codes[upages, co:co + L.region_bytes] = nb[:, :cb.shape[1]]
+            cache.k_meta[upages, mo:mo + L.meta_bytes // 4] = nm.reshape(len(upages), -1)[:, :mb.shape[1] * OM.PAGE]
+        OM._write_values(cache, upages, rows, z_v)
+    return write_latents
+
+
+def unrotate_keys_k(widest_group=False):
+    def unrotate_keys(cfg, zk):
+        if not cfg.ragged:
+            return OM.unrotate_fp64(zk, cfg.key.g)
+        out = np.zeros(np.shape(zk))
+        for h in range(cfg.h_kv):
+            L = cfg.key_head(h)
+            g = cfg.key.g if widest_group else L.g
+            out[:, h, :L.r] = OM.unrotate_fp64(np.asarray(zk)[:, h, :L.r], g)
+        return out
+    return unrotate_keys
+
+
 def prefill_k(shift=0):
     def prefill(cache, q, cu_q, B_k, B_v, block_table, seq_lens, select=None, heads=None):
         cfg = cache.cfg
@@ -368,7 +419,9 @@ PINS = {
     "pack_region": [lambda: TQ.test_pack_matches_hand_derived_bytes(),
                     lambda: TQ.test_pack_unpack_exhaustive(32, 0.25),
                     lambda: TQ.test_fp16_variant_page_bytes_by_hand()],
-    "write_latents": [lambda: TQ.test_write_latents_partial_pages_keep_other_rows()],
+    "write_latents": [lambda: TQ.test_write_latents_partial_pages_keep_other_rows(),
+                      lambda: TB.test_ragged_pages_hold_each_heads_own_codes()],
+    "unrotate_keys": [lambda: TA.test_ragged_ranks_decode_against_materialised()],
     "gather_sequence": [lambda: TA.test_decode_through_paged_cache_equals_direct()],
     "attend_latents": [lambda: TA.test_reassociated_equals_materialised(8, 2),
                        lambda: TA.test_decode_through_paged_cache_equals_direct()],
@@ -388,7 +441,7 @@ FAITHFUL = {
     "rope": rope_k(), "hadamard_fp64": hadamard_k(), "rotate_fl32": rotate_k(),
     "unrotate_fp64": unrotate_k(), "quantize_groups": quantize_k(), "dequantize_codes": dequantize_k(),
     "quantize_latent": quantize_latent_k(),
-    "pack_region": pack_k(), "write_latents": write_k(), "gather_sequence": gather_k(),
+    "pack_region": pack_k(), "write_latents": write_ragged_k(), "unrotate_keys": unrotate_keys_k(), "gather_sequence": gather_k(),
     "attend_latents": attend_k(), "partial_softmax": partial_k(), "lse_merge": merge_k(),
     "eq14_mean_bits": eq14_k(), "eq16_retained_fraction": eq16_k(), "project": project_k(), "prefill": prefill_k(),
     "decode_slice": decode_slice_k(), "merge_slices": merge_slices_k(), "decode_out": decode_out_k(),
@@ -419,6 +472,8 @@ PLANTS = {
     "3-bit tile: 1-bit plane before 2-bit plane": ("pack_region", pack_k(planes_swapped=True)),
     "metadata: zero in the low half": ("pack_region", pack_k(meta_swapped=True)),
     "append drops the in-page offset": ("write_latents", write_k(drop_offsets=True)),
+    "ragged heads stored in reverse order": ("write_latents", write_ragged_k(reverse_heads=True)),
+    "ragged heads unrotated with the widest group": ("unrotate_keys", unrotate_keys_k(widest_group=True)),
     "gather ignores the block table": ("gather_sequence", gather_k(ignore_table=True)),
     "scores scaled by 1/d, not 1/sqrt(d)": ("attend_latents", attend_k(scale_pow=1.0)),
     "GQA head maps to h mod h_kv": ("attend_latents", attend_k(kv_of="mod")),

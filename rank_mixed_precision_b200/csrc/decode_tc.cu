@@ -106,7 +106,7 @@ struct ScoreArgs {
   int ocnt_elems;
   const uint8_t* wimg; // [B][HG][ncols * d * 2] W in its shared-memory image
   unsigned int* status;
-  uint32_t off_trig, off_codes, off_meta, off_flags, off_bt, off_bar;
+  uint32_t off_trig, off_codes, off_meta, off_flags, off_bt, off_bar, off_red;
   uint32_t trig_stage, codes_page, meta_page, codes_stage, meta_stage, w_bytes;
   int NK;  // key-stage ring depth (the position tiles use two stages)
   uint32_t codes_pitch, meta_pitch;  // shared-memory page strides (padded against bank conflicts)
@@ -400,6 +400,8 @@ __global__ void __launch_bounds__(kAThreads, 1)
 
   // (before the wait: every kernel earlier than the query fold has completed)
   // zero the projection's sums and arrival counters (grid-stride over all CTAs)
+  // partial-score reduction buffer of the shared-KV-head epilogue: [2 tiles][4 heads][128 tokens]
+  for (int i = tid; i < 2 * 4 * kT; i += blockDim.x) reinterpret_cast<float*>(sm + a.off_red)[i] = 0.f;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + tid; i < a.oacc_elems; i += (int64_t)gridDim.x * blockDim.x)
     a.oacc[i] = 0.f;
   for (int i = blockIdx.x * blockDim.x + tid; i < a.ocnt_elems; i += gridDim.x * blockDim.x) a.ocnt[i] = 0u;
@@ -554,6 +556,112 @@ __global__ void __launch_bounds__(kAThreads, 1)
           mma_commit(&trempty[s]);
         }
       }
+    } else if (RK == 64 && G == 16 && a.kvpc == 1 && a.hpc == 4) {
+      // ---------------- epilogue, four query heads over one KV head (GQA) ----------------
+      // Warp (q4, gq): tokens 32 q4 .. + 31 (its TMEM lane quarter) and channel
+      // group gq (16 channels) of the shared key latent, for all four heads: the
+      // codes are unpacked and dequantised once, z^ = code s + zp, and each head
+      // takes 16 products from its G row.  The four groups' partial scores meet
+      // in shared memory; after a barrier of the 16 epilogue warps each thread
+      // finalises one (head, token).
+      const int q4 = warp & 3, gq = (warp - 2) >> 2;
+      const int t = q4 * 32 + lane;
+      const int t16 = t % kPage, p = t / kPage;
+      const int e = (warp - 2) * 32 + lane;
+      const int fh = e >> 7, ft = e & 127;  // this thread's (head, token) to finalise
+      float* red = reinterpret_cast<float*>(sm + a.off_red);
+      float mfin = -INFINITY;
+      for (int k = 0; k < ntile; ++k) {
+        const uint32_t c = it + k, s = c & 1, ph = (c >> 1) & 1;
+        const uint32_t ks = c % a.NK, kph = (c / a.NK) & 1;
+        const bool got = __all_sync(0xffffffffu, mbar_wait(&tfull[s], ph) && mbar_wait(&kfull[ks], kph));
+        if (!got && lane == 0) {
+          set_status(a.status, kDevWaitTimeout);
+          *failed = 1;
+        }
+        tc_fence_after();
+        const int tile = t0 + k;
+        const int j = tile * kT + t;
+        const int jf = tile * kT + ft;
+        const bool fvalid = jf < L && flags[ks * kPagesPerTile + ft / kPage] >= 0;
+        float* rb = red + (c & 1) * (4 * kT);
+        if (got) {
+          const uint32_t trow = tmem + s * 256 + ((uint32_t)(q4 * 32) << 16) + gq * 16;
+          const int pid = flags[ks * kPagesPerTile + p];
+          float zh[16];
+          if (j < L && pid >= 0) {
+            const uint8_t* region = sm + a.off_codes + ks * a.codes_stage + p * a.codes_pitch;
+            const uint32_t mw =
+                reinterpret_cast<const uint32_t*>(sm + a.off_meta + ks * a.meta_stage + p * a.meta_pitch)[gq * kPage + t16];
+            const float sc = __half2float(__ushort_as_half((unsigned short)(mw & 0xFFFF)));
+            const float zp = __half2float(__ushort_as_half((unsigned short)(mw >> 16)));
+            // x = 1 + code / 16 from the code bits under the mantissa of 1.0:
+            // z^ = code s + zp = x (16 s) + (zp - 16 s)
+            const float s16 = 16.f * sc, z0 = zp - s16;
+            uint32_t w[2];
+            if (gq < a.key.top_groups) {
+              const uint2 u = *reinterpret_cast<const uint2*>(region + gq * 128 + 8 * t16);
+              w[0] = u.x;
+              w[1] = u.y;
+            } else {
+              const uint8_t* tl = region + a.key.top_groups * 128 + (gq - a.key.top_groups) * 96;
+              const uint32_t lo = *reinterpret_cast<const uint32_t*>(tl + 4 * t16);
+              const uint32_t hi = *reinterpret_cast<const uint16_t*>(tl + 64 + 2 * t16);
+              w[0] = spread2_to_nibbles8(lo & 0xFFFFu) | (spread1_to_nibbles8(hi & 0xFFu) << 2);
+              w[1] = spread2_to_nibbles8(lo >> 16) | (spread1_to_nibbles8(hi >> 8) << 2);
+            }
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+#pragma unroll
+              for (int cc = 0; cc < 8; ++cc) {
+                const uint32_t bits = (cc >= 5 ? (w[q] >> (4 * cc - 19)) : (w[q] << (19 - 4 * cc))) & 0x00780000u;
+                zh[q * 8 + cc] = fmaf(mant(bits), s16, z0);
+              }
+          } else {
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) zh[cc] = 0.f;
+          }
+#pragma unroll
+          for (int hp = 0; hp < 4; hp += 2) {
+            uint32_t g0[16], g1[16];
+            tmem_issue_row<16>(trow + hp * 64, g0);
+            tmem_issue_row<16>(trow + (hp + 1) * 64, g1);
+            tmem_wait_row<16>(g0);
+            tmem_wait_row<16>(g1);
+            float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < 16; cc += 2) {
+              a0 = fmaf(zh[cc], __uint_as_float(g0[cc]), a0);
+              a1 = fmaf(zh[cc + 1], __uint_as_float(g0[cc + 1]), a1);
+              b0 = fmaf(zh[cc], __uint_as_float(g1[cc]), b0);
+              b1 = fmaf(zh[cc + 1], __uint_as_float(g1[cc + 1]), b1);
+            }
+            atomicAdd(rb + hp * kT + t, a0 + a1);
+            atomicAdd(rb + (hp + 1) * kT + t, b0 + b1);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&tempty[s]);
+          mbar_arrive(&kempty[ks]);
+        }
+        // every group's partial is in; the failure flag is decided once for all 16 warps
+        uint32_t stop;
+        asm volatile(
+            "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, 512, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+            : "=r"(stop)
+            : "r"((uint32_t)(!got || *failed))
+            : "memory");
+        if (stop) break;
+        const float score = fvalid ? rb[fh * kT + ft] : -INFINITY;
+        rb[fh * kT + ft] = 0.f;  // ready for the tile two ahead (a barrier of the next tile comes between)
+        if (jf < L) a.S[((int64_t)b * a.H + h0 + fh) * a.tpad + jf] = score;
+        mfin = fmaxf(mfin, score);
+      }
+      // this job's running maximum of head fh (one head per warp): one atomic per warp
+      const float m = warp_max(mfin);
+      if (lane == 0 && m != -INFINITY) atomicMax(&a.Mx[b * a.H + h0 + fh], ordered_bits(m));
     } else {
       // ---------------- epilogue: one thread per token ----------------
       const int q4 = warp & 3, hq = (warp - 2) >> 2;   // TMEM lane quarter, head quarter
@@ -1684,7 +1792,7 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
     o += 2 * A.trig_stage;
     // as many key stages as fit (page table, flags, barriers and alignment slack after them)
     const uint32_t tail = (uint32_t)(A.items_per_cta * kPagesPerTile * 4) + kMaxKeyStages * kPagesPerTile * 4 +
-                          (2 * kMaxKeyStages + 16) * 8 + 1024 + 64;
+                          (2 * kMaxKeyStages + 16) * 8 + 2 * 4 * kT * 4 + 1024 + 64;
     const uint32_t per_key = A.codes_stage + A.meta_stage;
     int nk = (int)((227u * 1024u - o - tail) / per_key);
     if (nk > kMaxKeyStages) nk = kMaxKeyStages;
@@ -1700,6 +1808,8 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
     o = A.off_bt + A.items_per_cta * kPagesPerTile * 4;
     A.off_bar = (o + 15) / 16 * 16;
     o = A.off_bar + (2 * kMaxKeyStages + 16) * 8;
+    A.off_red = (o + 15) / 16 * 16;
+    o = A.off_red + 2 * 4 * kT * 4;
     const size_t smem = o + 1024;  // alignment slack
     cudaError_t e;
     switch (f.rank_k) {

@@ -87,7 +87,7 @@ struct ScoreArgs {
   LatentGeom key;
   int H, h_kv, group, d, hpc, kvpc, ncols, HG;
   int max_pages, tiles_per_seq, tpad, max_position;
-  int items_per_cta, total_items;
+  int items_per_cta, batch;  // tiles per CTA at most (its page-table space); sequences
   int64_t n_pages;
   const __nv_bfloat16* q;
   const int32_t* block_table;
@@ -106,7 +106,7 @@ struct ScoreArgs {
   int ocnt_elems;
   const uint8_t* wimg; // [B][HG][ncols * d * 2] W in its shared-memory image
   unsigned int* status;
-  uint32_t off_trig, off_codes, off_meta, off_flags, off_bt, off_bar, off_red;
+  uint32_t off_trig, off_codes, off_meta, off_flags, off_bt, off_bar, off_red, off_pre;
   uint32_t trig_stage, codes_page, meta_page, codes_stage, meta_stage, w_bytes;
   int NK;  // key-stage ring depth (the position tiles use two stages)
   uint32_t codes_pitch, meta_pitch;  // shared-memory page strides (padded against bank conflicts)
@@ -432,22 +432,50 @@ __global__ void __launch_bounds__(kAThreads, 1)
   uint32_t jobs = 0;
 
   uint32_t it = 0;  // tiles through the pipeline so far (same count in every role)
-  int item = blockIdx.x * a.items_per_cta;
-  const int item_end = min(item + a.items_per_cta, a.total_items);
+  // The work items are the sequences' 128-token tiles that hold tokens, per head
+  // group: pre[b] = items of the sequences before b (HG x tiles each).  Every CTA
+  // takes an equal share of them, so sequences of unequal length balance.
+  int* pre = reinterpret_cast<int*>(sm + a.off_pre);  // [batch + 1]
+  if (warp == 0) {
+    int run = 0;
+    for (int b0 = 0; b0 < a.batch; b0 += 32) {
+      const int b = b0 + lane;
+      int v = 0;
+      if (b < a.batch) {
+        const int Lb = decode_len(a.seq_lens, a.pos0, a.qpos, b, a.max_pages, a.max_position);
+        v = Lb > 0 ? (Lb + kT - 1) / kT * a.HG : 0;
+      }
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      if (b < a.batch) pre[b + 1] = run + v;
+      run += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) pre[0] = 0;
+  }
+  __syncthreads();
+  const int total = pre[a.batch];
+  int item = (int)((int64_t)blockIdx.x * total / gridDim.x);
+  const int item_end = (int)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
   while (item < item_end) {
-    const int bhg = item / a.tiles_per_seq;
-    const int b = bhg / a.HG, hg = bhg % a.HG;
-    const int job_end = min(item_end, (bhg + 1) * a.tiles_per_seq);
-    const int tile_lo = item - bhg * a.tiles_per_seq;
-    const int tile_hi = job_end - bhg * a.tiles_per_seq;
+    // the sequence holding `item`: the last b with pre[b] <= item
+    int lo = 0, hi = a.batch;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pre[mid] <= item) lo = mid;
+      else hi = mid;
+    }
+    const int b = lo;
+    const int n_tiles = (pre[b + 1] - pre[b]) / a.HG;
+    const int rel = item - pre[b];
+    const int hg = rel / n_tiles;
+    const int job_end = min(item_end, pre[b] + (hg + 1) * n_tiles);
+    const int t0 = rel - hg * n_tiles, t1 = t0 + (job_end - item);
     item = job_end;
-    const int Lv = decode_len(a.seq_lens, a.pos0, a.qpos, b, a.max_pages, a.max_position);
-    const bool bad_len = Lv < 0;
-    const int L = bad_len ? 0 : Lv;
+    const int L = decode_len(a.seq_lens, a.pos0, a.qpos, b, a.max_pages, a.max_position);
     const int p0 = a.pos0 ? a.pos0[b] : 0;  // position of the sequence's first cached token
-    const int n_tiles = bad_len ? 0 : (L + kT - 1) / kT;
-    const int t0 = tile_lo, t1 = min(tile_hi, n_tiles);
-    if (t0 >= t1) continue;
     if (*failed) break;
     const int h0 = hg * a.hpc;
     const int kv0 = h0 / a.group;
@@ -1751,14 +1779,18 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   A.tiles_per_seq = t.tiles_per_seq;
   A.tpad = t.tpad;
   A.max_position = f.max_position;
-  A.total_items = batch * t.HG * t.tiles_per_seq;
+  A.batch = batch;
+  // the items that can hold tokens (every sequence at its longest); each CTA
+  // takes total / ctas of the ones that do, which is at most items_per_cta
+  const int max_items = batch * t.HG * t.tiles_per_seq;
   int ctas = sm_count();
-  if (ctas > A.total_items) ctas = A.total_items;
-  A.items_per_cta = (A.total_items + ctas - 1) / ctas;
+  if (ctas > max_items) ctas = max_items;
+  A.items_per_cta = (max_items + ctas - 1) / ctas;
   // a CTA's block-table entries sit in shared memory: beyond this many tiles
   // per CTA the grid grows past one wave instead
   if (A.items_per_cta > kMaxScoreItemsPerCta) A.items_per_cta = kMaxScoreItemsPerCta;
-  ctas = (A.total_items + A.items_per_cta - 1) / A.items_per_cta;
+  ctas = (max_items + A.items_per_cta - 1) / A.items_per_cta;
+  A.items_per_cta = (max_items + ctas - 1) / ctas;
   A.n_pages = cache.n_pages;
   A.q = q;
   A.block_table = block_table;
@@ -1792,7 +1824,7 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
     o += 2 * A.trig_stage;
     // as many key stages as fit (page table, flags, barriers and alignment slack after them)
     const uint32_t tail = (uint32_t)(A.items_per_cta * kPagesPerTile * 4) + kMaxKeyStages * kPagesPerTile * 4 +
-                          (2 * kMaxKeyStages + 16) * 8 + 2 * 4 * kT * 4 + 1024 + 64;
+                          (2 * kMaxKeyStages + 16) * 8 + 2 * 4 * kT * 4 + (uint32_t)(batch + 1) * 4 + 16 + 1024 + 64;
     const uint32_t per_key = A.codes_stage + A.meta_stage;
     int nk = (int)((227u * 1024u - o - tail) / per_key);
     if (nk > kMaxKeyStages) nk = kMaxKeyStages;
@@ -1810,6 +1842,8 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
     o = A.off_bar + (2 * kMaxKeyStages + 16) * 8;
     A.off_red = (o + 15) / 16 * 16;
     o = A.off_red + 2 * 4 * kT * 4;
+    A.off_pre = (o + 15) / 16 * 16;
+    o = A.off_pre + (uint32_t)(batch + 1) * 4;
     const size_t smem = o + 1024;  // alignment slack
     cudaError_t e;
     switch (f.rank_k) {

@@ -63,6 +63,19 @@ def test_llama3_gqa_shapes_small():
     check_attention(got, ref, "llama3 gqa small")
 
 
+def test_llama3_gqa_empty_sequences_between_others():
+    # the score kernel shares out only the tiles that hold tokens: empty
+    # sequences first, between others and last must be skipped, not shift them
+    w = gen.workload(3)
+    lens = [0, 300, 0, 1, 2100, 17, 0]
+    got, ref, st = run_decode(w, lens)
+    assert st == 0
+    check_attention(got, ref, "llama3 gqa with empty sequences")
+    for b, L in enumerate(lens):
+        if L == 0:
+            assert np.all(got[b] == 0)
+
+
 def test_cuda_core_path_longchat_shapes(monkeypatch):
     # the CUDA-core kernels remain the path for shapes the tensor-core kernels do not cover
     monkeypatch.setenv("STARKV_DECODE_PATH", "simt")

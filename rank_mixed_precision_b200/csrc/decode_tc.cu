@@ -78,6 +78,47 @@ __device__ __forceinline__ int decode_len(const int32_t* seq_lens, const int32_t
   }
   return L;
 }
+
+// Value CTAs of sequence b when `slots` CTAs are shared out over the batch in
+// proportion to the sequences' stage counts (ST tokens each): floor shares,
+// at least one for a sequence with tokens, the slots left over to the largest
+// remainders (ties to the lower index), at most `cap` and at most the
+// sequence's stages.  Run by one full warp; every lane returns the count.
+__device__ int value_splits_of(int b, const int32_t* seq_lens, const int32_t* pos0, const int32_t* qpos, int batch,
+                               int max_pages, int max_position, int ST, int slots, int cap) {
+  const int lane = threadIdx.x & 31;
+  auto stages = [&](int i) -> int64_t {
+    const int L = decode_len(seq_lens, pos0, qpos, i, max_pages, max_position);
+    return L > 0 ? (L + ST - 1) / ST : 0;
+  };
+  int64_t tot = 0;
+  for (int i = lane; i < batch; i += 32) tot += stages(i);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  const int64_t sb = stages(b);
+  if (sb == 0 || tot == 0) return 0;
+  int64_t used = 0, ahead = 0;  // floor shares in all; sequences whose remainder ranks before b's
+  const int64_t rb = ((int64_t)slots * sb) % tot;
+  const bool b_floor0 = (int64_t)slots * sb < tot;
+  for (int i = lane; i < batch; i += 32) {
+    const int64_t si = stages(i);
+    if (si == 0) continue;
+    const int64_t q = (int64_t)slots * si / tot, r = ((int64_t)slots * si) % tot;
+    used += q > 0 ? q : 1;
+    if (q > 0 && (r > rb || (r == rb && i < b))) ++ahead;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    used += __shfl_xor_sync(0xffffffffu, used, o);
+    ahead += __shfl_xor_sync(0xffffffffu, ahead, o);
+  }
+  int64_t k = (int64_t)slots * sb / tot;
+  if (k < 1) k = 1;
+  if (!b_floor0 && ahead < (int64_t)slots - used) ++k;
+  if (k > cap) k = cap;
+  if (k > sb) k = sb;
+  return (int)k;
+}
 }  // namespace
 
 // ===========================================================================
@@ -810,6 +851,8 @@ struct ValueArgs {
   float* lpart;  // [B][nclust][H]
   unsigned int* status;
   int CS, nclust;         // CTAs per cluster, clusters per sequence
+  int balanced, batch, slots;  // splits per sequence by length (CS = 1): over `slots` CTAs
+  int* vsplit;            // [B] each sequence's split count (balanced mode), for the projection
   uint32_t off_z, off_p, off_s, off_codes, off_meta, off_flags, off_bt, off_m, off_l, off_bar;
   uint32_t p_stage, s_box, s_box_bytes, s_stage;
   uint32_t codes_page, meta_page, codes_pitch, meta_pitch, codes_stage, meta_stage, tmem_cols;
@@ -871,10 +914,29 @@ __global__ void __launch_bounds__(kVThreads, 1)
   }
   const int seq_stages = (L + ST - 1) / ST;
   const int clust = split / a.CS;
-  // a cluster none of whose splits has tokens leaves as a whole (no partial)
-  if ((int)((int64_t)clust * a.CS * a.stages_total / a.splits) >= seq_stages) return;
-  const int st_lo = (int)((int64_t)split * a.stages_total / a.splits);
-  const int st_hi = min((int)((int64_t)(split + 1) * a.stages_total / a.splits), seq_stages);
+  int st_lo, st_hi;
+  if (a.balanced) {
+    // this sequence's share of the CTAs (CS = 1: a CTA beyond it leaves, no partial)
+    __shared__ int ks_s;
+    if (warp == 0) {
+      const int k = value_splits_of(b, a.seq_lens, a.pos0, a.qpos, a.batch, a.max_pages, a.max_position, ST,
+                                    a.slots, a.splits);
+      if (lane == 0) {
+        ks_s = k;
+        if (split == 0) a.vsplit[b] = k;
+      }
+    }
+    __syncthreads();
+    const int k = ks_s;
+    if (split >= k) return;
+    st_lo = (int)((int64_t)split * seq_stages / k);
+    st_hi = (int)((int64_t)(split + 1) * seq_stages / k);
+  } else {
+    // a cluster none of whose splits has tokens leaves as a whole (no partial)
+    if ((int)((int64_t)clust * a.CS * a.stages_total / a.splits) >= seq_stages) return;
+    st_lo = (int)((int64_t)split * a.stages_total / a.splits);
+    st_hi = min((int)((int64_t)(split + 1) * a.stages_total / a.splits), seq_stages);
+  }
   const int nst = st_hi > st_lo ? st_hi - st_lo : 0;
   const bool work = nst > 0;  // uniform across the CTA
 
@@ -1192,6 +1254,7 @@ struct ProjArgs {
   int H, h_kv, group, d, R;
   int splits, stages_total, st;  // value-kernel splits, stages and tokens per stage
   int cs, nclust;                // splits per cluster, clusters (partials) per sequence
+  const int* vsplit;             // [B] partials per sequence (balanced value splits), or NULL
   const float* part;     // [B][splits][H][R]
   const float* lpart;    // [B][splits][H]
   float* oacc;           // [B][H][d] fp32 sums (zeroed by the score kernel)
@@ -1242,7 +1305,7 @@ __global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, i
       if (L < 0) L = 0;
       const int nst = (L + a.st - 1) / a.st;
       const int nsp = nst > 0 ? min(a.splits, (int)(((int64_t)nst * a.splits - 1) / a.stages_total) + 1) : 0;
-      np = (nsp + a.cs - 1) / a.cs;
+      np = (nsp + a.cs - 1) / a.cs;  // (balanced splits: read after the wait below)
     }
     nparts_s[tid] = np;
   }
@@ -1265,6 +1328,8 @@ __global__ void __launch_bounds__(256) decode_project_kernel(const ProjArgs a, i
   }
   pdl_wait();  // partial sums, l and the zeroed accumulators
   pdl_launch_dependents();
+  // value splits shared out by length: the value kernel recorded each sequence's count
+  if (a.vsplit && tid < kProjM && b0 + tid < batch) nparts_s[tid] = a.vsplit[b0 + tid];
   __syncthreads();
   if (tid < kProjM) {
     const int b = b0 + tid, np = nparts_s[tid];
@@ -1579,9 +1644,10 @@ struct TcLayout {
   int hpc, kvpc, ncols, HG, tiles_per_seq, tpad, splits, stages_total, N, MT;
   int PS, nW, ST;  // value kernel: pages per stage, dequant warps, tokens per stage
   int CS, nclust;  // value kernel: CTAs per cluster (splits reduced on chip), clusters per sequence
+  int balanced, slots;  // value kernel: splits per sequence by length over `slots` CTAs (CS = 1)
   VSmem vs;        // value kernel shared memory
   bool ok;         // a valid value-kernel configuration exists
-  size_t off_S, off_mx, off_acc, off_l, off_w, off_oacc, off_ocnt, w_bytes, ws;
+  size_t off_S, off_mx, off_acc, off_l, off_w, off_oacc, off_ocnt, off_vsplit, w_bytes, ws;
 };
 
 TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
@@ -1624,15 +1690,34 @@ TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
     const double part_unit = 2.0 * f.num_q_heads * f.rank_v * 4.0;
     const int threads = (kVRoleWarps + t.nW) * 32;
     VSmem probe;  // shared memory at the largest split count considered (for the residency query)
-    t.ok = value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, s0, probe);
+    // Value ranks up to 512 (a split's partial at most 64 KiB per head set):
+    // each sequence gets CTAs in proportion to its length, one per SM in all,
+    // and writes one partial per CTA (no cluster sums); the kernel computes the
+    // shares from the sequence lengths.  A CTA may then hold a whole sequence.
+    t.balanced = 0;
+    t.slots = sms;
+    if (f.rank_v <= 512 && bt >= 2) {
+      int cap = 2 * ((sms + bt - 1) / bt);
+      if (cap > t.stages_total) cap = t.stages_total;
+      if (cap < 1) cap = 1;
+      if (value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, 1, t.vs)) {
+        t.ok = true;
+        t.balanced = 1;
+        t.splits = cap;
+        t.CS = 1;
+      }
+    }
+    if (!t.balanced) t.ok = value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, s0, probe);
     while (!t.ok && s0 < t.stages_total) {  // very long contexts: more splits, smaller page tables
       s0 = s0 * 2 < t.stages_total ? s0 * 2 : t.stages_total;
       t.ok = value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, s0, probe);
     }
     double best = -1.0;
-    t.splits = 1;
-    t.CS = 1;
-    for (int cs = 8; cs >= 1 && t.ok; cs >>= 1) {
+    if (!t.balanced) {
+      t.splits = 1;
+      t.CS = 1;
+    }
+    for (int cs = 8; cs >= 1 && t.ok && !t.balanced; cs >>= 1) {
       int sp = (s0 / cs) * cs;
       if (cs > 1 && bt * (sp / cs) > 0) {
         const int resident = value_max_clusters(cs, threads, probe.smem);
@@ -1650,7 +1735,7 @@ TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
     }
     // a split's block-table entries live in shared memory: long contexts need
     // enough splits (in whole clusters) for that table to fit
-    if (t.ok) {
+    if (t.ok && !t.balanced) {
       t.ok = value_smem(c, t.N, t.nW, t.PS, t.ST, t.stages_total, t.splits, t.vs);
       while (!t.ok && t.splits < t.stages_total) {
         t.splits += t.CS;
@@ -1676,6 +1761,8 @@ TcLayout tc_layout(const Ctx& c, int batch, int max_pages) {
   o += al((size_t)batch * f.num_q_heads * f.head_dim * 4);
   t.off_ocnt = o;
   o += al((size_t)f.num_q_heads * ((batch + 15) / 16) * 4);
+  t.off_vsplit = o;
+  o += al((size_t)batch * 4);
   t.ws = o;
   return t;
 }
@@ -1866,6 +1953,10 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   B.ST = t.ST;
   B.CS = t.CS;
   B.nclust = t.nclust;
+  B.balanced = t.balanced;
+  B.batch = batch;
+  B.slots = t.slots;
+  B.vsplit = reinterpret_cast<int*>(w + t.off_vsplit);
   B.max_pages = max_pages;
   B.tpad = t.tpad;
   B.splits = t.splits;
@@ -1931,6 +2022,7 @@ cudaError_t launch_decode_tc(const Ctx& c, const starkv_cache& cache, const __nv
   P.st = t.ST;
   P.cs = t.CS;
   P.nclust = t.nclust;
+  P.vsplit = t.balanced ? reinterpret_cast<const int*>(w + t.off_vsplit) : nullptr;
   P.part = acc;
   P.lpart = lsum;
   P.seq_lens = seq_lens;
